@@ -1,0 +1,155 @@
+/*
+ * zha.h -- C ABI of libzha: tree-indexed sparse decode attention on B200 (sm_100a).
+ *
+ * The method ("Subquadratic Attention with a Hierarchical Tree-Structured
+ * Indexer", abstract): a tree of recursively compressed key summaries is kept
+ * over the KV cache; at decode time each query walks the tree from the top
+ * down and keeps a sparse subset of keys; exact attention then runs over that
+ * subset.  The tree grows in depth as the cache grows.  The tree is static over
+ * token order ("ALHR" news item, technical features: static trees route keys
+ * hierarchically).  This library fixes the open points as follows:
+ *
+ *   leaf i            = mean of keys t in [i*leaf_block, min((i+1)*leaf_block, N))
+ *   node i, level l   = unweighted mean of its existing children
+ *                       j in [b*i, min(b*i+b, n_{l-1}))
+ *   levels            L = smallest L >= 1 with b^L >= n0 = ceil(N / leaf_block);
+ *                       level L holds the single root, level 0 the leaves
+ *   routing           survivors = {root}; for l = L-1 .. 0: score every child c
+ *                       of a survivor by q . S_l[c] (unscaled, fp32), keep the
+ *                       top-min(beam, #candidates) by score, lower index first
+ *                       on equal scores
+ *   attention         softmax(scale * q . K[t]) weighted V over the tokens
+ *                       t < N of the selected leaves (exact, split-KV online
+ *                       softmax with an fp32 combine)
+ *
+ * Conventions for every call:
+ *   - Every pointer named d_* is device memory owned by the caller.  The
+ *     library never allocates device memory (no cudaMalloc anywhere).
+ *   - Layouts are dense row-major:
+ *       K, V  [batch, kv_heads, capacity_tokens, head_dim]  (tree's kv_dtype)
+ *       Q, O  [batch, q_heads, nq, head_dim]
+ *       leaf_idx / leaf_score  [batch, q_heads, nq, beam]
+ *     Query head h reads KV head h / (q_heads / kv_heads).
+ *   - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and return a status.  Argument errors are found on the
+ *     host before any launch (ZHA_ERR_INVALID_ARG, ZHA_ERR_CAPACITY,
+ *     ZHA_ERR_UNSUPPORTED) and leave the tree unchanged.  A failed launch
+ *     returns ZHA_ERR_CUDA.  Problems only the device can see (a leaf index
+ *     out of range, a bounded wait that ran out) are recorded in a device
+ *     error word that zha_tree_check reads.
+ *   - A zha_tree handle is not thread-safe; calls that share a tree must be
+ *     ordered by the caller (same stream, or events).
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ZHA_OK = 0,
+  ZHA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad order of calls  */
+  ZHA_ERR_CAPACITY = 2,    /* seq_len beyond the tree's capacity_tokens              */
+  ZHA_ERR_UNSUPPORTED = 3, /* shape outside what the kernels are built for            */
+  ZHA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed             */
+  ZHA_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (reported by check)       */
+  ZHA_ERR_DEVICE = 6       /* a kernel met invalid data, e.g. a leaf index >= n0      */
+} zha_status;
+
+typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
+
+/* Geometry of one tree set: one tree per (batch, kv head) "unit". */
+typedef struct {
+  int batch;                 /* >= 1                                               */
+  int kv_heads;              /* >= 1; batch * kv_heads <= 65535                    */
+  int head_dim;              /* 64 or 128                                          */
+  int branching;             /* b >= 2                                             */
+  int leaf_block;            /* tokens per leaf >= 1                               */
+  long long capacity_tokens; /* rows allocated per unit in K and V, >= 1          */
+  zha_dtype kv_dtype;        /* storage type of K, V                               */
+} zha_tree_desc;
+
+typedef struct zha_tree zha_tree; /* opaque host handle */
+
+/* Device bytes the caller must provide to zha_tree_init: a 256-byte header
+ * (device error word) followed by the fp32 summaries of every unit, laid out
+ * unit-major, level-contiguous with capacity-sized levels.  0 on a bad desc. */
+size_t zha_tree_workspace_bytes(const zha_tree_desc* desc);
+
+/* Creates a host handle over caller-owned workspace (>= zha_tree_workspace_bytes,
+ * 256-byte aligned).  The tree starts empty (seq_len 0).  Clears the device error
+ * word with a synchronous cudaMemset on the current device.  *out receives the
+ * handle; free it with zha_tree_destroy. */
+zha_status zha_tree_init(const zha_tree_desc* desc, void* d_workspace, size_t workspace_bytes,
+                         zha_tree** out);
+
+/* Frees the host handle only; the workspace stays the caller's. */
+zha_status zha_tree_destroy(zha_tree* tree);
+
+/* Builds every summary from tokens [0, seq_len) of d_K (replacing any previous
+ * state).  seq_len == 0 leaves an empty tree.  ZHA_ERR_CAPACITY if seq_len >
+ * capacity_tokens. */
+zha_status zha_tree_build(zha_tree* tree, const void* d_K, long long seq_len, void* stream);
+
+/* Extends the tree to tokens [0, new_seq_len): the caller has already written
+ * rows [seq_len, new_seq_len) of K.  Recomputes the leaves that received tokens
+ * and all of their ancestors; adds levels when the leaves outgrow b^L.
+ * new_seq_len must be >= the current seq_len (equal: no-op). */
+zha_status zha_tree_append(zha_tree* tree, const void* d_K, long long new_seq_len, void* stream);
+
+/* Top-down beam routing of nq queries per query head.
+ *   d_Q          [batch, q_heads, nq, head_dim] in q_dtype; q_heads % kv_heads == 0
+ *   beam         1 .. 1024, and beam * branching <= 4096
+ *   d_leaf_idx   out [batch, q_heads, nq, beam] int32: selected leaves, ascending,
+ *                -1 after the last one (only when the tree has fewer than beam leaves)
+ *   d_leaf_score out, nullable: q . S_0[leaf] (fp32) beside each index, NaN on padding
+ *   d_trace      out, nullable: [batch, q_heads, nq, L, beam] int32, the nodes kept at
+ *                levels L-1 .. 0 in that order, ascending, -1 padded (L = zha_tree_levels)
+ * The tree must be non-empty.  nq == 0 is a no-op. */
+zha_status zha_route(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                     int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* stream);
+
+/* Device scratch bytes zha_sparse_attn_decode needs for this shape (0 when the
+ * call needs none).  The value depends on the tree geometry, q_heads, nq, beam
+ * and the device's SM count, not on seq_len. */
+size_t zha_attn_scratch_bytes(const zha_tree* tree, int q_heads, int nq, int beam);
+
+/* Exact softmax attention of each query over the tokens t < seq_len of its leaves.
+ *   d_Q, d_leaf_idx  as produced for / by zha_route (indices < 0 are skipped)
+ *   d_K, d_V         the cache the tree was built over
+ *   scale            multiplies q . k before the softmax (e.g. 1/sqrt(head_dim))
+ *   d_O              out [batch, q_heads, nq, head_dim] in o_dtype (bf16: RNE)
+ *   d_scratch        >= zha_attn_scratch_bytes(tree, q_heads, nq, beam) bytes
+ *                    (may be NULL when that is 0); contents need no initialisation
+ * An index >= n0 sets ZHA_ERR_DEVICE in the error word and is skipped. */
+zha_status zha_sparse_attn_decode(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype,
+                                  int q_heads, int nq, const void* d_K, const void* d_V,
+                                  const int* d_leaf_idx, int beam, float scale, void* d_O,
+                                  zha_dtype o_dtype, void* d_scratch, size_t scratch_bytes,
+                                  void* stream);
+
+/* Synchronizes `stream`, then reads and clears the device error word:
+ * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */
+zha_status zha_tree_check(zha_tree* tree, void* stream);
+
+/* Getters.  Levels are numbered from the leaves (0) to the root (zha_tree_levels). */
+long long zha_tree_seq_len(const zha_tree* tree);
+int zha_tree_levels(const zha_tree* tree);                        /* L; 0 when empty   */
+long long zha_tree_level_nodes(const zha_tree* tree, int level);  /* n_level now       */
+long long zha_tree_level_offset(const zha_tree* tree, int level); /* row offset in unit */
+long long zha_tree_unit_rows(const zha_tree* tree);               /* rows per unit      */
+const float* zha_tree_summaries(const zha_tree* tree); /* device: [units, unit_rows, head_dim] */
+/* Kernel launches issued through this handle since zha_tree_init (all calls). */
+long long zha_tree_launch_count(const zha_tree* tree);
+
+const char* zha_status_string(zha_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZHA_H */

@@ -1,0 +1,250 @@
+// Summary pyramid: leaf means over leaf blocks of K, then unweighted means of the
+// existing children, level by level up to the root ("Subquadratic Attention with a
+// Hierarchical Tree-Structured Indexer", abstract: recursively compressed key summaries
+// over the KV cache; the tree deepens as the cache grows).
+//
+// One launch ("pass") computes a first level from its source rows (K tokens for the
+// leaves, or the stored fp32 level below) and up to k further levels above it inside
+// the CTA.  A CTA owns `chunk` consecutive first-level nodes, a multiple of b^k, so the
+// k upper levels of its subtree need no other CTA.  Sums are formed in fp64 and kept in
+// shared memory in fp64 between the levels of a pass; each level is rounded once to
+// fp32 when stored.  Only nodes inside the touched range [lo, hi] of each level are
+// recomputed; the others are read back from the pyramid (append).
+//
+// Memory: the first pass streams K once with 16-byte coalesced loads (a row of
+// head_dim elements is read by LPR consecutive lanes, one node per lane group, 8 rows
+// in flight per lane) and writes each summary row once.
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "zha_internal.h"
+
+namespace zha {
+
+constexpr int kPassThreads = 256;
+constexpr int kMaxPassLevels = 8;  // first level + up to 7 above it in one CTA
+constexpr int kChunkTarget = 16;   // at least this many first-level nodes per CTA
+constexpr int kChunkMaxPow = 32;   // b^k <= 32 bounds the CTA's fp64 shared memory
+
+struct PassArgs {
+  const char* src;                    // unit 0, row 0 of the source level
+  long long src_unit_stride;          // bytes between units
+  long long n_src;                    // rows present at the source level
+  long long blk0;                     // source rows per first-level node
+  int b;
+  int k;                              // levels above the first, inside the CTA
+  int chunk;                          // first-level nodes per CTA (multiple of b^k)
+  float* pyr;                         // unit 0 of the pyramid
+  long long pyr_unit_stride;          // floats between units
+  long long lvl_off[kMaxPassLevels];  // row offset of the pass's level m inside a unit
+  long long lvl_n[kMaxPassLevels];    // nodes at level m
+  long long lo[kMaxPassLevels];       // touched range at level m (inclusive)
+  long long hi[kMaxPassLevels];
+  long long chunk0;                   // chunk index of blockIdx.x == 0
+};
+
+template <typename TIn, int D>
+__global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassArgs a) {
+  constexpr int VEC = Vec16<TIn>::N;  // elements per 16-byte load
+  constexpr int LPR = D / VEC;        // lanes covering one row
+  constexpr int SPW = 32 / LPR;       // node slots per warp
+  constexpr int SLOTS = (kPassThreads / 32) * SPW;
+  constexpr long long ROWB = (long long)D * sizeof(TIn);
+  static_assert(LPR <= 32 && 32 % LPR == 0, "row must split evenly over a warp");
+
+  extern __shared__ double smem_d[];
+  double* bufA = smem_d;                        // [chunk][D]
+  double* bufB = smem_d + (size_t)a.chunk * D;  // [chunk / b][D]
+
+  const int unit = blockIdx.y;
+  const long long chunk = a.chunk0 + blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slot = warp * SPW + lane / LPR;
+  const int col = (lane % LPR) * VEC;
+  const char* src = a.src + (long long)unit * a.src_unit_stride + (long long)col * sizeof(TIn);
+  float* pyr_u = a.pyr + (long long)unit * a.pyr_unit_stride;
+
+  // ---- first level of the pass: one node per lane group
+  const long long base0 = chunk * a.chunk;
+  for (int j = slot; j < a.chunk; j += SLOTS) {
+    const long long i = base0 + j;
+    if (i >= a.lvl_n[0]) break;  // nodes ascend with j
+    float* dst = pyr_u + (a.lvl_off[0] + i) * D + col;
+    double* sm = bufA + (size_t)j * D + col;
+    if (i >= a.lo[0] && i <= a.hi[0]) {
+      const long long r0 = i * a.blk0;
+      const long long r1 = min(r0 + a.blk0, a.n_src);
+      const long long nrows = r1 - r0;
+      const char* p = src + r0 * ROWB;
+      double acc[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
+      long long r = 0;
+      for (; r + 8 <= nrows; r += 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = ldg16(p + (r + u) * ROWB);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float f[VEC];
+          Vec16<TIn>::to_f32(v[u], f);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[e] += (double)f[e];
+        }
+      }
+      for (; r < nrows; ++r) {
+        float f[VEC];
+        Vec16<TIn>::to_f32(ldg16(p + r * ROWB), f);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += (double)f[e];
+      }
+      const double cnt = (double)nrows;
+      float out[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        acc[e] = acc[e] / cnt;
+        out[e] = (float)acc[e];
+        sm[e] = acc[e];
+      }
+#pragma unroll
+      for (int e = 0; e < VEC; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(out[e], out[e + 1], out[e + 2], out[e + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < VEC; e += 4) {
+        const float4 s = *reinterpret_cast<const float4*>(dst + e);
+        sm[e] = s.x;
+        sm[e + 1] = s.y;
+        sm[e + 2] = s.z;
+        sm[e + 3] = s.w;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- upper levels of the pass, fp64 in shared memory (ping-pong A/B)
+  double* cur = bufA;
+  double* nxt = bufB;
+  int child_nodes = a.chunk;  // nodes of level m-1 owned by this CTA
+  for (int m = 1; m <= a.k; ++m) {
+    const int nn = child_nodes / a.b;
+    const long long basem = chunk * nn;   // first node of level m owned by this CTA
+    const long long basec = basem * a.b;  // its first child
+    for (int idx = threadIdx.x; idx < nn * D; idx += kPassThreads) {
+      const int j = idx / D, e = idx - (idx / D) * D;
+      const long long i = basem + j;
+      if (i >= a.lvl_n[m]) continue;
+      double v;
+      float* dst = pyr_u + (a.lvl_off[m] + i) * D + e;
+      if (i >= a.lo[m] && i <= a.hi[m]) {
+        const long long c0 = i * a.b;
+        const long long c1 = min(c0 + (long long)a.b, a.lvl_n[m - 1]);
+        double s = 0.0;
+        for (long long c = c0; c < c1; ++c) s += cur[(size_t)(c - basec) * D + e];
+        v = s / (double)(c1 - c0);
+        *dst = (float)v;
+      } else {
+        v = (double)*dst;
+      }
+      nxt[(size_t)j * D + e] = v;
+    }
+    __syncthreads();
+    double* tmp = cur;
+    cur = nxt;
+    nxt = tmp;
+    child_nodes = nn;
+  }
+}
+
+int levels_for(long long n0, long long b) {
+  if (n0 <= 0) return 0;
+  int L = 1;
+  long long span = b;
+  while (span < n0) {
+    span *= b;
+    ++L;
+  }
+  return L;
+}
+
+namespace {
+
+template <typename TIn, int D>
+cudaError_t launch_pass(const PassArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+  auto kern = pyramid_pass_kernel<TIn, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPassThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+long long ipow(long long b, int k) {
+  long long r = 1;
+  for (int i = 0; i < k; ++i) r *= b;
+  return r;
+}
+
+}  // namespace
+
+cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long lo,
+                           long long hi, cudaStream_t stream, int* launches) {
+  const int D = t->desc.head_dim;
+  const long long b = t->desc.branching;
+  const int L = t->L;
+  int kmax = 0;
+  while (ipow(b, kmax + 1) <= kChunkMaxPow && kmax + 1 < kMaxPassLevels) ++kmax;
+  int count = 0;
+  for (int level = 0; level <= L;) {
+    const int k = std::min(kmax, L - level);
+    const long long bk = ipow(b, k);
+    const long long rep = bk >= kChunkTarget ? 1 : (kChunkTarget + bk - 1) / bk;
+    const long long chunk = bk * rep;
+    const long long span = ipow(b, level);  // leaves under one node of `level`
+    PassArgs a{};
+    a.b = (int)b;
+    a.k = k;
+    a.chunk = (int)chunk;
+    a.pyr = t->pyr;
+    a.pyr_unit_stride = t->unit_rows * D;
+    long long lo_l = lo / span, hi_l = hi / span;
+    for (int m = 0; m <= k; ++m) {
+      const long long sm = ipow(b, m);
+      a.lvl_off[m] = t->off[level + m];
+      a.lvl_n[m] = t->n[level + m];
+      a.lo[m] = lo_l / sm;
+      a.hi[m] = std::min(hi_l / sm, t->n[level + m] - 1);
+    }
+    const bool from_tokens = level == 0;
+    const size_t esz = (from_tokens && t->desc.kv_dtype == ZHA_BF16) ? 2 : 4;
+    if (from_tokens) {
+      a.src = static_cast<const char*>(d_K);
+      a.src_unit_stride = t->desc.capacity_tokens * D * (long long)esz;
+      a.n_src = N;
+      a.blk0 = t->desc.leaf_block;
+    } else {
+      a.src = reinterpret_cast<const char*>(t->pyr + t->off[level - 1] * D);
+      a.src_unit_stride = t->unit_rows * D * 4;
+      a.n_src = t->n[level - 1];
+      a.blk0 = b;
+    }
+    const long long c0 = a.lo[0] / chunk, c1 = a.hi[0] / chunk;
+    a.chunk0 = c0;
+    dim3 grid((unsigned)(c1 - c0 + 1), (unsigned)t->units);
+    const size_t smem = (size_t)(chunk + (k > 0 ? chunk / b : 0)) * D * sizeof(double);
+    cudaError_t e;
+    if (from_tokens && t->desc.kv_dtype == ZHA_BF16)
+      e = D == 128 ? launch_pass<uint16_t, 128>(a, grid, smem, stream)
+                   : launch_pass<uint16_t, 64>(a, grid, smem, stream);
+    else
+      e = D == 128 ? launch_pass<float, 128>(a, grid, smem, stream)
+                   : launch_pass<float, 64>(a, grid, smem, stream);
+    if (e != cudaSuccess) return e;
+    ++count;
+    ++t->launches;
+    level += k + 1;
+  }
+  if (launches) *launches = count;
+  return cudaSuccess;
+}
+
+}  // namespace zha

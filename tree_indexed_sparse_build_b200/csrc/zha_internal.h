@@ -1,0 +1,70 @@
+// Host-side state of a tree set and the launch entry points each kernel file provides.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/zha.h"
+
+namespace zha {
+
+constexpr int kMaxLevels = 48;      // levels 0 .. root; 2^47 leaves is far beyond any capacity
+constexpr size_t kHeaderBytes = 256;
+constexpr int kMaxBeam = 1024;
+constexpr int kMaxCandidates = 4096;  // beam * branching bound for the route kernel
+
+// Bits of the device error word.
+enum : unsigned { kDevErrTimeout = 1u, kDevErrBadLeaf = 2u };
+
+}  // namespace zha
+
+struct zha_tree {
+  zha_tree_desc desc;
+  char* ws;                    // caller's workspace
+  size_t ws_bytes;
+  unsigned* d_err;             // device error word (workspace header)
+  float* pyr;                  // summaries: [units][unit_rows][head_dim] fp32
+  long long units;
+  long long unit_rows;         // rows per unit, all capacity-sized levels
+  int Lcap;                    // levels for a full cache
+  long long ncap[zha::kMaxLevels];  // capacity nodes per level
+  long long off[zha::kMaxLevels];   // row offset of each level inside a unit
+  long long N;                 // tokens currently summarised
+  int L;                       // current levels (root at level L); 0 when empty
+  long long n[zha::kMaxLevels];     // current nodes per level
+  long long launches;          // kernels launched through this handle
+  int sms;                     // SMs of the device the tree was created on
+  int device;
+};
+
+namespace zha {
+
+// Levels above the leaves for n0 leaves: smallest L >= 1 with b^L >= n0 (0 if n0 == 0).
+int levels_for(long long n0, long long b);
+
+// Summary passes (tree_build.cu): recompute leaves [lo, hi] and all their ancestors
+// up to level L, given tokens [0, N) of K.  Returns a cudaError_t.
+cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long lo,
+                           long long hi, cudaStream_t stream, int* launches);
+
+// Route (route.cu).
+cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads,
+                         int nq, int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
+                         cudaStream_t stream);
+
+// Attention (attend.cu).
+struct AttnPlan {
+  int leaves_per_split;
+  int splits;
+  int stage_tokens;
+  int stages;          // smem buffers (1 or 2)
+  size_t smem_bytes;
+  size_t scratch_bytes;
+};
+AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam);
+cudaError_t launch_attention(zha_tree* t, const AttnPlan& plan, const void* d_Q,
+                             zha_dtype q_dtype, int q_heads, int nq, const void* d_K,
+                             const void* d_V, const int* d_leaf_idx, int beam, float scale,
+                             void* d_O, zha_dtype o_dtype, void* d_scratch, cudaStream_t stream);
+
+}  // namespace zha

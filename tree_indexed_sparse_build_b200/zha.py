@@ -1,0 +1,284 @@
+"""Thin ctypes binding of libzha (include/zha.h).
+
+The functions keep the C names and only marshal arguments: torch tensors become
+device pointers, the current torch stream becomes the cudaStream_t.  Every step
+of the computation runs in libzha's CUDA kernels; there is no other code path,
+and importing this module fails loudly when libzha.so has not been built.
+
+``Tree`` bundles a handle with a caller-owned workspace tensor for convenience.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzha.so")
+
+ZHA_OK, ZHA_ERR_INVALID_ARG, ZHA_ERR_CAPACITY, ZHA_ERR_UNSUPPORTED = 0, 1, 2, 3
+ZHA_ERR_CUDA, ZHA_ERR_TIMEOUT, ZHA_ERR_DEVICE = 4, 5, 6
+ZHA_F32, ZHA_BF16 = 0, 1
+
+EXPORTED = [
+    "zha_tree_workspace_bytes", "zha_tree_init", "zha_tree_destroy", "zha_tree_build",
+    "zha_tree_append", "zha_route", "zha_attn_scratch_bytes", "zha_sparse_attn_decode",
+    "zha_tree_check", "zha_tree_seq_len", "zha_tree_levels", "zha_tree_level_nodes",
+    "zha_tree_level_offset", "zha_tree_unit_rows", "zha_tree_summaries", "zha_tree_launch_count",
+    "zha_status_string",
+]
+
+
+class zha_tree_desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("branching", ctypes.c_int), ("leaf_block", ctypes.c_int),
+                ("capacity_tokens", ctypes.c_longlong), ("kv_dtype", ctypes.c_int)]
+
+
+class ZhaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+_P, _I, _LL, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libzha.  Raises if the library is missing (build it first)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libzha.so not built at {LIB_PATH}; run "
+                               "`python -m tree_indexed_sparse_build_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "zha_tree_workspace_bytes": (_SZ, [ctypes.POINTER(zha_tree_desc)]),
+            "zha_tree_init": (_I, [ctypes.POINTER(zha_tree_desc), _P, _SZ, ctypes.POINTER(_P)]),
+            "zha_tree_destroy": (_I, [_P]),
+            "zha_tree_build": (_I, [_P, _P, _LL, _P]),
+            "zha_tree_append": (_I, [_P, _P, _LL, _P]),
+            "zha_route": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]),
+            "zha_attn_scratch_bytes": (_SZ, [_P, _I, _I, _I]),
+            "zha_sparse_attn_decode": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _I, ctypes.c_float,
+                                            _P, _I, _P, _SZ, _P]),
+            "zha_tree_check": (_I, [_P, _P]),
+            "zha_tree_seq_len": (_LL, [_P]),
+            "zha_tree_levels": (_I, [_P]),
+            "zha_tree_level_nodes": (_LL, [_P, _I]),
+            "zha_tree_level_offset": (_LL, [_P, _I]),
+            "zha_tree_unit_rows": (_LL, [_P]),
+            "zha_tree_summaries": (_P, [_P]),
+            "zha_tree_launch_count": (_LL, [_P]),
+            "zha_status_string": (ctypes.c_char_p, [_I]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().zha_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != ZHA_OK:
+        raise ZhaError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libzha takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libzha takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return ZHA_BF16
+    if dt == torch.float32:
+        return ZHA_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+# ---------------------------------------------------------------- C-named wrappers
+
+def zha_tree_workspace_bytes(desc: zha_tree_desc) -> int:
+    return int(lib().zha_tree_workspace_bytes(ctypes.byref(desc)))
+
+
+def zha_tree_init(desc: zha_tree_desc, workspace: torch.Tensor) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().zha_tree_init(ctypes.byref(desc), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), ctypes.byref(h)),
+           "zha_tree_init")
+    return h
+
+
+def zha_tree_destroy(handle) -> None:
+    _check(lib().zha_tree_destroy(handle), "zha_tree_destroy")
+
+
+def zha_tree_build(handle, K: torch.Tensor, seq_len: int, stream=None) -> None:
+    _check(lib().zha_tree_build(handle, _ptr(K), seq_len, _stream(stream)), "zha_tree_build")
+
+
+def zha_tree_append(handle, K: torch.Tensor, new_seq_len: int, stream=None) -> None:
+    _check(lib().zha_tree_append(handle, _ptr(K), new_seq_len, _stream(stream)), "zha_tree_append")
+
+
+def zha_route(handle, Q: torch.Tensor, beam: int, leaf_idx: torch.Tensor,
+              leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
+              stream=None) -> None:
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_route(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(leaf_idx),
+                           _ptr(leaf_score), _ptr(trace), _stream(stream)), "zha_route")
+
+
+def zha_attn_scratch_bytes(handle, q_heads: int, nq: int, beam: int) -> int:
+    return int(lib().zha_attn_scratch_bytes(handle, q_heads, nq, beam))
+
+
+def zha_sparse_attn_decode(handle, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                           leaf_idx: torch.Tensor, beam: int, scale: float, O: torch.Tensor,
+                           scratch: torch.Tensor | None = None, stream=None) -> None:
+    B, Hq, nq, _ = Q.shape
+    nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
+    _check(lib().zha_sparse_attn_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(K),
+                                        _ptr(V), _ptr(leaf_idx), beam, scale, _ptr(O),
+                                        dtype_code(O.dtype), _ptr(scratch), nbytes,
+                                        _stream(stream)), "zha_sparse_attn_decode")
+
+
+def zha_tree_check(handle, stream=None) -> int:
+    return int(lib().zha_tree_check(handle, _stream(stream)))
+
+
+def zha_tree_seq_len(handle) -> int:
+    return int(lib().zha_tree_seq_len(handle))
+
+
+def zha_tree_levels(handle) -> int:
+    return int(lib().zha_tree_levels(handle))
+
+
+def zha_tree_level_nodes(handle, level: int) -> int:
+    return int(lib().zha_tree_level_nodes(handle, level))
+
+
+def zha_tree_level_offset(handle, level: int) -> int:
+    return int(lib().zha_tree_level_offset(handle, level))
+
+
+def zha_tree_unit_rows(handle) -> int:
+    return int(lib().zha_tree_unit_rows(handle))
+
+
+def zha_tree_launch_count(handle) -> int:
+    return int(lib().zha_tree_launch_count(handle))
+
+
+# ---------------------------------------------------------------- convenience owner
+
+class Tree:
+    """A tree set over a [batch, kv_heads, capacity, head_dim] cache, with its workspace."""
+
+    def __init__(self, batch: int, kv_heads: int, head_dim: int, branching: int,
+                 leaf_block: int, capacity: int, kv_dtype: torch.dtype, device="cuda"):
+        self.desc = zha_tree_desc(batch, kv_heads, head_dim, branching, leaf_block, capacity,
+                                  dtype_code(kv_dtype))
+        nbytes = zha_tree_workspace_bytes(self.desc)
+        if nbytes == 0:
+            raise ZhaError(ZHA_ERR_UNSUPPORTED, "zha_tree_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.handle = zha_tree_init(self.desc, self.workspace)
+        self._scratch = None
+
+    def close(self):
+        if self.handle is not None:
+            zha_tree_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def seq_len(self) -> int:
+        return zha_tree_seq_len(self.handle)
+
+    @property
+    def levels(self) -> int:
+        return zha_tree_levels(self.handle)
+
+    @property
+    def launches(self) -> int:
+        return zha_tree_launch_count(self.handle)
+
+    def level_nodes(self, level: int) -> int:
+        return zha_tree_level_nodes(self.handle, level)
+
+    def build(self, K: torch.Tensor, seq_len: int, stream=None):
+        zha_tree_build(self.handle, K, seq_len, stream)
+
+    def append(self, K: torch.Tensor, new_seq_len: int, stream=None):
+        zha_tree_append(self.handle, K, new_seq_len, stream)
+
+    def summaries(self) -> torch.Tensor:
+        """[units, unit_rows, head_dim] fp32 view of the workspace's summaries."""
+        rows = zha_tree_unit_rows(self.handle)
+        units = self.desc.batch * self.desc.kv_heads
+        d = self.desc.head_dim
+        return self.workspace[256:256 + units * rows * d * 4].view(torch.float32).view(units, rows, d)
+
+    def level(self, level: int) -> torch.Tensor:
+        """[units, n_level, head_dim] view of one level's summaries."""
+        off = zha_tree_level_offset(self.handle, level)
+        return self.summaries()[:, off:off + self.level_nodes(level)]
+
+    def route(self, Q: torch.Tensor, beam: int, scores: bool = False, trace: bool = False,
+              stream=None):
+        B, Hq, nq, _ = Q.shape
+        idx = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=Q.device)
+        sc = torch.empty((B, Hq, nq, beam), dtype=torch.float32, device=Q.device) if scores else None
+        tr = (torch.empty((B, Hq, nq, max(self.levels, 1), beam), dtype=torch.int32, device=Q.device)
+              if trace else None)
+        zha_route(self.handle, Q, beam, idx, sc, tr, stream)
+        return idx, sc, tr
+
+    def scratch_for(self, q_heads: int, nq: int, beam: int, device) -> torch.Tensor | None:
+        need = zha_attn_scratch_bytes(self.handle, q_heads, nq, beam)
+        if need == 0:
+            return None
+        if self._scratch is None or self._scratch.numel() < need:
+            self._scratch = torch.empty(need, dtype=torch.uint8, device=device)
+        return self._scratch
+
+    def attend(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, leaf_idx: torch.Tensor,
+               beam: int, scale: float, out_dtype: torch.dtype = torch.bfloat16,
+               O: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        B, Hq, nq, d = Q.shape
+        if O is None:
+            O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
+        scratch = self.scratch_for(Hq, nq, beam, Q.device)
+        zha_sparse_attn_decode(self.handle, Q, K, V, leaf_idx, beam, scale, O, scratch, stream)
+        return O
+
+    def check(self, stream=None) -> int:
+        return zha_tree_check(self.handle, stream)
