@@ -1,0 +1,644 @@
+#!/usr/bin/env python
+"""Benchmark of tree-indexed sparse decode attention on B200.
+
+Default (one GPU): the 128K decode workload -- batch 4, 8 KV heads, 32 query
+heads, d = 128, bf16 cache of 131,072 tokens, b = 16, leaf block 32, beam 16.
+A step is one decode step over the whole batch: append one token to every
+(batch, KV head) tree (ancestor recompression, depth growth on the first
+step), route one query per query head, attend.  Each step is replayed from its
+own CUDA graph with graph-captured events around each call; an L2 flush
+(512 MiB memset) runs between steps, outside the events.  The same JSON line
+also carries the 1M-token throughput figures (64 queries per head) and the
+256K build / append figures.
+
+``--impl reference`` times the fp64 oracle instead (host cores, bounded sample).
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode queries/sec at 128K and 1M ctx; route+attend HBM GB/s vs B200 peak"
+UNIT = "queries/s"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 512 << 20
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def levels_for(n0: int, b: int) -> int:
+    if n0 <= 0:
+        return 0
+    L, span = 1, b
+    while span < n0:
+        span *= b
+        L += 1
+    return L
+
+
+def level_counts(N: int, lb: int, b: int) -> list[int]:
+    n0 = -(-N // lb)
+    L = levels_for(n0, b)
+    out, n = [], n0
+    for _ in range(L + 1):
+        out.append(n)
+        n = -(-n // b)
+    return out
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def path_bytes(idx, trace, counts, N, lb, b, d, kv_bytes, g, out_bytes):
+    """Algorithmic bytes of one route call and one attend call, plus per-query counts.
+
+    Bytes are the union per (batch, KV head) of distinct summary rows scored (fp32) and
+    of distinct leaf-token K/V rows attended, plus Q in, indices and O out.
+    """
+    B, Hq, nq, beam = idx.shape
+    L = trace.shape[3]
+    Hkv = Hq // g
+    route_rows = 0
+    attend_tokens = 0
+    scored = []
+    keys = []
+    ar = np.arange(b)
+    for bb in range(B):
+        for h in range(Hkv):
+            tr = trace[bb, h * g:(h + 1) * g].reshape(-1, L, beam)
+            lv = idx[bb, h * g:(h + 1) * g].reshape(-1, beam)
+            nqq = tr.shape[0]
+            per_q = np.full(nqq, counts[L - 1], np.int64)
+            route_rows += counts[L - 1]
+            for li in range(1, L):
+                l = L - 1 - li
+                s = tr[:, li - 1, :].astype(np.int64)
+                ch = s[:, :, None] * b + ar[None, None, :]
+                ok = (s[:, :, None] >= 0) & (ch < counts[l])
+                per_q += ok.reshape(nqq, -1).sum(axis=1)
+                route_rows += np.unique(ch[ok]).size
+            scored.append(per_q)
+            valid = lv >= 0
+            tok = np.where(valid, np.minimum((lv.astype(np.int64) + 1) * lb, N) - lv.astype(np.int64) * lb, 0)
+            keys.append(tok.sum(axis=1))
+            u = np.unique(lv[valid])
+            attend_tokens += int((np.minimum((u + 1) * lb, N) - u * lb).sum())
+    q = B * Hq * nq
+    route_b = route_rows * d * 4 + q * d * kv_bytes + q * beam * 4
+    attend_b = attend_tokens * 2 * d * kv_bytes + q * d * kv_bytes + q * beam * 4 + q * d * out_bytes
+    return {"route_bytes": int(route_b), "attend_bytes": int(attend_b),
+            "summaries_per_query": float(np.concatenate(scored).mean()),
+            "keys_per_query": float(np.concatenate(keys).mean())}
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples: list[tuple[int, int]] = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                if not uuid.startswith("GPU-"):
+                    uuid = "GPU-" + uuid
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception as e:  # NVML absent: report no clocks rather than fail the bench
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        while not self._stop.is_set():
+            try:
+                mhz = int(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                rs = int(get_reasons(self.h)) if get_reasons else 0
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+                    "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        names = sorted(v for k, v in self.REASONS.items() if bits & k and k != 0x1)
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(mhz)}
+
+
+def kernel_traffic(kernel: str):
+    """dram bytes per launch recorded from an ncu capture, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+        src = os.path.join(ROOT, "tree_indexed_sparse_build_b200", "csrc", rec["source"])
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+                return None
+        return rec["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def _graph_events(n):
+    import torch
+    return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
+
+
+def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
+    """128K decode steps: append 1 token + route + attend, one CUDA graph per step."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, zha
+
+    N, cap = w.seq_len, w.seq_len + W + K
+    w = w.with_(seed=w.seed + 7919 * rank)
+    Qs = np.stack([synth.queries(w, step=s) for s in range(W + K)])
+    Kn = synth.keys(w, capacity=cap)
+    Vn = synth.values(w, capacity=cap)
+    Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qs, dev)
+    B, Hq, nq, d, beam = w.batch, w.q_heads, 1, w.head_dim, w.beam
+    tree = zha.Tree(B, w.kv_heads, d, w.branching, w.leaf_block, cap, torch.bfloat16)
+    tree.build(Kd, N)
+    scratch = tree.scratch_for(Hq, nq, beam, dev)
+    idx = torch.empty((K, B, Hq, nq, beam), dtype=torch.int32, device=dev)
+    O = torch.empty((K, B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
+    Ls = [levels_for(-(-(N + W + s + 1) // w.leaf_block), w.branching) for s in range(K)]
+    traces = [torch.empty((B, Hq, nq, Ls[s], beam), dtype=torch.int32, device=dev) for s in range(K)]
+    Ow = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
+    for s in range(W):
+        tree.append(Kd, N + s + 1)
+        i, _, _ = tree.route(Qd[s], beam)
+        tree.attend(Qd[s], Kd, Vd, i, beam, w.scale, O=Ow)
+    torch.cuda.synchronize()
+
+    def one_step(s, e):
+        st = W + s
+        e[0].record()
+        zha.zha_tree_append(tree.handle, Kd, N + st + 1)
+        e[1].record()
+        zha.zha_route(tree.handle, Qd[st], beam, idx[s], None, traces[s])
+        e[2].record()
+        zha.zha_sparse_attn_decode(tree.handle, Qd[st], Kd, Vd, idx[s], beam, w.scale, O[s], scratch)
+        e[3].record()
+
+    graphs, evs = [], []
+    l0 = tree.launches
+    if eager:  # same launches without graphs (for profilers that cannot replay graph nodes)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+        with sampler_factory() as smp:
+            for s in range(K):
+                flush.zero_()
+                one_step(s, evs[s])
+            torch.cuda.synchronize()
+        launches = (tree.launches - l0) / K
+    else:
+        cap_stream = torch.cuda.Stream()
+        for s in range(K):
+            e = _graph_events(4)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
+                one_step(s, e)
+            graphs.append(g)
+            evs.append(e)
+        launches = (tree.launches - l0) / K
+        torch.cuda.synchronize()
+        with sampler_factory() as smp:
+            for s in range(K):
+                flush.zero_()
+                graphs[s].replay()
+            torch.cuda.synchronize()
+    t_app = np.array([evs[s][0].elapsed_time(evs[s][1]) for s in range(K)])
+    t_rte = np.array([evs[s][1].elapsed_time(evs[s][2]) for s in range(K)])
+    t_att = np.array([evs[s][2].elapsed_time(evs[s][3]) for s in range(K)])
+    t_step = np.array([evs[s][0].elapsed_time(evs[s][3]) for s in range(K)])
+    assert tree.check() == zha.ZHA_OK, "device error word set during the timed steps"
+
+    idx_n, tr_n = idx.cpu().numpy(), [t.cpu().numpy() for t in traces]
+    acc = {"route_bytes": 0, "attend_bytes": 0, "summaries_per_query": 0.0, "keys_per_query": 0.0}
+    for s in range(K):
+        Nst = N + W + s + 1
+        pb = path_bytes(idx_n[s], tr_n[s], level_counts(Nst, w.leaf_block, w.branching), Nst,
+                        w.leaf_block, w.branching, d, 2, w.group, 2)
+        for k in acc:
+            acc[k] += pb[k] / K
+    del graphs
+    res = {"step_ms": t_step, "append_ms": t_app, "route_ms": t_rte, "attend_ms": t_att,
+           "queries_per_step": B * Hq * nq, "launches_per_step": launches, "clocks": smp.summary(),
+           **acc}
+
+    # End to end through the public API: per step, H2D of the new K/V rows and the query
+    # from pinned memory, append + route + attend, D2H of the output, synchronize.
+    tree.build(Kd, N)
+    hk = torch.from_numpy(np.ascontiguousarray(Kn[:, :, N:N + W + K])).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(np.ascontiguousarray(Vn[:, :, N:N + W + K])).view(torch.bfloat16).pin_memory()
+    hq = torch.from_numpy(Qs).view(torch.bfloat16).pin_memory()
+    ho = torch.empty((K, B, Hq, nq, d), dtype=torch.bfloat16).pin_memory()
+    qbuf = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
+    obuf = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
+    ibuf = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=dev)
+
+    def e2e_step(s, out_slot):
+        pos = N + s
+        Kd[:, :, pos].copy_(hk[:, :, s], non_blocking=True)
+        Vd[:, :, pos].copy_(hv[:, :, s], non_blocking=True)
+        qbuf.copy_(hq[s], non_blocking=True)
+        tree.append(Kd, pos + 1)
+        zha.zha_route(tree.handle, qbuf, beam, ibuf)
+        zha.zha_sparse_attn_decode(tree.handle, qbuf, Kd, Vd, ibuf, beam, w.scale, obuf, scratch)
+        if out_slot is not None:
+            ho[out_slot].copy_(obuf, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for s in range(W):
+        e2e_step(s, None)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(K):
+        e2e_step(W + s, s)
+    e1.record()
+    torch.cuda.synchronize()
+    res["e2e_ms_per_step"] = e0.elapsed_time(e1) / K
+    res["h2d_bytes_per_step"] = int(2 * B * w.kv_heads * d * 2 + B * Hq * nq * d * 2)
+    res["d2h_bytes_per_step"] = int(B * Hq * nq * d * 2)
+    # parity spot check of the last e2e output against the graph run is not meaningful
+    # (different steps); correctness is covered by the -m gpu tests.
+    tree.close()
+    return res
+
+
+def run_1m(W, K, rank, dev, flush, eager=False):
+    """1M-token cache, 8 KV heads: route + attend with 64 queries per head (throughput)
+    and with 1 query per head (single step)."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+
+    w = workloads.get("deep_1m")
+    w = w.with_(seed=w.seed + 7919 * rank)
+    nqt = workloads.THROUGHPUT_NQ
+    Qn = synth.queries(w, nq=nqt)
+    Kn = synth.keys(w, Q=Qn)
+    Vn = synth.values(w)
+    Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
+    del Kn, Vn
+    d, beam, N = w.head_dim, w.beam, w.seq_len
+    tree = zha.Tree(w.batch, w.kv_heads, d, w.branching, w.leaf_block, N, torch.bfloat16)
+    tree.build(Kd, N)
+    torch.cuda.synchronize()
+    counts = level_counts(N, w.leaf_block, w.branching)
+    out = {}
+    for mode, nq in (("throughput", nqt), ("single", 1)):
+        Q = Qd[:, :, :nq].contiguous()
+        idx = torch.empty((w.batch, w.q_heads, nq, beam), dtype=torch.int32, device=dev)
+        tr = torch.empty((w.batch, w.q_heads, nq, tree.levels, beam), dtype=torch.int32, device=dev)
+        O = torch.empty((w.batch, w.q_heads, nq, d), dtype=torch.bfloat16, device=dev)
+        scratch = tree.scratch_for(w.q_heads, nq, beam, dev)
+
+        def one_step(e):
+            e[0].record()
+            zha.zha_route(tree.handle, Q, beam, idx, None, tr)
+            e[1].record()
+            zha.zha_sparse_attn_decode(tree.handle, Q, Kd, Vd, idx, beam, w.scale, O, scratch)
+            e[2].record()
+
+        l0 = tree.launches
+        if eager:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            run = lambda: one_step(e)  # noqa: E731
+            run()
+            launches = tree.launches - l0
+        else:
+            e = _graph_events(3)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=torch.cuda.Stream(), capture_error_mode="thread_local"):
+                one_step(e)
+            launches = tree.launches - l0
+            run = g.replay
+        for _ in range(W):
+            run()
+        torch.cuda.synchronize()
+        tr_ms, at_ms = [], []
+        for _ in range(K):
+            flush.zero_()
+            run()
+            torch.cuda.synchronize()
+            tr_ms.append(e[0].elapsed_time(e[1]))
+            at_ms.append(e[1].elapsed_time(e[2]))
+        pb = path_bytes(idx.cpu().numpy(), tr.cpu().numpy(), counts, N, w.leaf_block,
+                        w.branching, d, 2, w.group, 2)
+        out[mode] = {"route_ms": np.array(tr_ms), "attend_ms": np.array(at_ms),
+                     "queries_per_step": w.batch * w.q_heads * nq, "launches_per_step": launches, **pb}
+        del run
+    out["dense_bytes_per_step"] = int(2 * N * d * 2 * w.kv_heads * w.batch)
+    out["levels"] = tree.levels
+    tree.close()
+    return out
+
+
+def run_build_256k(W, K, dev, flush):
+    """256K cache: build from scratch, append 4,096 tokens in one call, route + attend 64
+    queries per head."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+
+    w = workloads.get("build_256k")
+    Qn = synth.queries(w)
+    Kn = synth.keys(w)
+    Vn = synth.values(w)
+    Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
+    del Kn, Vn
+    d, N, cap = w.head_dim, w.seq_len, w.capacity
+    tree = zha.Tree(w.batch, w.kv_heads, d, w.branching, w.leaf_block, cap, torch.bfloat16)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    build_ms, append_ms, ra_ms = [], [], []
+    for it in range(W + max(1, min(K, 10))):
+        flush.zero_()
+        ev[0].record()
+        tree.build(Kd, N)
+        ev[1].record()
+        flush.zero_()
+        ev[2].record()
+        tree.append(Kd, cap)
+        ev[3].record()
+        flush.zero_()
+        ev[4].record()
+        idx, _, _ = tree.route(Qd, w.beam)
+        tree.attend(Qd, Kd, Vd, idx, w.beam, w.scale)
+        ev[5].record()
+        torch.cuda.synchronize()
+        if it >= W:
+            build_ms.append(ev[0].elapsed_time(ev[1]))
+            append_ms.append(ev[2].elapsed_time(ev[3]))
+            ra_ms.append(ev[4].elapsed_time(ev[5]))
+    counts = level_counts(N, w.leaf_block, w.branching)
+    rows = sum(counts)
+    build_bytes = N * d * 2 * w.units + rows * d * 4 * w.units
+    q = w.batch * w.q_heads * w.nq
+    res = {"build_ms": float(np.mean(build_ms)), "build_bytes": int(build_bytes),
+           "build_gbs": build_bytes / (np.mean(build_ms) * 1e-3) / 1e9,
+           "append_4096_ms": float(np.mean(append_ms)), "levels_after_append": tree.levels,
+           "route_attend_ms": float(np.mean(ra_ms)), "queries": q,
+           "qps": q / (np.mean(ra_ms) * 1e-3)}
+    tree.close()
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), warmup: int = 0):
+    """Time the fp64 oracle on decode steps of `w` for a few units (single thread).
+
+    Setup (not timed): each sampled unit's tree over the first N tokens.  Timed: per step
+    and unit, append one token, route the unit's query heads, attend each.
+    """
+    import oracle
+    from tree_indexed_sparse_build_b200 import synth
+
+    N = w.seq_len
+    cap = N + warmup + max_steps
+    units = list(units)
+    Kn = synth.keys(w, capacity=cap, units=units)
+    Vn = synth.values(w, capacity=cap, units=units)
+    trees = {u: oracle.OracleTree(w.head_dim, w.leaf_block, w.branching).build(
+        Kn[u // w.kv_heads, u % w.kv_heads], N) for u in units}
+
+    def step(s):
+        q = synth.queries(w, step=s)
+        n = 0
+        for u in units:
+            b, h = divmod(u, w.kv_heads)
+            t = trees[u]
+            t.append(Kn[b, h], N + s + 1)
+            qs = synth.to_f64(q[b, h * w.group:(h + 1) * w.group, 0])
+            res = t.route(qs, w.beam)
+            for i in range(qs.shape[0]):
+                oracle.attend(qs[i], Kn[b, h], Vn[b, h], N + s + 1, w.leaf_block,
+                              res["leaves"][i], w.scale)
+                n += 1
+        return n
+
+    for s in range(warmup):
+        step(s)
+    t0 = time.perf_counter()
+    nq = steps = 0
+    per_step = []
+    while steps < max_steps and (time.perf_counter() - t0) < seconds:
+        ts = time.perf_counter()
+        nq += step(warmup + steps)
+        per_step.append(time.perf_counter() - ts)
+        steps += 1
+    el = time.perf_counter() - t0
+    return {"value": nq / el, "queries": nq, "seconds": el, "steps": steps, "units": len(units),
+            "per_step_s": per_step}
+
+
+# ----------------------------------------------------------------------------- main
+
+def workload_config(w):
+    return {"workload": f"{w.name}: decode steps (append 1 token, route, attend) over a "
+                        f"{w.seq_len}-token bf16 cache",
+            "batch": w.batch, "kv_heads": w.kv_heads, "q_heads": w.q_heads,
+            "head_dim": w.head_dim, "seq_len": w.seq_len, "branching": w.branching,
+            "leaf_block": w.leaf_block, "beam": w.beam, "nq": 1, "kv_dtype": "bf16",
+            "out_dtype": "bf16",
+            "l2": f"flushed between steps ({FLUSH_BYTES >> 20} MiB memset outside the timed events)",
+            "inputs": "seeded synthetic: K ~ N(0,1) + rank-8 positional drift, V, Q ~ N(0,1)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=61)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-1m", action="store_true")
+    ap.add_argument("--no-build", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the same kernels without CUDA graphs (for profilers)")
+    args = ap.parse_args()
+    K, W = args.steps, args.warmup
+
+    from tree_indexed_sparse_build_b200 import workloads
+    w = workloads.get("decode_128k")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        r = oracle_decode_sample(w, seconds=1e9, max_steps=K, warmup=W, units=(0,))
+        t = float(np.sum(r["per_step_s"]))
+        qps = r["queries"] / t
+        line = {"impl": "reference", "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": K, "warmup": W, "ms_per_step": 1e3 * t / max(r["steps"], 1),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": workload_config(w),
+                "cpu_baseline": {"value": qps, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                 "sample": f"1 (batch, KV head) unit, {r['steps']} decode steps x "
+                                           f"{w.group} query heads, single-threaded fp64 C oracle"},
+                "e2e": {"value": qps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    sampler = lambda: ClockSampler(local)  # noqa: E731
+
+    barrier()
+    torch.cuda.synchronize()
+    r = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager)
+    torch.cuda.synchronize()
+    barrier()
+
+    peak, peak_kind = hbm_peak()
+    step_ms = max_over_ranks(float(r["step_ms"].mean()))
+    qps = r["queries_per_step"] * world / (step_ms * 1e-3)
+    e2e_ms = max_over_ranks(r["e2e_ms_per_step"])
+    kern = {}
+    for name, ms_key, b_key in (("route", "route_ms", "route_bytes"),
+                                ("attend", "attend_ms", "attend_bytes")):
+        ms = float(r[ms_key].mean())
+        kern[name] = {"ms": ms, "bytes": int(r[b_key]), "gbs": r[b_key] / (ms * 1e-3) / 1e9}
+    kern["append"] = {"ms": float(r["append_ms"].mean())}
+    dom = max(("route", "attend"), key=lambda k: kern[k]["ms"])
+    dom_kernel = {"route": "route_tma_kernel", "attend": "attend_kernel"}[dom]
+    ra_bytes = r["route_bytes"] + r["attend_bytes"]
+    ra_ms = float((r["route_ms"] + r["attend_ms"]).mean())
+
+    line = {
+        "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w),
+        "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": kern[dom]["gbs"],
+                     "peak": peak, "unit": "GB/s", "frac": kern[dom]["gbs"] / peak,
+                     "traffic": kernel_traffic(dom_kernel), "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": kern[dom]["bytes"]},
+        "route_attend": {"gbs": ra_bytes / (ra_ms * 1e-3) / 1e9, "frac": ra_bytes / (ra_ms * 1e-3) / 1e9 / peak,
+                         "ms": ra_ms, "bytes": int(ra_bytes)},
+        "kernels": kern,
+        "keys_per_query": r["keys_per_query"], "summaries_per_query": r["summaries_per_query"],
+        "e2e": {"value": r["queries_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": r["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": r["d2h_bytes_per_step"]},
+        "gpu_launches": int(round(r["launches_per_step"] * K)),
+        "launch_mode": "eager" if args.eager else "cuda_graph_per_step",
+        "clocks": r["clocks"],
+    }
+
+    if not args.no_1m:
+        m = run_1m(W, K, rank, dev, flush, eager=args.eager)
+        one = {}
+        for mode in ("throughput", "single"):
+            x = m[mode]
+            ms = float((x["route_ms"] + x["attend_ms"]).mean())
+            ms = max_over_ranks(ms)
+            byts = x["route_bytes"] + x["attend_bytes"]
+            one[mode] = {"qps": x["queries_per_step"] * world / (ms * 1e-3), "ms_per_step": ms,
+                         "route_ms": float(x["route_ms"].mean()), "attend_ms": float(x["attend_ms"].mean()),
+                         "route_attend_gbs": byts / (ms * 1e-3) / 1e9,
+                         "frac_of_peak": byts / (ms * 1e-3) / 1e9 / peak,
+                         "route_gbs": x["route_bytes"] / (x["route_ms"].mean() * 1e-3) / 1e9,
+                         "attend_gbs": x["attend_bytes"] / (x["attend_ms"].mean() * 1e-3) / 1e9,
+                         "bytes_per_step": int(byts), "keys_per_query": x["keys_per_query"],
+                         "summaries_per_query": x["summaries_per_query"],
+                         "queries_per_step": x["queries_per_step"]}
+        one["dense_bytes_per_step"] = m["dense_bytes_per_step"]
+        one["workload"] = ("deep_1m: 1 x 8 KV heads x 64 query heads, d 128, 1,048,576 bf16 tokens, "
+                           "b 8, leaf block 4, beam 8; throughput = 64 queries per head per step")
+        one["launches_per_step"] = {k: m[k]["launches_per_step"] for k in ("throughput", "single")}
+        line["ctx_1m"] = one
+
+    if not args.no_build and rank == 0:
+        line["build_256k"] = run_build_256k(W, K, dev, flush)
+
+    if rank == 0 and world == 1:
+        try:
+            cb = oracle_decode_sample(w, seconds=args.cpu_seconds, max_steps=64,
+                                      units=tuple(range(8)))
+            line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": f"{cb['units']} (batch, KV head) unit(s) x {cb['steps']} "
+                                              f"decode steps x {w.group} query heads of decode_128k, "
+                                              "single-threaded fp64 C oracle"}
+        except Exception as e:  # the baseline must never sink the GPU number
+            line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": f"failed: {e}"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -9,11 +9,7 @@ from tree_indexed_sparse_build_b200.workloads import Workload
 
 
 def torch_of(x: np.ndarray, device):
-    import torch
-    t = torch.from_numpy(np.ascontiguousarray(x))
-    if x.dtype == np.uint16:
-        t = t.view(torch.bfloat16)
-    return t.to(device)
+    return synth.to_torch(x, device)
 
 
 def make_inputs(w: Workload, capacity: int | None = None, nq: int | None = None):

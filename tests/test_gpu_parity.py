@@ -46,6 +46,11 @@ CASES = [
     _wl("bf16_d64_b3", 1, 3, 3, 64, 777, "bf16", 3, 5, 3, 4, 106),
     _wl("f32_d128_b5", 2, 1, 2, 128, 1234, "f32", 5, 7, 6, 3, 107),
     _wl("f32_d64_b2_lb1", 1, 1, 2, 64, 300, "f32", 2, 1, 5, 4, 108),
+    # > 2 queries per SM: one warp per query, several queries per CTA
+    _wl("bf16_d128_narrow", 2, 2, 8, 128, 6000, "bf16", 8, 16, 8, 32, 111),
+    _wl("f32_d64_narrow", 1, 2, 4, 64, 3000, "f32", 4, 8, 5, 80, 113),
+    # widest level (beam * b = 512 rows) too large to stage: register-batched route kernel
+    _wl("bf16_d128_regpath", 1, 1, 2, 128, 20000, "bf16", 8, 4, 64, 2, 112),
 ]
 
 

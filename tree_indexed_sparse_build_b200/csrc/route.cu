@@ -6,15 +6,25 @@
 // scored by q . S_l[c] in fp32, and the top-min(beam, #candidates) are kept, ordered by
 // score descending with the lower node index first on equal scores.
 //
-// GPU mapping: one warp per query.  Candidates are the children of the survivors, kept
-// in ascending node order (survivors ascend, children of a node are contiguous), so
-// candidate k belongs to survivor k / b.  Eight lanes read one 512-byte summary row
-// (d = 128) with 16-byte loads, four rows per warp step and four steps in flight.  A
-// candidate's key packs (order-preserving score bits, inverted node index) into 64 bits,
-// so "greater key" is exactly "ranks first".  The B-th largest key is found by a 64-step
-// binary search on the key bits with a warp-wide count per step (stopping early once
-// exactly B keys remain), and the kept candidates are compacted with a ballot in
-// candidate order, which keeps the survivors ascending without a sort.
+// GPU mapping.  A candidate's key packs (order-preserving score bits, inverted node
+// index) into 64 bits, so "greater key" is exactly "ranks first".  Candidates are the
+// children of the survivors in ascending node order (survivors ascend, the children of
+// a node are contiguous rows), so candidate k belongs to survivor k / b.
+//
+// Main kernel (route_tma_kernel): each level's candidate rows are staged in shared
+// memory by one 1-D bulk copy (non-multicast TMA) per survivor -- its b children are
+// one contiguous run of rows -- all completing on the query's mbarrier, so a level costs
+// one memory round trip whatever its width and holds no registers while in flight.
+// Few queries ("wide"): one query per CTA with up to 16 warps scoring from shared memory.
+// Many queries ("narrow"): several queries per CTA, one warp each, no CTA barriers.
+// Eight lanes score one row (16-byte shared loads, shuffle reduction).  One warp per
+// query then finds the B-th largest key by a binary search on the key bits that starts
+// below the common prefix of the largest and smallest score, with a warp-wide count per
+// step (stopping as soon as exactly B keys remain), and compacts the kept candidates
+// with a ballot in candidate order, which keeps the survivors ascending without a sort.
+//
+// Fallback kernel (route_reg_kernel) for levels too wide to stage in shared memory:
+// the same selection, with candidate rows loaded into registers in batches.
 #include <algorithm>
 
 #include "device_common.cuh"
@@ -22,7 +32,7 @@
 
 namespace zha {
 
-constexpr int kRouteWarps = 4;
+constexpr int kRouteMaxWarps = 16;
 
 struct RouteArgs {
   const void* Q;
@@ -33,12 +43,40 @@ struct RouteArgs {
   long long off[kMaxLevels];
   long long n[kMaxLevels];
   int L, b, beam, cmax;
-  int warp_smem_words;  // 8-byte words of shared memory per warp
+  int wpq, qpc;           // warps per query, queries per CTA
+  int query_smem_words;   // 8-byte words of shared memory per query
   int* leaf_idx;
   float* leaf_score;
   int* trace;
   long long total_queries;
+  unsigned* err;           // device error word (bounded waits)
+  int query_smem_bytes;    // shared memory per query (staged kernel)
 };
+
+constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+
+// Shared-memory layout of one query in the staged kernel.
+struct RouteSmem {
+  size_t rows, keys, surv_a, surv_b, leaf_sc, bar, total;
+};
+__host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam) {
+  RouteSmem s;
+  s.rows = 0;
+  size_t o = (size_t)cmax * D * 4;
+  s.keys = o;
+  o += (size_t)cmax * 8;
+  s.surv_a = o;
+  o += (size_t)beam * 4;
+  s.surv_b = o;
+  o += (size_t)beam * 4;
+  s.leaf_sc = o;
+  o += (size_t)beam * 4;
+  o = (o + 7) / 8 * 8;
+  s.bar = o;
+  o += 8;
+  s.total = (o + 127) / 128 * 128;
+  return s;
+}
 
 __device__ __forceinline__ unsigned long long route_key(float s, int node) {
   s = s + 0.0f;  // -0 -> +0 so equal scores tie exactly
@@ -53,29 +91,100 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
   return __uint_as_float(u);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs a) {
-  constexpr int NJ = D / 32;  // 16-byte chunks per lane per row
-  constexpr int U = 4;        // warp steps (4 rows each) in flight
-  extern __shared__ unsigned long long route_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long qg = (long long)blockIdx.x * kRouteWarps + warp;
-  if (qg >= a.total_queries) return;  // no block-level barrier in this kernel
+// The beam-th largest of keys[0, C) (C > beam; keys distinct).  Binary search on the
+// score word first (cached in registers, one bit per step, warp-wide counts), stopping as
+// soon as exactly `beam` keys are at or above the threshold; only when scores tie at the
+// threshold does it continue on the index word, read from shared memory.
+__device__ unsigned long long kth_largest_key(const unsigned long long* keys, int C, int beam,
+                                              int lane) {
+  constexpr int R = 8;  // score words cached per lane (C <= 256 needs no shared reads)
+  uint32_t hi[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int k = lane + 32 * i;
+    hi[i] = k < C ? (uint32_t)(keys[k] >> 32) : 0u;
+  }
+  // Every key's score word lies in [hmin, hmax]; their common leading bits are fixed.
+  uint32_t lmax = 0u, lmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+    if (lane + 32 * i < C) {
+      lmax = max(lmax, hi[i]);
+      lmin = min(lmin, hi[i]);
+    }
+  for (int k = lane + 32 * R; k < C; k += 32) {
+    const uint32_t h = (uint32_t)(keys[k] >> 32);
+    lmax = max(lmax, h);
+    lmin = min(lmin, h);
+  }
+  const uint32_t hmax = __reduce_max_sync(0xffffffffu, lmax);
+  const uint32_t hmin = __reduce_min_sync(0xffffffffu, lmin);
+  const uint32_t diff = hmax ^ hmin;
+  const int top = diff ? 31 - __clz(diff) : -1;  // highest bit where scores differ
+  // T <= hmin, so count(>= T) == C > beam holds before the first step.
+  uint32_t T = top < 0 ? hmax : (top >= 31 ? 0u : (hmax & ~((2u << top) - 1u)));
+#pragma unroll 1
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    unsigned cnt = 0;
+#pragma unroll
+    for (int i = 0; i < R; ++i) cnt += hi[i] >= cand ? 1u : 0u;
+    for (int k = lane + 32 * R; k < C; k += 32) cnt += (uint32_t)(keys[k] >> 32) >= cand ? 1u : 0u;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= (unsigned)beam) {
+      T = cand;
+      if (cnt == (unsigned)beam) return (unsigned long long)T << 32;
+    }
+  }
+  // Scores tie at T: keep every key with a larger score and the `need` tied keys with
+  // the largest index words (= lowest node indices).
+  unsigned gt = 0;
+#pragma unroll
+  for (int i = 0; i < R; ++i) gt += hi[i] > T ? 1u : 0u;
+  for (int k = lane + 32 * R; k < C; k += 32) gt += (uint32_t)(keys[k] >> 32) > T ? 1u : 0u;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const unsigned need = (unsigned)beam - gt;
+  uint32_t Tl = 0u;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = Tl | (1u << bit);
+    unsigned cnt = 0;
+    for (int k = lane; k < C; k += 32) {
+      const unsigned long long key = keys[k];
+      cnt += ((uint32_t)(key >> 32) == T && (uint32_t)key >= cand) ? 1u : 0u;
+    }
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= need) {
+      Tl = cand;
+      if (cnt == need) break;
+    }
+  }
+  return ((unsigned long long)T << 32) | Tl;
+}
 
-  unsigned long long* keys = route_smem + (size_t)warp * a.warp_smem_words;
+template <int D, int U>
+__global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const RouteArgs a) {
+  constexpr int NJ = D / 32;  // 16-byte chunks per lane per row
+  extern __shared__ unsigned long long route_smem[];
+  __shared__ int s_m[kRouteMaxWarps];  // survivors per query of the CTA
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = warp / a.wpq, wq = warp - qi * a.wpq;
+  const long long qg = (long long)blockIdx.x * a.qpc + qi;
+  const bool valid = qg < a.total_queries;
+
+  unsigned long long* keys = route_smem + (size_t)qi * a.query_smem_words;
   int* surv_a = reinterpret_cast<int*>(keys + a.cmax);
   int* surv_b = surv_a + a.beam;
   float* leaf_sc = reinterpret_cast<float*>(surv_b + a.beam);
 
-  const long long hq_flat = qg / a.nq;  // b * q_heads + h
-  const int h = (int)(hq_flat % a.q_heads);
-  const long long bb = hq_flat / a.q_heads;
-  const long long unit = bb * a.kv_heads + h / a.group;
-  const int l8 = lane & 7, grp = lane >> 3;
-
-  // This lane's slice of q: chunks c = l8 + 8j, dims 4c .. 4c+3.
+  long long unit = 0;
   float q[NJ * 4];
-  {
+  const int l8 = lane & 7, grp = lane >> 3;
+  if (valid) {
+    const long long hq_flat = qg / a.nq;  // b * q_heads + h
+    const int h = (int)(hq_flat % a.q_heads);
+    unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
+    // This lane's slice of q: chunks c = l8 + 8j, dims 4c .. 4c+3.
     const long long qo = qg * D;
 #pragma unroll
     for (int j = 0; j < NJ; ++j)
@@ -86,21 +195,25 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs
                                 : static_cast<const float*>(a.Q)[dim];
       }
   }
+  if (wq == 0 && lane == 0) {
+    surv_a[0] = 0;  // the root
+    s_m[qi] = valid ? 1 : 0;
+  }
+  __syncthreads();
 
   const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
-  if (lane == 0) surv_a[0] = 0;  // the root
-  __syncwarp();
   int* cur = surv_a;
   int* nxt = surv_b;
-  int m = 1;
   for (int l = a.L - 1; l >= 0; --l) {
-    const long long nl = a.n[l];
-    const long long last = cur[m - 1];
-    const int nc_last = (int)min((long long)a.b, nl - (long long)a.b * last);
-    const int C = (m - 1) * a.b + nc_last;
+    const int m = s_m[qi];
+    int C = 0;
+    if (m > 0) {
+      const long long last = cur[m - 1];
+      C = (m - 1) * a.b + (int)min((long long)a.b, a.n[l] - (long long)a.b * last);
+    }
     const float* S = pyr_u + a.off[l] * D;
-
-    for (int k0 = 0; k0 < C; k0 += 4 * U) {
+#pragma unroll 1
+    for (int k0 = wq * 4 * U; k0 < C; k0 += a.wpq * 4 * U) {
       float4 v[U][NJ];
       int node[U];
 #pragma unroll
@@ -133,53 +246,215 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs
         if (l8 == 0 && k < C) keys[k] = route_key(s, node[u]);
       }
     }
-    __syncwarp();
-
-    // Threshold T = the beam-th largest key (0 keeps everything when C <= beam).
-    unsigned long long T = 0ull;
-    if (C > a.beam) {
-      for (int bit = 63; bit >= 0; --bit) {
-        const unsigned long long cand = T | (1ull << bit);
-        unsigned cnt = 0;
-        for (int k = lane; k < C; k += 32) cnt += keys[k] >= cand ? 1u : 0u;
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
-        if (cnt >= (unsigned)a.beam) {
-          T = cand;
-          if (cnt == (unsigned)a.beam) break;
+    __syncthreads();
+    if (wq == 0 && C > 0) {
+      // Threshold = the beam-th largest key (0 keeps everything when C <= beam).
+      const unsigned long long T = C > a.beam ? kth_largest_key(keys, C, a.beam, lane) : 0ull;
+      int base = 0;
+      for (int k0 = 0; k0 < C; k0 += 32) {
+        const int k = k0 + lane;
+        const unsigned long long key = k < C ? keys[k] : 0ull;
+        const bool keep = k < C && key >= T;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+          const int pos = base + __popc(bal & ((1u << lane) - 1u));
+          nxt[pos] = key_node(key);
+          if (l == 0) leaf_sc[pos] = key_score(key);
         }
+        base += __popc(bal);
       }
-    }
-    // Ordered compaction of the kept candidates.
-    int base = 0;
-    for (int k0 = 0; k0 < C; k0 += 32) {
-      const int k = k0 + lane;
-      const unsigned long long key = k < C ? keys[k] : 0ull;
-      const bool keep = k < C && key >= T;
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      if (keep) {
-        const int pos = base + __popc(bal & ((1u << lane) - 1u));
-        nxt[pos] = key_node(key);
-        if (l == 0) leaf_sc[pos] = key_score(key);
+      __syncwarp();
+      if (a.trace) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < base ? nxt[k] : -1;
       }
-      base += __popc(bal);
+      if (lane == 0) s_m[qi] = base;
     }
-    __syncwarp();
-    m = base;
-    if (a.trace) {
-      int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
-      for (int k = lane; k < a.beam; k += 32) tr[k] = k < m ? nxt[k] : -1;
-    }
+    __syncthreads();
     int* tmp = cur;
     cur = nxt;
     nxt = tmp;
   }
-  int* out = a.leaf_idx + qg * a.beam;
-  for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
-  if (a.leaf_score) {
-    float* os = a.leaf_score + qg * a.beam;
-    for (int k = lane; k < a.beam; k += 32) os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
+  if (valid && wq == 0) {
+    const int m = s_m[qi];
+    int* out = a.leaf_idx + qg * a.beam;
+    for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
+    if (a.leaf_score) {
+      float* os = a.leaf_score + qg * a.beam;
+      for (int k = lane; k < a.beam; k += 32)
+        os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
+    }
   }
 }
+
+// Ordered compaction of the keys >= T of keys[0, C) into nxt (node ids; leaf scores when
+// `leaf`).  One warp; returns how many were kept.
+__device__ __forceinline__ int compact_kept(const unsigned long long* keys, int C,
+                                            unsigned long long T, int* nxt, float* leaf_sc,
+                                            bool leaf, int lane) {
+  int base = 0;
+  for (int k0 = 0; k0 < C; k0 += 32) {
+    const int k = k0 + lane;
+    const unsigned long long key = k < C ? keys[k] : 0ull;
+    const bool keep = k < C && key >= T;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = base + __popc(bal & ((1u << lane) - 1u));
+      nxt[pos] = key_node(key);
+      if (leaf) leaf_sc[pos] = key_score(key);
+    }
+    base += __popc(bal);
+  }
+  return base;
+}
+
+// Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq.  Otherwise qpc queries
+// per CTA with one warp each, synchronised only within the warp.
+template <int D, bool WIDE>
+__global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const RouteArgs a) {
+  constexpr int NJ = D / 32;
+  extern __shared__ __align__(128) unsigned char rsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = WIDE ? 0 : warp;
+  const int wq = WIDE ? warp : 0;
+  const int nw = WIDE ? (int)(blockDim.x >> 5) : 1;
+  const long long qg = (long long)blockIdx.x * (WIDE ? 1 : a.qpc) + qi;
+  const bool valid = qg < a.total_queries;
+  const RouteSmem Ls = route_smem_layout(D, a.cmax, a.beam);
+  unsigned char* base = rsm + (size_t)qi * a.query_smem_bytes;
+  float* rows = reinterpret_cast<float*>(base + Ls.rows);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + Ls.keys);
+  int* surv_a = reinterpret_cast<int*>(base + Ls.surv_a);
+  int* surv_b = reinterpret_cast<int*>(base + Ls.surv_b);
+  float* leaf_sc = reinterpret_cast<float*>(base + Ls.leaf_sc);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + Ls.bar);
+  __shared__ int s_m[kRouteMaxWarps];
+
+  long long unit = 0;
+  float q[NJ * 4];
+  const int l8 = lane & 7, grp = lane >> 3;
+  if (valid) {
+    const long long hq_flat = qg / a.nq;
+    const int h = (int)(hq_flat % a.q_heads);
+    unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
+    const long long qo = qg * D;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const long long dim = qo + (l8 + 8 * j) * 4 + e;
+        q[j * 4 + e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[dim])
+                                : static_cast<const float*>(a.Q)[dim];
+      }
+  }
+  if (wq == 0 && lane == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    surv_a[0] = 0;  // the root
+    s_m[qi] = valid ? 1 : 0;
+  }
+  if (WIDE) __syncthreads(); else __syncwarp();
+
+  const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
+  int* cur = surv_a;
+  int* nxt = surv_b;
+  uint32_t parity = 0;
+  for (int l = a.L - 1; l >= 0; --l) {
+    const int m = s_m[qi];
+    int C = 0;
+    if (m > 0) {
+      const long long last = cur[m - 1];
+      C = (m - 1) * a.b + (int)min((long long)a.b, a.n[l] - (long long)a.b * last);
+    }
+    const float* S = pyr_u + a.off[l] * D;
+    if (wq == 0 && C > 0) {
+      // one bulk copy per survivor: its children are consecutive rows
+      if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)C * D * 4);
+      __syncwarp();
+      fence_proxy_async_smem();
+      for (int j = lane; j < m; j += 32) {
+        const long long node0 = (long long)a.b * cur[j];
+        const int nc = (int)min((long long)a.b, a.n[l] - node0);
+        bulk_copy_g2s(rows + (size_t)j * a.b * D, S + node0 * D, (uint32_t)nc * D * 4, bar);
+      }
+    }
+    const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+    const bool failed = WIDE ? (__syncthreads_or(!ok) != 0) : __any_sync(0xffffffffu, !ok);
+    if (failed) {
+      if (wq == 0 && lane == 0 && C > 0)  // let the copies land before the CTA exits
+        mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+      return;  // every thread of the CTA (WIDE) or warp (narrow) leaves here together
+    }
+    if (C > 0) parity ^= 1u;
+    // score: eight lanes per row, rows k = 4 * (wq + nw * i) + grp
+    for (int k0 = 4 * wq; k0 < C; k0 += 4 * nw) {
+      const int k = k0 + grp;
+      float s = 0.f;
+      if (k < C) {
+        const float4* row = reinterpret_cast<const float4*>(rows + (size_t)k * D);
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const float4 v = row[l8 + 8 * j];
+          s = fmaf(q[4 * j + 0], v.x, s);
+          s = fmaf(q[4 * j + 1], v.y, s);
+          s = fmaf(q[4 * j + 2], v.z, s);
+          s = fmaf(q[4 * j + 3], v.w, s);
+        }
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (l8 == 0 && k < C) keys[k] = route_key(s, a.b * cur[k / a.b] + k % a.b);
+    }
+    if (WIDE) __syncthreads(); else __syncwarp();
+    if (wq == 0 && C > 0) {
+      const unsigned long long T = C > a.beam ? kth_largest_key(keys, C, a.beam, lane) : 0ull;
+      const int kept = compact_kept(keys, C, T, nxt, leaf_sc, l == 0, lane);
+      __syncwarp();
+      if (a.trace) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
+      }
+      if (lane == 0) s_m[qi] = kept;
+    }
+    if (WIDE) __syncthreads(); else __syncwarp();
+    int* tmp = cur;
+    cur = nxt;
+    nxt = tmp;
+  }
+  if (valid && wq == 0) {
+    const int m = s_m[qi];
+    int* out = a.leaf_idx + qg * a.beam;
+    for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
+    if (a.leaf_score) {
+      float* os = a.leaf_score + qg * a.beam;
+      for (int k = lane; k < a.beam; k += 32)
+        os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
+    }
+  }
+}
+
+namespace {
+template <int D, bool WIDE>
+cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
+                          cudaStream_t s) {
+  auto kern = route_tma_kernel<D, WIDE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<blocks, threads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int U>
+cudaError_t run_route(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
+                      cudaStream_t s) {
+  auto kern = route_reg_kernel<D, U>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<blocks, threads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+}  // namespace
 
 cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads,
                          int nq, int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
@@ -205,27 +480,59 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   for (int l = 0; l < t->L; ++l)
     cmax = std::max(cmax, std::min(std::min((long long)beam, t->n[l + 1]) * a.b, t->n[l]));
   a.cmax = (int)cmax;
-  // keys (8 B each) + two survivor lists (4 B) + leaf scores (4 B), rounded to 8 B words
-  const long long words = cmax + (3LL * beam * 4 + 7) / 8;
-  a.warp_smem_words = (int)words;
+  a.total_queries = (long long)t->desc.batch * q_heads * nq;
   a.leaf_idx = d_leaf_idx;
   a.leaf_score = d_leaf_score;
   a.trace = d_trace;
-  a.total_queries = (long long)t->desc.batch * q_heads * nq;
-  const size_t smem = (size_t)words * 8 * kRouteWarps;
-  const long long blocks = (a.total_queries + kRouteWarps - 1) / kRouteWarps;
+  a.err = t->d_err;
   cudaError_t e;
-  if (D == 128) {
-    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<128><<<(unsigned)blocks, kRouteWarps * 32, smem, stream>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<64><<<(unsigned)blocks, kRouteWarps * 32, smem, stream>>>(a);
+
+  // Staged kernel when a query's widest level fits in shared memory.
+  const size_t per_query = route_smem_layout(D, (int)cmax, beam).total;
+  constexpr size_t kSmemCap = 200 * 1024;
+  if (per_query <= kSmemCap) {
+    a.query_smem_bytes = (int)per_query;
+    const bool wide = a.total_queries <= 2LL * t->sms;
+    if (wide) {
+      const int wpq = (int)std::max(1LL, std::min<long long>(kRouteMaxWarps, (cmax + 15) / 16));
+      a.wpq = wpq;
+      a.qpc = 1;
+      const unsigned blocks = (unsigned)a.total_queries;
+      e = D == 128 ? run_route_tma<128, true>(a, blocks, 32 * wpq, per_query, stream)
+                   : run_route_tma<64, true>(a, blocks, 32 * wpq, per_query, stream);
+    } else {
+      const int qpc = (int)std::max<size_t>(1, std::min<size_t>(8, (96 * 1024) / per_query));
+      a.wpq = 1;
+      a.qpc = qpc;
+      const unsigned blocks = (unsigned)((a.total_queries + qpc - 1) / qpc);
+      e = D == 128 ? run_route_tma<128, false>(a, blocks, 32 * qpc, per_query * qpc, stream)
+                   : run_route_tma<64, false>(a, blocks, 32 * qpc, per_query * qpc, stream);
+    }
+    ++t->launches;
+    return e;
   }
+
+  // Register kernel.  Warps per query: enough to cover the widest level in one batch, but
+  // no more than the SMs can hold for this many queries.
+  constexpr int kU128 = 2, kU64 = 4;
+  const int rows_per_batch = 4 * (D == 128 ? kU128 : kU64);
+  const long long need = (cmax + rows_per_batch - 1) / rows_per_batch;
+  const long long room = std::max(1LL, (long long)t->sms * 32 / std::max(1LL, a.total_queries));
+  int wpq = (int)std::min<long long>(kRouteMaxWarps, std::min(need, room));
+  wpq = std::max(wpq, 1);
+  const int cta_warps = wpq > 8 ? kRouteMaxWarps : 8;
+  a.wpq = wpq;
+  a.qpc = std::max(1, cta_warps / wpq);
+  // keys (8 B each) + two survivor lists (4 B) + leaf scores (4 B), rounded to 8 B words
+  const long long words = cmax + (3LL * beam * 4 + 7) / 8;
+  a.query_smem_words = (int)words;
+  const size_t smem = (size_t)words * 8 * a.qpc;
+  const int threads = a.qpc * a.wpq * 32;
+  const unsigned blocks = (unsigned)((a.total_queries + a.qpc - 1) / a.qpc);
+  e = D == 128 ? run_route<128, kU128>(a, blocks, threads, smem, stream)
+               : run_route<64, kU64>(a, blocks, threads, smem, stream);
   ++t->launches;
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace zha

@@ -156,6 +156,114 @@ __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassAr
   }
 }
 
+// Small appends in one launch.  One CTA per unit stages, with 1-D bulk copies (TMA) on
+// one mbarrier, everything the touched path needs: the tokens of the touched leaves
+// [lo, hi] (one contiguous run) and, for every level l >= 1, the stored children of the
+// touched nodes (one contiguous run per level).  It then recomputes the leaves in fp64
+// and walks up: a touched node averages its existing children, taking touched children
+// from the fp64 values just computed and the others from the staged rows.  One memory
+// round trip for the whole path.  Used when hi - lo + 1 <= kPathMaxLeaves and the staged
+// rows fit in shared memory.
+constexpr int kPathMaxLeaves = 8;
+constexpr int kPathThreads = 256;
+constexpr size_t kPathSmemCap = 160 * 1024;
+constexpr long long kPathWaitCycles = 2000000000LL;
+
+struct AppendPathArgs {
+  const char* K;               // unit 0, token 0
+  long long k_unit_stride;     // bytes between units
+  long long N, lb;
+  int b, L;
+  float* pyr;
+  long long pyr_unit_stride;   // floats
+  long long off[kMaxLevels];
+  long long n[kMaxLevels];
+  long long lo, hi;            // touched leaves
+  long long sib0[kMaxLevels];  // first staged child row at level l - 1, for l >= 1
+  int sib_rows[kMaxLevels];    // staged child rows for level l
+  int sib_off[kMaxLevels];     // byte offset of those rows in shared memory
+  int tok_rows;                // staged token rows
+  int fp64_off;                // byte offset of the two fp64 node buffers
+  int bar_off;
+  unsigned* err;
+};
+
+template <typename TIn, int D>
+__global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendPathArgs a) {
+  extern __shared__ __align__(128) unsigned char psm[];
+  const int unit = blockIdx.x;
+  const char* Ku = a.K + (long long)unit * a.k_unit_stride;
+  float* pyr_u = a.pyr + (long long)unit * a.pyr_unit_stride;
+  const TIn* tok = reinterpret_cast<const TIn*>(psm);
+  double* cur = reinterpret_cast<double*>(psm + a.fp64_off);
+  double* nxt = cur + kPathMaxLeaves * D;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(psm + a.bar_off);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    uint32_t bytes = (uint32_t)a.tok_rows * D * sizeof(TIn);
+    for (int l = 1; l <= a.L; ++l) bytes += (uint32_t)a.sib_rows[l] * D * 4;
+    mbar_arrive_expect_tx(bar, bytes);
+    const long long r0 = a.lo * a.lb;
+    bulk_copy_g2s(psm, Ku + r0 * D * (long long)sizeof(TIn), (uint32_t)a.tok_rows * D * sizeof(TIn), bar);
+    for (int l = 1; l <= a.L; ++l)
+      if (a.sib_rows[l] > 0)
+        bulk_copy_g2s(psm + a.sib_off[l], pyr_u + (a.off[l - 1] + a.sib0[l]) * D,
+                      (uint32_t)a.sib_rows[l] * D * 4, bar);
+  }
+  __syncthreads();
+  const bool ok = mbar_wait_bounded(bar, 0, a.err, kDevErrTimeout, kPathWaitCycles);
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) mbar_wait_bounded(bar, 0, a.err, kDevErrTimeout, kPathWaitCycles);
+    return;
+  }
+
+  // leaves
+  const int nn = (int)(a.hi - a.lo + 1);
+  for (int idx = threadIdx.x; idx < nn * D; idx += kPathThreads) {
+    const int j = idx / D, e = idx - (idx / D) * D;
+    const long long i = a.lo + j;
+    const long long r0 = i * a.lb, r1 = min(r0 + a.lb, a.N);
+    const long long base = r0 - a.lo * a.lb;
+    double s = 0.0;
+    for (long long r = 0; r < r1 - r0; ++r) {
+      if constexpr (sizeof(TIn) == 2)
+        s += (double)bf16_bits_to_f32(tok[(base + r) * D + e]);
+      else
+        s += (double)tok[(base + r) * D + e];
+    }
+    const double v = s / (double)(r1 - r0);
+    cur[j * D + e] = v;
+    pyr_u[(a.off[0] + i) * D + e] = (float)v;
+  }
+  __syncthreads();
+
+  long long lo = a.lo, hi = a.hi;
+  for (int l = 1; l <= a.L; ++l) {
+    const long long plo = lo / a.b, phi = hi / a.b;
+    const int np = (int)(phi - plo + 1);
+    const float* sib = reinterpret_cast<const float*>(psm + a.sib_off[l]);
+    for (int idx = threadIdx.x; idx < np * D; idx += kPathThreads) {
+      const int j = idx / D, e = idx - (idx / D) * D;
+      const long long i = plo + j;
+      const long long c0 = i * a.b, c1 = min(c0 + (long long)a.b, a.n[l - 1]);
+      double s = 0.0;
+      for (long long c = c0; c < c1; ++c)
+        s += (c >= lo && c <= hi) ? cur[(c - lo) * D + e] : (double)sib[(c - a.sib0[l]) * D + e];
+      const double v = s / (double)(c1 - c0);
+      nxt[j * D + e] = v;
+      pyr_u[(a.off[l] + i) * D + e] = (float)v;
+    }
+    __syncthreads();
+    double* tmp = cur;
+    cur = nxt;
+    nxt = tmp;
+    lo = plo;
+    hi = phi;
+  }
+}
+
 int levels_for(long long n0, long long b) {
   if (n0 <= 0) return 0;
   int L = 1;
@@ -178,6 +286,15 @@ cudaError_t launch_pass(const PassArgs& a, dim3 grid, size_t smem, cudaStream_t 
   return cudaGetLastError();
 }
 
+template <typename TIn, int D>
+cudaError_t launch_path(const AppendPathArgs& a, unsigned grid, size_t smem, cudaStream_t s) {
+  auto kern = append_path_kernel<TIn, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPathThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
 long long ipow(long long b, int k) {
   long long r = 1;
   for (int i = 0; i < k; ++i) r *= b;
@@ -189,6 +306,59 @@ long long ipow(long long b, int k) {
 cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long lo,
                            long long hi, cudaStream_t stream, int* launches) {
   const int D = t->desc.head_dim;
+  if (hi - lo + 1 <= kPathMaxLeaves) {
+    // a few touched leaves (small appends, tiny trees): one launch walks the path to the root
+    AppendPathArgs a{};
+    const bool bf = t->desc.kv_dtype == ZHA_BF16;
+    const int esz = bf ? 2 : 4;
+    a.K = static_cast<const char*>(d_K);
+    a.k_unit_stride = t->desc.capacity_tokens * D * (long long)esz;
+    a.N = N;
+    a.lb = t->desc.leaf_block;
+    a.b = t->desc.branching;
+    a.L = t->L;
+    a.pyr = t->pyr;
+    a.pyr_unit_stride = t->unit_rows * D;
+    for (int l = 0; l <= t->L; ++l) {
+      a.off[l] = t->off[l];
+      a.n[l] = t->n[l];
+    }
+    a.lo = lo;
+    a.hi = hi;
+    a.err = t->d_err;
+    a.tok_rows = (int)(std::min((hi + 1) * a.lb, N) - lo * a.lb);
+    size_t o = (size_t)a.tok_rows * D * esz;
+    long long clo = lo, chi = hi;
+    for (int l = 1; l <= t->L; ++l) {
+      const long long plo = clo / a.b, phi = chi / a.b;
+      const long long r0 = plo * a.b, r1 = std::min((phi + 1) * a.b, t->n[l - 1]);
+      o = (o + 127) / 128 * 128;
+      a.sib0[l] = r0;
+      a.sib_rows[l] = (int)(r1 - r0);
+      a.sib_off[l] = (int)o;
+      o += (size_t)(r1 - r0) * D * 4;
+      clo = plo;
+      chi = phi;
+    }
+    o = (o + 127) / 128 * 128;
+    a.fp64_off = (int)o;
+    o += 2 * (size_t)kPathMaxLeaves * D * sizeof(double);
+    a.bar_off = (int)o;
+    o += 8;
+    if (o <= kPathSmemCap) {
+      const unsigned grid = (unsigned)t->units;
+      cudaError_t e;
+      if (bf)
+        e = D == 128 ? launch_path<uint16_t, 128>(a, grid, o, stream)
+                     : launch_path<uint16_t, 64>(a, grid, o, stream);
+      else
+        e = D == 128 ? launch_path<float, 128>(a, grid, o, stream)
+                     : launch_path<float, 64>(a, grid, o, stream);
+      ++t->launches;
+      if (launches) *launches = 1;
+      return e;
+    }
+  }
   const long long b = t->desc.branching;
   const int L = t->L;
   int kmax = 0;

@@ -227,3 +227,12 @@ def values(w: Workload, capacity: int | None = None, units: list[int] | None = N
     for u in (range(w.units) if units is None else units):
         flat[u] = normal(w.seed, STREAM_V, u << 40, cap * d, w.kv_dtype)
     return out
+
+
+def to_torch(x: np.ndarray, device):
+    """Move a stored array to a torch device; uint16 bf16 bit patterns become torch.bfloat16."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if x.dtype == np.uint16:
+        t = t.view(torch.bfloat16)
+    return t.to(device)
