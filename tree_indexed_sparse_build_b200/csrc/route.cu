@@ -17,11 +17,14 @@
 // one memory round trip whatever its width and holds no registers while in flight.
 // Few queries ("wide"): one query per CTA with up to 16 warps scoring from shared memory.
 // Many queries ("narrow"): several queries per CTA, one warp each, no CTA barriers.
-// Eight lanes score one row (16-byte shared loads, shuffle reduction).  One warp per
-// query then finds the B-th largest key by a binary search on the key bits that starts
-// below the common prefix of the largest and smallest score, with a warp-wide count per
-// step (stopping as soon as exactly B keys remain), and compacts the kept candidates
-// with a ballot in candidate order, which keeps the survivors ascending without a sort.
+// Four lanes score one row from shared memory against q held in registers (each lane a
+// quarter of the dims; the chunk order alternates between neighbouring rows so the two
+// rows of a shared-memory phase use opposite bank halves), two rows per lane in flight.
+// One warp per query then holds the candidate keys in registers, finds the B-th largest
+// by a binary search on the key bits with ballot-based warp counts (starting below the
+// common prefix of the largest and smallest score, stopping as soon as exactly B keys
+// remain), and compacts the kept candidates with ballots in candidate order, which keeps
+// the survivors ascending without a sort.
 //
 // Fallback kernel (route_reg_kernel) for levels too wide to stage in shared memory:
 // the same selection, with candidate rows loaded into registers in batches.
@@ -57,24 +60,28 @@ constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
 // Shared-memory layout of one query in the staged kernel.
 struct RouteSmem {
-  size_t rows, keys, surv_a, surv_b, leaf_sc, bar, total;
+  size_t rows, keys, cand, surv_a, surv_b, leaf_sc, bar, total;
 };
+__host__ __device__ inline size_t route_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam) {
   RouteSmem s;
-  s.rows = 0;
-  size_t o = (size_t)cmax * D * 4;
-  s.keys = o;
+  size_t o = 0;
+  s.rows = o;   // candidate summary rows, fp32 [cmax][D]
+  o += (size_t)cmax * D * 4;
+  s.keys = o;   // candidate keys [cmax]
   o += (size_t)cmax * 8;
+  s.cand = o;   // candidate node ids [cmax]
+  o += (size_t)cmax * 4;
   s.surv_a = o;
   o += (size_t)beam * 4;
   s.surv_b = o;
   o += (size_t)beam * 4;
   s.leaf_sc = o;
   o += (size_t)beam * 4;
-  o = (o + 7) / 8 * 8;
+  o = route_align(o, 8);
   s.bar = o;
   o += 8;
-  s.total = (o + 127) / 128 * 128;
+  s.total = route_align(o, 128);
   return s;
 }
 
@@ -89,6 +96,90 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
   const uint32_t ord = (uint32_t)(k >> 32);
   const uint32_t u = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
   return __uint_as_float(u);
+}
+
+// Threshold T with exactly `beam` of keys[0, C) >= T (C > beam; keys distinct), found by
+// one warp.  kr holds this lane's keys k = lane + 32 i (i < R; 0 past C), keys beyond 32 R
+// are read from shared memory.  Binary search on the score word, one bit per step, with
+// the warp-wide count taken from ballots; it starts below the common prefix of the
+// largest and smallest score word and stops as soon as exactly `beam` keys remain.  If
+// the whole score word ties at the boundary, the same search runs on the index word of
+// the tied keys (larger index word = lower node index = kept first).
+template <int R>
+__device__ unsigned long long select_threshold(const unsigned long long (&kr)[R],
+                                               const unsigned long long* keys, int C, int beam,
+                                               int lane) {
+  uint32_t h[R];
+  uint32_t lmax = 0u, lmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    h[i] = (uint32_t)(kr[i] >> 32);
+    if (lane + 32 * i < C) {
+      lmax = max(lmax, h[i]);
+      lmin = min(lmin, h[i]);
+    }
+  }
+  const bool tail = C > 32 * R;
+  for (int k = lane + 32 * R; k < C; k += 32) {
+    const uint32_t x = (uint32_t)(keys[k] >> 32);
+    lmax = max(lmax, x);
+    lmin = min(lmin, x);
+  }
+  const uint32_t hmax = __reduce_max_sync(0xffffffffu, lmax);
+  const uint32_t hmin = __reduce_min_sync(0xffffffffu, lmin);
+  const uint32_t diff = hmax ^ hmin;
+  const int top = diff ? 31 - __clz(diff) : -1;
+  // T <= hmin, so count(>= T) == C > beam holds before the first step.
+  uint32_t T = top < 0 ? hmax : (top >= 31 ? 0u : (hmax & ~((2u << top) - 1u)));
+#pragma unroll 1
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    unsigned cnt = 0;
+#pragma unroll
+    for (int i = 0; i < R; ++i) cnt += __popc(__ballot_sync(0xffffffffu, h[i] >= cand));
+    if (tail) {
+      unsigned t = 0;
+      for (int k = lane + 32 * R; k < C; k += 32) t += (uint32_t)(keys[k] >> 32) >= cand ? 1u : 0u;
+      cnt += __reduce_add_sync(0xffffffffu, t);
+    }
+    if (cnt >= (unsigned)beam) {
+      T = cand;
+      if (cnt == (unsigned)beam) return (unsigned long long)T << 32;
+    }
+  }
+  // Ties on the score word T: keep every larger score and the `need` tied keys with the
+  // largest index words.
+  unsigned gt = 0;
+#pragma unroll
+  for (int i = 0; i < R; ++i) gt += __popc(__ballot_sync(0xffffffffu, h[i] > T));
+  if (tail) {
+    unsigned t = 0;
+    for (int k = lane + 32 * R; k < C; k += 32) t += (uint32_t)(keys[k] >> 32) > T ? 1u : 0u;
+    gt += __reduce_add_sync(0xffffffffu, t);
+  }
+  const unsigned need = (unsigned)beam - gt;
+  uint32_t Tl = 0u;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = Tl | (1u << bit);
+    unsigned cnt = 0;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      cnt += __popc(__ballot_sync(0xffffffffu, h[i] == T && (uint32_t)kr[i] >= cand && lane + 32 * i < C));
+    if (tail) {
+      unsigned t = 0;
+      for (int k = lane + 32 * R; k < C; k += 32) {
+        const unsigned long long key = keys[k];
+        t += ((uint32_t)(key >> 32) == T && (uint32_t)key >= cand) ? 1u : 0u;
+      }
+      cnt += __reduce_add_sync(0xffffffffu, t);
+    }
+    if (cnt >= need) {
+      Tl = cand;
+      if (cnt == need) break;
+    }
+  }
+  return ((unsigned long long)T << 32) | Tl;
 }
 
 // The beam-th largest of keys[0, C) (C > beam; keys distinct).  Binary search on the
@@ -287,32 +378,13 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
   }
 }
 
-// Ordered compaction of the keys >= T of keys[0, C) into nxt (node ids; leaf scores when
-// `leaf`).  One warp; returns how many were kept.
-__device__ __forceinline__ int compact_kept(const unsigned long long* keys, int C,
-                                            unsigned long long T, int* nxt, float* leaf_sc,
-                                            bool leaf, int lane) {
-  int base = 0;
-  for (int k0 = 0; k0 < C; k0 += 32) {
-    const int k = k0 + lane;
-    const unsigned long long key = k < C ? keys[k] : 0ull;
-    const bool keep = k < C && key >= T;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = base + __popc(bal & ((1u << lane) - 1u));
-      nxt[pos] = key_node(key);
-      if (leaf) leaf_sc[pos] = key_score(key);
-    }
-    base += __popc(bal);
-  }
-  return base;
-}
-
-// Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq.  Otherwise qpc queries
-// per CTA with one warp each, synchronised only within the warp.
+// Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq, the query's warps
+// synchronised by CTA barriers.  Otherwise qpc queries per CTA with one warp each,
+// synchronised only within the warp.
 template <int D, bool WIDE>
 __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const RouteArgs a) {
-  constexpr int NJ = D / 32;
+  constexpr int CPL = D / 16;  // 16-byte chunks of a row per lane (4 lanes per row)
+  constexpr int R = 8;         // candidate keys held per lane in the selecting warp
   extern __shared__ __align__(128) unsigned char rsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = WIDE ? 0 : warp;
@@ -322,45 +394,41 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
   const bool valid = qg < a.total_queries;
   const RouteSmem Ls = route_smem_layout(D, a.cmax, a.beam);
   unsigned char* base = rsm + (size_t)qi * a.query_smem_bytes;
-  float* rows = reinterpret_cast<float*>(base + Ls.rows);
+  const float* rows = reinterpret_cast<const float*>(base + Ls.rows);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + Ls.keys);
+  int* cand = reinterpret_cast<int*>(base + Ls.cand);
   int* surv_a = reinterpret_cast<int*>(base + Ls.surv_a);
   int* surv_b = reinterpret_cast<int*>(base + Ls.surv_b);
   float* leaf_sc = reinterpret_cast<float*>(base + Ls.leaf_sc);
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + Ls.bar);
-  __shared__ int s_m[kRouteMaxWarps];
+
+  auto group_sync = [&]() {
+    if (WIDE) __syncthreads(); else __syncwarp();
+  };
 
   long long unit = 0;
-  float q[NJ * 4];
-  const int l8 = lane & 7, grp = lane >> 3;
   if (valid) {
     const long long hq_flat = qg / a.nq;
     const int h = (int)(hq_flat % a.q_heads);
     unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
-    const long long qo = qg * D;
-#pragma unroll
-    for (int j = 0; j < NJ; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const long long dim = qo + (l8 + 8 * j) * 4 + e;
-        q[j * 4 + e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[dim])
-                                : static_cast<const float*>(a.Q)[dim];
-      }
   }
+  const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
   if (wq == 0 && lane == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
     surv_a[0] = 0;  // the root
-    s_m[qi] = valid ? 1 : 0;
   }
-  if (WIDE) __syncthreads(); else __syncwarp();
+  group_sync();
 
-  const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
+  // Four lanes per row: lane (rg = lane / 4, sub = lane % 4) reads chunks 4 (j ^ par) + sub,
+  // par = rg & 1, so the two rows of a shared-memory phase use opposite bank halves.
+  const int sub = lane & 3, rg = lane >> 2, par = rg & 1;
+  float4 qv[CPL];
   int* cur = surv_a;
   int* nxt = surv_b;
+  int m = valid ? 1 : 0;
   uint32_t parity = 0;
   for (int l = a.L - 1; l >= 0; --l) {
-    const int m = s_m[qi];
     int C = 0;
     if (m > 0) {
       const long long last = cur[m - 1];
@@ -368,14 +436,28 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
     }
     const float* S = pyr_u + a.off[l] * D;
     if (wq == 0 && C > 0) {
-      // one bulk copy per survivor: its children are consecutive rows
+      // one bulk copy per survivor (its children are consecutive rows) + candidate ids
       if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)C * D * 4);
       __syncwarp();
       fence_proxy_async_smem();
       for (int j = lane; j < m; j += 32) {
         const long long node0 = (long long)a.b * cur[j];
         const int nc = (int)min((long long)a.b, a.n[l] - node0);
-        bulk_copy_g2s(rows + (size_t)j * a.b * D, S + node0 * D, (uint32_t)nc * D * 4, bar);
+        bulk_copy_g2s((void*)(rows + (size_t)j * a.b * D), S + node0 * D, (uint32_t)nc * D * 4, bar);
+      }
+      for (int k = lane; k < C; k += 32) cand[k] = a.b * cur[k / a.b] + k % a.b;
+    }
+    if (l == a.L - 1 && valid) {  // load q while the first level is in flight
+      const long long qo = qg * D;
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int c = 4 * (j ^ par) + sub;
+        float f[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          f[e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[qo + 4 * c + e])
+                          : static_cast<const float*>(a.Q)[qo + 4 * c + e];
+        qv[j] = make_float4(f[0], f[1], f[2], f[3]);
       }
     }
     const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
@@ -383,47 +465,85 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
     if (failed) {
       if (wq == 0 && lane == 0 && C > 0)  // let the copies land before the CTA exits
         mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
-      return;  // every thread of the CTA (WIDE) or warp (narrow) leaves here together
+      return;  // the whole group leaves together
     }
+    if (!WIDE) __syncwarp();  // candidate ids written by other lanes
     if (C > 0) parity ^= 1u;
-    // score: eight lanes per row, rows k = 4 * (wq + nw * i) + grp
-    for (int k0 = 4 * wq; k0 < C; k0 += 4 * nw) {
-      const int k = k0 + grp;
-      float s = 0.f;
-      if (k < C) {
-        const float4* row = reinterpret_cast<const float4*>(rows + (size_t)k * D);
+
+    // score: rows r = 8 (wq + nw t) + rg, two rows per lane in flight
+    for (int r0 = 8 * wq; r0 < C; r0 += 16 * nw) {
+      float acc[2][4];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-          const float4 v = row[l8 + 8 * j];
-          s = fmaf(q[4 * j + 0], v.x, s);
-          s = fmaf(q[4 * j + 1], v.y, s);
-          s = fmaf(q[4 * j + 2], v.z, s);
-          s = fmaf(q[4 * j + 3], v.w, s);
+      for (int u = 0; u < 2; ++u) {
+        const int r = r0 + 8 * nw * u + rg;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[u][e] = 0.f;
+        if (r < C) {
+          const float4* row = reinterpret_cast<const float4*>(rows + (size_t)r * D);
+#pragma unroll
+          for (int j = 0; j < CPL; ++j) {
+            const float4 v = row[4 * (j ^ par) + sub];
+            acc[u][0] = fmaf(qv[j].x, v.x, acc[u][0]);
+            acc[u][1] = fmaf(qv[j].y, v.y, acc[u][1]);
+            acc[u][2] = fmaf(qv[j].z, v.z, acc[u][2]);
+            acc[u][3] = fmaf(qv[j].w, v.w, acc[u][3]);
+          }
         }
       }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if (l8 == 0 && k < C) keys[k] = route_key(s, a.b * cur[k / a.b] + k % a.b);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float s = (acc[u][0] + acc[u][1]) + (acc[u][2] + acc[u][3]);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        const int r = r0 + 8 * nw * u + rg;
+        if (sub == 0 && r < C) keys[r] = route_key(s, cand[r]);
+      }
     }
-    if (WIDE) __syncthreads(); else __syncwarp();
+    group_sync();
     if (wq == 0 && C > 0) {
-      const unsigned long long T = C > a.beam ? kth_largest_key(keys, C, a.beam, lane) : 0ull;
-      const int kept = compact_kept(keys, C, T, nxt, leaf_sc, l == 0, lane);
+      unsigned long long kr[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) kr[i] = lane + 32 * i < C ? keys[lane + 32 * i] : 0ull;
+      const unsigned long long T = C > a.beam ? select_threshold<R>(kr, keys, C, a.beam, lane) : 0ull;
+      // ordered compaction of the keys >= T
+      int kept = 0;
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int k = lane + 32 * i;
+        const bool keep = k < C && kr[i] >= T;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+          const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+          nxt[pos] = cand[k];
+          if (l == 0) leaf_sc[pos] = key_score(kr[i]);
+        }
+        kept += __popc(bal);
+      }
+      for (int k0 = 32 * R; k0 < C; k0 += 32) {
+        const int k = k0 + lane;
+        const unsigned long long key = k < C ? keys[k] : 0ull;
+        const bool keep = k < C && key >= T;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+          const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+          nxt[pos] = cand[k];
+          if (l == 0) leaf_sc[pos] = key_score(key);
+        }
+        kept += __popc(bal);
+      }
       __syncwarp();
-      if (a.trace) {
+      if (a.trace && valid) {
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
         for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
       }
-      if (lane == 0) s_m[qi] = kept;
     }
-    if (WIDE) __syncthreads(); else __syncwarp();
+    m = min(C, a.beam);
+    group_sync();
     int* tmp = cur;
     cur = nxt;
     nxt = tmp;
   }
   if (valid && wq == 0) {
-    const int m = s_m[qi];
     int* out = a.leaf_idx + qg * a.beam;
     for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
     if (a.leaf_score) {
@@ -494,7 +614,7 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
     a.query_smem_bytes = (int)per_query;
     const bool wide = a.total_queries <= 2LL * t->sms;
     if (wide) {
-      const int wpq = (int)std::max(1LL, std::min<long long>(kRouteMaxWarps, (cmax + 15) / 16));
+      const int wpq = (int)std::max(1LL, std::min<long long>(kRouteMaxWarps, (cmax + 31) / 32));  // 8 rows per warp step, two steps in flight
       a.wpq = wpq;
       a.qpc = 1;
       const unsigned blocks = (unsigned)a.total_queries;
