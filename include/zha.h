@@ -132,6 +132,26 @@ zha_status zha_sparse_attn_decode(const zha_tree* tree, const void* d_Q, zha_dty
                                   zha_dtype o_dtype, void* d_scratch, size_t scratch_bytes,
                                   void* stream);
 
+/* zha_sparse_attn_decode for callers that cannot allocate device memory -- an operator
+ * hook handed only its input and output pointers, with no workspace, or a code path
+ * where cudaMalloc is off limits because it synchronizes the device or because device
+ * memory belongs to another allocator.  (The source pages have no counterpart: this is
+ * a calling convention of this library.)  Same arguments, results and checks as
+ * zha_sparse_attn_decode minus the scratch pair: the split-KV partials go to a fixed
+ * device array inside this library of zha_noalloc_scratch_capacity() bytes (256 KiB),
+ * which every GPU that loads the library holds until the process exits.  Shapes whose
+ * partials need more return ZHA_ERR_CAPACITY (use zha_sparse_attn_decode for them).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with the tree's device current) and caches it; make that first call before any stream
+ * capture.  No call allocates or frees device memory.  All calls share the one array and
+ * nothing in it needs clearing between calls, so calls whose kernels overlap on the GPU
+ * (other streams, other threads) race on it: order them. */
+zha_status zha_sparse_attn_decode_noalloc(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype,
+                                          int q_heads, int nq, const void* d_K, const void* d_V,
+                                          const int* d_leaf_idx, int beam, float scale, void* d_O,
+                                          zha_dtype o_dtype, void* stream);
+size_t zha_noalloc_scratch_capacity(void);
+
 /* Synchronizes `stream`, then reads and clears the device error word:
  * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */
 zha_status zha_tree_check(zha_tree* tree, void* stream);

@@ -26,7 +26,7 @@ EXPORTED = [
     "zha_tree_append", "zha_route", "zha_attn_scratch_bytes", "zha_sparse_attn_decode",
     "zha_tree_check", "zha_tree_seq_len", "zha_tree_levels", "zha_tree_level_nodes",
     "zha_tree_level_offset", "zha_tree_unit_rows", "zha_tree_summaries", "zha_tree_launch_count",
-    "zha_status_string",
+    "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
 ]
 
 
@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
             "zha_attn_scratch_bytes": (_SZ, [_P, _I, _I, _I]),
             "zha_sparse_attn_decode": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _I, ctypes.c_float,
                                             _P, _I, _P, _SZ, _P]),
+            "zha_sparse_attn_decode_noalloc": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _I,
+                                                    ctypes.c_float, _P, _I, _P]),
+            "zha_noalloc_scratch_capacity": (_SZ, []),
             "zha_tree_check": (_I, [_P, _P]),
             "zha_tree_seq_len": (_LL, [_P]),
             "zha_tree_levels": (_I, [_P]),
@@ -162,6 +165,21 @@ def zha_sparse_attn_decode(handle, Q: torch.Tensor, K: torch.Tensor, V: torch.Te
                                         _ptr(V), _ptr(leaf_idx), beam, scale, _ptr(O),
                                         dtype_code(O.dtype), _ptr(scratch), nbytes,
                                         _stream(stream)), "zha_sparse_attn_decode")
+
+
+def zha_sparse_attn_decode_noalloc(handle, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                                   leaf_idx: torch.Tensor, beam: int, scale: float,
+                                   O: torch.Tensor, stream=None) -> None:
+    """zha_sparse_attn_decode with the library's own fixed scratch (no caller buffer)."""
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_sparse_attn_decode_noalloc(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq,
+                                                _ptr(K), _ptr(V), _ptr(leaf_idx), beam, scale,
+                                                _ptr(O), dtype_code(O.dtype), _stream(stream)),
+           "zha_sparse_attn_decode_noalloc")
+
+
+def zha_noalloc_scratch_capacity() -> int:
+    return int(lib().zha_noalloc_scratch_capacity())
 
 
 def zha_tree_check(handle, stream=None) -> int:
