@@ -178,7 +178,7 @@ class ClockSampler:
 
 def kernel_traffic(kernel: str):
     """dram bytes per launch recorded from an ncu capture, if the kernel source is unchanged."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
             rec = json.load(f).get(kernel)
