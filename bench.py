@@ -199,13 +199,19 @@ def _graph_events(n):
 
 
 def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
-    """128K decode steps: append 1 token + route + attend, one CUDA graph per step."""
+    """128K decode steps: append 1 token + route + attend, one CUDA graph per step.
+
+    Timed pass (the bench value): steps W .. W+K-1, each graph bracketed by a start and an
+    end event only.  Kernel pass (per-call times for the roofline): steps W+K .. W+2K-1
+    with events between the calls as well (extra graph nodes between the kernels cost a
+    few microseconds, which is why they stay out of the timed pass).
+    """
     import torch
     from tree_indexed_sparse_build_b200 import synth, zha
 
-    N, cap = w.seq_len, w.seq_len + W + K
+    N, cap = w.seq_len, w.seq_len + W + 2 * K
     w = w.with_(seed=w.seed + 7919 * rank)
-    Qs = np.stack([synth.queries(w, step=s) for s in range(W + K)])
+    Qs = np.stack([synth.queries(w, step=s) for s in range(W + 2 * K)])
     Kn = synth.keys(w, capacity=cap)
     Vn = synth.values(w, capacity=cap)
     Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qs, dev)
@@ -213,10 +219,11 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
     tree = zha.Tree(B, w.kv_heads, d, w.branching, w.leaf_block, cap, torch.bfloat16)
     tree.build(Kd, N)
     scratch = tree.scratch_for(Hq, nq, beam, dev)
-    idx = torch.empty((K, B, Hq, nq, beam), dtype=torch.int32, device=dev)
-    O = torch.empty((K, B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
-    Ls = [levels_for(-(-(N + W + s + 1) // w.leaf_block), w.branching) for s in range(K)]
-    traces = [torch.empty((B, Hq, nq, Ls[s], beam), dtype=torch.int32, device=dev) for s in range(K)]
+    idx = torch.empty((2 * K, B, Hq, nq, beam), dtype=torch.int32, device=dev)
+    O = torch.empty((2 * K, B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
+    Ls = [levels_for(-(-(N + W + s + 1) // w.leaf_block), w.branching) for s in range(2 * K)]
+    traces = [torch.empty((B, Hq, nq, Ls[s], beam), dtype=torch.int32, device=dev)
+              for s in range(2 * K)]
     Ow = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
     for s in range(W):
         tree.append(Kd, N + s + 1)
@@ -225,56 +232,86 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
     torch.cuda.synchronize()
 
     def one_step(s, e):
+        """Step W+s; e = [start, end] or [start, after append, after route, end]."""
         st = W + s
         e[0].record()
         zha.zha_tree_append(tree.handle, Kd, N + st + 1)
-        e[1].record()
+        if len(e) == 4:
+            e[1].record()
         zha.zha_route(tree.handle, Qd[st], beam, idx[s], None, traces[s])
-        e[2].record()
+        if len(e) == 4:
+            e[2].record()
         zha.zha_sparse_attn_decode(tree.handle, Qd[st], Kd, Vd, idx[s], beam, w.scale, O[s], scratch)
-        e[3].record()
+        e[-1].record()
 
-    graphs, evs = [], []
+    def make(nev):
+        if eager:  # same launches without graphs (for profilers that cannot replay graph nodes)
+            return [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+        return _graph_events(nev)
+
+    # timed pass
     l0 = tree.launches
-    if eager:  # same launches without graphs (for profilers that cannot replay graph nodes)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    outer, graphs = [], []
+    cap_stream = torch.cuda.Stream()
+    if eager:
+        outer = [make(2) for _ in range(K)]
         with sampler_factory() as smp:
             for s in range(K):
                 flush.zero_()
-                one_step(s, evs[s])
+                one_step(s, outer[s])
             torch.cuda.synchronize()
-        launches = (tree.launches - l0) / K
     else:
-        cap_stream = torch.cuda.Stream()
         for s in range(K):
-            e = _graph_events(4)
+            e = make(2)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
                 one_step(s, e)
             graphs.append(g)
-            evs.append(e)
-        launches = (tree.launches - l0) / K
+            outer.append(e)
         torch.cuda.synchronize()
         with sampler_factory() as smp:
             for s in range(K):
                 flush.zero_()
                 graphs[s].replay()
             torch.cuda.synchronize()
-    t_app = np.array([evs[s][0].elapsed_time(evs[s][1]) for s in range(K)])
-    t_rte = np.array([evs[s][1].elapsed_time(evs[s][2]) for s in range(K)])
-    t_att = np.array([evs[s][2].elapsed_time(evs[s][3]) for s in range(K)])
-    t_step = np.array([evs[s][0].elapsed_time(evs[s][3]) for s in range(K)])
+    launches = (tree.launches - l0) / K
+    t_step = np.array([outer[s][0].elapsed_time(outer[s][1]) for s in range(K)])
+
+    # kernel pass
+    inner, graphs2 = [], []
+    if eager:
+        inner = [make(4) for _ in range(K)]
+        for s in range(K):
+            flush.zero_()
+            one_step(K + s, inner[s])
+        torch.cuda.synchronize()
+    else:
+        for s in range(K):
+            e = make(4)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
+                one_step(K + s, e)
+            graphs2.append(g)
+            inner.append(e)
+        torch.cuda.synchronize()
+        for s in range(K):
+            flush.zero_()
+            graphs2[s].replay()
+        torch.cuda.synchronize()
+    t_app = np.array([inner[s][0].elapsed_time(inner[s][1]) for s in range(K)])
+    t_rte = np.array([inner[s][1].elapsed_time(inner[s][2]) for s in range(K)])
+    t_att = np.array([inner[s][2].elapsed_time(inner[s][3]) for s in range(K)])
     assert tree.check() == zha.ZHA_OK, "device error word set during the timed steps"
 
     idx_n, tr_n = idx.cpu().numpy(), [t.cpu().numpy() for t in traces]
     acc = {"route_bytes": 0, "attend_bytes": 0, "summaries_per_query": 0.0, "keys_per_query": 0.0}
-    for s in range(K):
+    for s in range(K, 2 * K):  # the kernel pass's calls, whose times the roofline uses
         Nst = N + W + s + 1
         pb = path_bytes(idx_n[s], tr_n[s], level_counts(Nst, w.leaf_block, w.branching), Nst,
                         w.leaf_block, w.branching, d, 2, w.group, 2)
         for k in acc:
             acc[k] += pb[k] / K
-    del graphs
+    del graphs, graphs2
     res = {"step_ms": t_step, "append_ms": t_app, "route_ms": t_rte, "attend_ms": t_att,
            "queries_per_step": B * Hq * nq, "launches_per_step": launches, "clocks": smp.summary(),
            **acc}
@@ -347,40 +384,47 @@ def run_1m(W, K, rank, dev, flush, eager=False):
         scratch = tree.scratch_for(w.q_heads, nq, beam, dev)
 
         def one_step(e):
+            """route + attend; e = [start, end] or [start, after route, end]."""
             e[0].record()
             zha.zha_route(tree.handle, Q, beam, idx, None, tr)
-            e[1].record()
+            if len(e) == 3:
+                e[1].record()
             zha.zha_sparse_attn_decode(tree.handle, Q, Kd, Vd, idx, beam, w.scale, O, scratch)
-            e[2].record()
+            e[-1].record()
 
+        runs = {}
         l0 = tree.launches
-        if eager:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-            run = lambda: one_step(e)  # noqa: E731
-            run()
-            launches = tree.launches - l0
-        else:
-            e = _graph_events(3)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=torch.cuda.Stream(), capture_error_mode="thread_local"):
-                one_step(e)
-            launches = tree.launches - l0
-            run = g.replay
-        for _ in range(W):
-            run()
-        torch.cuda.synchronize()
-        tr_ms, at_ms = [], []
-        for _ in range(K):
-            flush.zero_()
-            run()
+        for nev in (2, 3):  # timed (start/end only), then per-call times
+            if eager:
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+                runs[nev] = (e, (lambda e=e: one_step(e)))
+            else:
+                e = _graph_events(nev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=torch.cuda.Stream(), capture_error_mode="thread_local"):
+                    one_step(e)
+                runs[nev] = (e, g.replay, g)
+        launches = (tree.launches - l0) // 2
+        times = {}
+        for nev in (2, 3):
+            e, run = runs[nev][0], runs[nev][1]
+            for _ in range(W):
+                run()
             torch.cuda.synchronize()
-            tr_ms.append(e[0].elapsed_time(e[1]))
-            at_ms.append(e[1].elapsed_time(e[2]))
+            rows = []
+            for _ in range(K):
+                flush.zero_()
+                run()
+                torch.cuda.synchronize()
+                rows.append([e[i].elapsed_time(e[i + 1]) for i in range(nev - 1)])
+            times[nev] = np.array(rows)
+        tr_ms, at_ms = times[3][:, 0], times[3][:, 1]
+        step_ms = times[2][:, 0]
         pb = path_bytes(idx.cpu().numpy(), tr.cpu().numpy(), counts, N, w.leaf_block,
                         w.branching, d, 2, w.group, 2)
-        out[mode] = {"route_ms": np.array(tr_ms), "attend_ms": np.array(at_ms),
+        out[mode] = {"route_ms": tr_ms, "attend_ms": at_ms, "step_ms": step_ms,
                      "queries_per_step": w.batch * w.q_heads * nq, "launches_per_step": launches, **pb}
-        del run
+        del runs
     out["dense_bytes_per_step"] = int(2 * N * d * 2 * w.kv_heads * w.batch)
     out["levels"] = tree.levels
     tree.close()
@@ -602,8 +646,7 @@ def main():
         one = {}
         for mode in ("throughput", "single"):
             x = m[mode]
-            ms = float((x["route_ms"] + x["attend_ms"]).mean())
-            ms = max_over_ranks(ms)
+            ms = max_over_ranks(float(x["step_ms"].mean()))
             byts = x["route_bytes"] + x["attend_bytes"]
             one[mode] = {"qps": x["queries_per_step"] * world / (ms * 1e-3), "ms_per_step": ms,
                          "route_ms": float(x["route_ms"].mean()), "attend_ms": float(x["attend_ms"].mean()),

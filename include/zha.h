@@ -138,7 +138,7 @@ zha_status zha_sparse_attn_decode(const zha_tree* tree, const void* d_Q, zha_dty
  * memory belongs to another allocator.  (The source pages have no counterpart: this is
  * a calling convention of this library.)  Same arguments, results and checks as
  * zha_sparse_attn_decode minus the scratch pair: the split-KV partials go to a fixed
- * device array inside this library of zha_noalloc_scratch_capacity() bytes (256 KiB),
+ * device array inside this library of zha_noalloc_scratch_capacity() bytes (128 KiB),
  * which every GPU that loads the library holds until the process exits.  Shapes whose
  * partials need more return ZHA_ERR_CAPACITY (use zha_sparse_attn_decode for them).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,

@@ -78,7 +78,7 @@ def test_calls_reject_null_tree_on_host():
     assert lib.zha_tree_check(None, None) == zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_tree_levels(None) == -1
     assert lib.zha_attn_scratch_bytes(None, 8, 1, 4) == 0
-    assert lib.zha_noalloc_scratch_capacity() == 256 * 1024
+    assert lib.zha_noalloc_scratch_capacity() == 128 * 1024
 
 
 def test_init_rejects_bad_workspace_without_touching_the_device():

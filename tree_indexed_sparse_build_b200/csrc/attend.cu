@@ -8,25 +8,37 @@
 // GPU mapping: one CTA per (query, split), where a split is a contiguous run of the
 // query's beam slots.  A leaf's K rows (and V rows) are contiguous in memory, so each
 // leaf piece of a stage is fetched with one 1-D bulk copy (non-multicast TMA) into a
-// shared-memory stage, completing on an mbarrier; two stages alternate so the next
-// copy overlaps this stage's arithmetic.  Each thread scores whole tokens from shared
-// memory (16-byte chunks visited in a per-row rotated order, which keeps the eight
-// lanes of a shared-memory phase on distinct banks), the block keeps a running max and
-// sum in the log2 domain, and each lane accumulates head_dim/32 output dims over a
-// quarter of the tokens.  A split writes (acc, m, l) partials to caller scratch and a
-// second kernel combines them; a single split writes O directly.
+// shared-memory stage, completing on an mbarrier; the lanes of warp 0 issue the copies
+// of a stage in parallel.  Splits are sized so a split is usually a single stage; when a
+// split spans several stages, two stage buffers alternate so the next copy overlaps this
+// stage's arithmetic.  Four lanes score a token against q held in registers (neighbouring
+// tokens read their chunks in opposite orders, so the two tokens of a shared-memory phase
+// hit opposite bank halves).  Each warp keeps its own online softmax (running max and sum
+// in the log2 domain) over the tokens it owns; each lane accumulates head_dim/32 output
+// dims; the four warps merge at the end.
+//
+// Splits of one query are merged in one of two ways:
+//  - cluster path (at most 8 splits): the splits of a query form one thread-block cluster
+//    and send their (acc, max, sum) to the rank-0 CTA's shared memory (distributed shared
+//    memory); rank 0 merges and writes O.  No scratch, no second kernel.
+//  - scratch path (more splits): partials go to caller scratch and combine_kernel merges.
 //
 // Every wait on an mbarrier is bounded by a clock budget; on expiry the kernel records
 // kDevErrTimeout in the device error word and stops using the stage (no trap).
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "device_common.cuh"
 #include "zha_internal.h"
 
+namespace cg = cooperative_groups;
+
 namespace zha {
 
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = kAttnThreads / 32;
+constexpr int kMaxClusterSplits = 8;
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
 struct AttnArgs {
@@ -42,22 +54,20 @@ struct AttnArgs {
   int lps, splits, stage_tokens, nbuf;
   void* O;
   int o_bf16;
-  float* partial;  // [queries][splits][D + 2]
+  float* partial;  // scratch path: [queries][splits][D + 2]
   unsigned* err;
   long long total_items;
 };
 
 // Shared-memory layout, identical on host and device.
 struct AttnSmem {
-  size_t qs, red, meta, lids, lpos, sc, accr, kv, total;
+  size_t red, meta, lids, lpos, pw, accr, part, kv, total;
 };
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline AttnSmem attn_smem_layout(int D, int row_bytes, int lps, int stage_tokens,
-                                                     int nbuf) {
+                                                     int nbuf, bool cluster) {
   AttnSmem s;
   size_t o = 16;  // two mbarriers
-  s.qs = o;
-  o += (size_t)D * 4;
   s.red = o;
   o += 8 * 4;
   s.meta = o;
@@ -66,10 +76,12 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int D, int row_bytes, int l
   o += (size_t)lps * 4;
   s.lpos = o;
   o += (size_t)(lps + 1) * 4;
-  s.sc = align_up(o, 16);
-  o = s.sc + (size_t)stage_tokens * 4;
+  s.pw = align_up(o, 16);  // per-warp softmax weights of one round [warps][16]
+  o = s.pw + (size_t)kAttnWarps * 16 * 4;
   s.accr = align_up(o, 16);
   o = s.accr + (size_t)kAttnWarps * D * 4;
+  s.part = align_up(o, 16);  // cluster path, rank 0: the splits' partials [8][D + 2]
+  o = s.part + (cluster ? (size_t)kMaxClusterSplits * (D + 2) * 4 : 0);
   s.kv = align_up(o, 128);
   s.total = s.kv + (size_t)nbuf * 2 * stage_tokens * row_bytes;
   return s;
@@ -105,16 +117,19 @@ __device__ __forceinline__ void load_v(const float* p, float* o) {
 }
 
 // Issue the bulk copies of stage `s` (tokens [s*TS, s*TS + TS) of the work item's token
-// sequence) into buffer `buf`.  Called by one thread.
+// sequence) into buffers kbuf/vbuf.  Called by all lanes of one warp: lane 0 registers the
+// stage's byte count on the barrier, then each lane copies the pieces of its leaves.
 template <int ROWB>
 __device__ void issue_stage(const AttnArgs& a, const char* Ku, const char* Vu, const int* lids,
                             const int* lpos, int nle, int s, unsigned char* kbuf,
-                            unsigned char* vbuf, uint64_t* bar) {
+                            unsigned char* vbuf, uint64_t* bar, int lane) {
   const int TS = a.stage_tokens;
   const int total = lpos[nle];
   const int w0 = s * TS, w1 = min(w0 + TS, total);
-  mbar_arrive_expect_tx(bar, (uint32_t)(2 * (w1 - w0) * ROWB));
-  for (int j = 0; j < nle; ++j) {
+  if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * (w1 - w0) * ROWB));
+  __syncwarp();
+  fence_proxy_async_smem();
+  for (int j = lane; j < nle; j += 32) {
     const int p0 = lpos[j], p1 = lpos[j + 1];
     const int a0 = max(p0, w0), a1 = min(p1, w1);
     if (a0 >= a1) continue;
@@ -126,29 +141,30 @@ __device__ void issue_stage(const AttnArgs& a, const char* Ku, const char* Vu, c
   }
 }
 
-template <typename TKV, int D>
+template <typename TKV, int D, bool CLUSTER>
 __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) {
   constexpr int E = sizeof(TKV);
   constexpr int ROWB = D * E;
-  constexpr int VEC = 16 / E;
-  constexpr int NCH = ROWB / 16;  // 16-byte chunks per row (power of two)
+  constexpr int VEC = 16 / E;     // elements per 16-byte chunk
+  constexpr int NCH = ROWB / 16;  // 16-byte chunks per row
+  constexpr int CPL = NCH / 4;    // chunks per lane, four lanes per token
   constexpr int DPL = D / 32;     // output dims per lane
-  static_assert((NCH & (NCH - 1)) == 0, "chunks per row must be a power of two");
+  static_assert(NCH % 8 == 0, "row must split into an even number of chunks per lane");
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const AttnSmem L = attn_smem_layout(D, ROWB, a.lps, a.stage_tokens, a.nbuf);
+  const AttnSmem L = attn_smem_layout(D, ROWB, a.lps, a.stage_tokens, a.nbuf, CLUSTER);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-  float* qs = reinterpret_cast<float*>(smem + L.qs);
   float* red = reinterpret_cast<float*>(smem + L.red);
   int* meta = reinterpret_cast<int*>(smem + L.meta);
   int* lids = reinterpret_cast<int*>(smem + L.lids);
   int* lpos = reinterpret_cast<int*>(smem + L.lpos);
-  float* sc = reinterpret_cast<float*>(smem + L.sc);
   float* accr = reinterpret_cast<float*>(smem + L.accr);
+  float* part = reinterpret_cast<float*>(smem + L.part);
   unsigned char* kv = smem + L.kv;
   const int TS = a.stage_tokens;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* pw = reinterpret_cast<float*>(smem + L.pw) + warp * 16;
   const long long item = blockIdx.x;
   const long long qg = item / a.splits;
   const int split = (int)(item - qg * a.splits);
@@ -157,48 +173,101 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
   const long long unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
   const char* Ku = a.K + unit * a.kv_unit_stride;
   const char* Vu = a.V + unit * a.kv_unit_stride;
+  pdl_wait();
+  pdl_release();
+  // cluster path: announce this CTA has started (waited on before any distributed
+  // shared-memory write into the rank-0 CTA)
+  if (CLUSTER && a.splits > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  if (tid == 0) {
-    int cnt = 0, pos = 0;
+  // Query slice into registers, 16-byte loads (four lanes per token: lane (tg = lane / 4,
+  // sub = lane % 4) holds chunks 4 (j ^ par) + sub of q, par = tg & 1, so the two tokens of
+  // a shared-memory phase read opposite bank halves).
+  const int sub = lane & 3, tg = lane >> 2, par = tg & 1;
+  float qv[CPL][VEC];
+  {
+    const unsigned char* qrow = static_cast<const unsigned char*>(a.Q) + qg * D * (a.q_bf16 ? 2 : 4);
+    if (a.q_bf16) {
+      // bf16 q: a 16-byte chunk of q holds 8 values; this lane's chunk c of VEC elements
+      // spans VEC * 2 bytes
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int c = 4 * (j ^ par) + sub;
+#pragma unroll
+        for (int e = 0; e < VEC; e += 8) {
+          const uint4 v = ldg16(qrow + (size_t)(c * VEC + e) * 2);
+          float f[8];
+          Vec16<uint16_t>::to_f32(v, f);
+#pragma unroll
+          for (int k = 0; k < 8 && e + k < VEC; ++k) qv[j][e + k] = f[k];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int c = 4 * (j ^ par) + sub;
+#pragma unroll
+        for (int e = 0; e < VEC; e += 4) {
+          const uint4 v = ldg16(qrow + (size_t)(c * VEC + e) * 4);
+          float f[4];
+          Vec16<float>::to_f32(v, f);
+#pragma unroll
+          for (int k = 0; k < 4 && e + k < VEC; ++k) qv[j][e + k] = f[k];
+        }
+      }
+    }
+  }
+  // Leaf list of this split, built by warp 0: valid leaves compacted in slot order, with
+  // the prefix of their token counts (their offsets in the split's token sequence).
+  if (warp == 0) {
     const int s0 = split * a.lps, s1 = min(s0 + a.lps, a.beam);
     const int* li = a.leaf_idx + qg * a.beam;
-    for (int s = s0; s < s1; ++s) {
-      const int j = li[s];
-      if (j < 0) continue;
+    int cnt = 0, pos = 0;
+    for (int c0 = s0; c0 < s1; c0 += 32) {
+      const int sl = c0 + lane;
+      int j = sl < s1 ? li[sl] : -1;
       if ((long long)j >= a.n0) {
         atomicOr(a.err, kDevErrBadLeaf);
-        continue;
+        j = -1;
       }
-      const long long t0 = (long long)j * a.lb;
-      const long long t1 = min(t0 + a.lb, a.N);
-      lids[cnt] = j;
-      lpos[cnt] = pos;
-      pos += (int)(t1 - t0);
-      ++cnt;
+      const bool ok = j >= 0;
+      const int ntok = ok ? (int)(min((long long)j * a.lb + a.lb, a.N) - (long long)j * a.lb) : 0;
+      int incl = ntok;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, ok);
+      if (ok) {
+        const int k = cnt + __popc(bal & ((1u << lane) - 1u));
+        lids[k] = j;
+        lpos[k] = pos + incl - ntok;
+      }
+      cnt += __popc(bal);
+      pos += __shfl_sync(0xffffffffu, incl, 31);
     }
-    lpos[cnt] = pos;
-    meta[0] = cnt;
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    fence_mbar_init();
-  }
-  for (int d = tid; d < D; d += kAttnThreads) {
-    const long long qi = qg * D + d;
-    qs[d] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[qi])
-                     : static_cast<const float*>(a.Q)[qi];
+    if (lane == 0) {
+      lpos[cnt] = pos;
+      meta[0] = cnt;
+      mbar_init(&bar[0], 1);
+      mbar_init(&bar[1], 1);
+      fence_mbar_init();
+    }
+    __syncwarp();
+    const int total0 = pos;
+    const int nst0 = (total0 + TS - 1) / TS;
+    for (int s = 0; s < min(a.nbuf, nst0); ++s)
+      issue_stage<ROWB>(a, Ku, Vu, lids, lpos, cnt, s, kv + (size_t)s * 2 * TS * ROWB,
+                        kv + (size_t)s * 2 * TS * ROWB + (size_t)TS * ROWB, &bar[s], lane);
   }
   __syncthreads();
   const int nle = meta[0];
   const int total = lpos[nle];
   const int nstages = (total + TS - 1) / TS;
   const size_t stage_bytes = (size_t)TS * ROWB;
-  if (tid == 0) {
-    for (int s = 0; s < min(a.nbuf, nstages); ++s)
-      issue_stage<ROWB>(a, Ku, Vu, lids, lpos, nle, s, kv + (size_t)s * 2 * stage_bytes,
-                        kv + (size_t)s * 2 * stage_bytes + stage_bytes, &bar[s]);
-  }
 
-  float m_run = -INFINITY, l_run = 0.f;
+  // this warp's running softmax state over the tokens it owns
+  float m_w = -INFINITY, l_w = 0.f;
   float acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
@@ -209,75 +278,90 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
     const int buf = a.nbuf == 2 ? (s & 1) : 0;
     const uint32_t parity = (uint32_t)((a.nbuf == 2 ? (s >> 1) : s) & 1);
     const bool ok = mbar_wait_bounded(&bar[buf], parity, a.err, kDevErrTimeout, kWaitCycles);
+    // one barrier per stage: the stage's data is visible to all, every warp has finished
+    // the previous stage (whose buffer the next copy may now overwrite)
     if (__syncthreads_or(!ok)) {
       failed = true;
       failed_stage = s;
       break;
     }
+    if (warp == 0 && a.nbuf == 2 && s >= 1 && s + 1 < nstages) {
+      const int nb = (s + 1) & 1;
+      issue_stage<ROWB>(a, Ku, Vu, lids, lpos, nle, s + 1, kv + (size_t)nb * 2 * stage_bytes,
+                        kv + (size_t)nb * 2 * stage_bytes + stage_bytes, &bar[nb], lane);
+    }
     const unsigned char* Ks = kv + (size_t)buf * 2 * stage_bytes;
     const unsigned char* Vs = Ks + stage_bytes;
     const int cnt = min(TS, total - s * TS);
 
-    // scores
-    float lmax = -INFINITY;
-    for (int t = tid; t < cnt; t += kAttnThreads) {
-      const unsigned char* row = Ks + (size_t)t * ROWB;
-      float dot = 0.f;
+    // rounds of 64 tokens: this warp takes tokens t0 + tg and t0 + 32 + tg
+    for (int t0 = 8 * warp; t0 < cnt; t0 += 64) {
+      float sc[2];
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        const int cc = (c + t) & (NCH - 1);
-        const uint4 v = *reinterpret_cast<const uint4*>(row + cc * 16);
-        float f[VEC];
-        Vec16<TKV>::to_f32(v, f);
-        const float* qq = qs + cc * VEC;
+      for (int u = 0; u < 2; ++u) {
+        const int t = t0 + 32 * u + tg;
+        float d0 = 0.f, d1 = 0.f;
+        if (t < cnt) {
+          const unsigned char* row = Ks + (size_t)t * ROWB;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) dot = fmaf(qq[e], f[e], dot);
+          for (int j = 0; j < CPL; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + (4 * (j ^ par) + sub) * 16);
+            float f[VEC];
+            Vec16<TKV>::to_f32(v, f);
+#pragma unroll
+            for (int e = 0; e < VEC; e += 2) {
+              d0 = fmaf(qv[j][e], f[e], d0);
+              d1 = fmaf(qv[j][e + 1], f[e + 1], d1);
+            }
+          }
+        }
+        float d = d0 + d1;
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        sc[u] = t < cnt ? d * a.qk_scale : -INFINITY;
       }
-      const float sv = dot * a.qk_scale;
-      sc[t] = sv;
-      lmax = fmaxf(lmax, sv);
-    }
-    lmax = warp_max(lmax);
-    if (lane == 0) red[warp] = lmax;
-    __syncthreads();
-    lmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    const float m_new = fmaxf(m_run, lmax);
-    const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
-    float lsum = 0.f;
-    for (int t = tid; t < cnt; t += kAttnThreads) {
-      const float p = exp2f(sc[t] - m_new);
-      sc[t] = p;
-      lsum += p;
-    }
-    lsum = warp_sum(lsum);
-    if (lane == 0) red[4 + warp] = lsum;
-    __syncthreads();
-    lsum = (red[4] + red[5]) + (red[6] + red[7]);
-    l_run = l_run * alpha + lsum;
-    m_run = m_new;
-
-    // weighted V: this warp takes tokens t = warp, warp + 4, ...; this lane DPL dims
+      float mg = fmaxf(sc[0], sc[1]);
+      mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 4));
+      mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 8));
+      mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 16));
+      const float m_new = fmaxf(m_w, mg);
+      const float alpha = m_w == -INFINITY ? 0.f : exp2f(m_w - m_new);
+      const float p0 = sc[0] == -INFINITY ? 0.f : exp2f(sc[0] - m_new);
+      const float p1 = sc[1] == -INFINITY ? 0.f : exp2f(sc[1] - m_new);
+      l_w = l_w * alpha + (sub == 0 ? p0 + p1 : 0.f);  // per lane; summed over the warp at the end
+      m_w = m_new;
+      if (sub == 0) {
+        pw[tg] = p0;
+        pw[8 + tg] = p1;
+      }
+      __syncwarp();
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] *= alpha;
-    for (int t = warp; t < cnt; t += kAttnWarps) {
-      const float p = sc[t];
-      float v[DPL];
-      load_v<D>(reinterpret_cast<const TKV*>(Vs + (size_t)t * ROWB) + lane * DPL, v);
+      for (int e = 0; e < DPL; ++e) acc[e] *= alpha;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(p, v[e], acc[e]);
+      for (int j = 0; j < 16; ++j) {
+        const int t = t0 + (j < 8 ? j : 24 + j);  // tokens t0 .. t0+7 and t0+32 .. t0+39
+        if (t < cnt) {
+          const float p = pw[j];
+          float v[DPL];
+          load_v<D>(reinterpret_cast<const TKV*>(Vs + (size_t)t * ROWB) + lane * DPL, v);
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(p, v[e], acc[e]);
+        }
+      }
+      __syncwarp();
     }
-    __syncthreads();  // every read of this buffer and of sc is done
-    if (tid == 0 && s + a.nbuf < nstages) {
-      fence_proxy_async_smem();
-      issue_stage<ROWB>(a, Ku, Vu, lids, lpos, nle, s + a.nbuf, kv + (size_t)buf * 2 * stage_bytes,
-                        kv + (size_t)buf * 2 * stage_bytes + stage_bytes, &bar[buf]);
+    if (a.nbuf == 1 && s + 1 < nstages) {
+      __syncthreads();  // single buffer: everyone is done with it before it is refilled
+      if (warp == 0)
+        issue_stage<ROWB>(a, Ku, Vu, lids, lpos, nle, s + 1, kv, kv + stage_bytes, &bar[0], lane);
     }
   }
 
+  float o = 0.f, M = -INFINITY, l = 0.f;
   if (failed) {
     // Give copies still in flight (the stage that timed out and the one after it) a
-    // second bounded wait before the CTA's shared memory is released, then poison the
-    // output so the failure is visible besides the error word.
+    // second bounded wait before the CTA's shared memory is released; the output of this
+    // split is poisoned so the failure is visible besides the error word.
     if (tid == 0) {
       for (int s = failed_stage; s < min(failed_stage + a.nbuf, nstages); ++s) {
         const int buf = a.nbuf == 2 ? (s & 1) : 0;
@@ -286,46 +370,72 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
       }
     }
     __syncthreads();
+    o = __int_as_float(0x7fc00000);
+    M = 0.f;
+    l = __int_as_float(0x7fc00000);
+  } else {
+    // merge the four warps' states
+    l_w = warp_sum(l_w);
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) accr[warp * D + lane * DPL + e] = acc[e];
+    if (lane == 0) {
+      red[warp] = m_w;
+      red[4 + warp] = l_w;
+    }
+    __syncthreads();
     if (tid < D) {
-      const float nanv = __int_as_float(0x7fc00000);
-      if (a.splits == 1) {
-        if (a.o_bf16)
-          static_cast<uint16_t*>(a.O)[qg * D + tid] = f32_to_bf16_bits(nanv);
-        else
-          static_cast<float*>(a.O)[qg * D + tid] = nanv;
-      } else {
-        float* pp = a.partial + (qg * a.splits + split) * (D + 2);
-        pp[tid] = nanv;
-        if (tid == 0) {
-          pp[D] = 0.f;
-          pp[D + 1] = nanv;
-        }
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, red[w]);
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w) {
+        const float sw = red[w] == -INFINITY ? 0.f : exp2f(red[w] - M);
+        o = fmaf(sw, accr[w * D + tid], o);
+        l = fmaf(sw, red[4 + w], l);
       }
     }
-    return;
   }
 
-  // cross-warp reduction of the accumulators
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) accr[warp * D + lane * DPL + e] = acc[e];
-  __syncthreads();
-  if (tid < D) {
-    float o = 0.f;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) o += accr[w * D + tid];
-    if (a.splits == 1) {
-      const float r = l_run > 0.f ? o / l_run : 0.f;
+  if (a.splits == 1) {
+    if (tid < D) {
+      const float r = failed ? o : (l > 0.f ? o / l : 0.f);
       if (a.o_bf16)
         static_cast<uint16_t*>(a.O)[qg * D + tid] = f32_to_bf16_bits(r);
       else
         static_cast<float*>(a.O)[qg * D + tid] = r;
-    } else {
-      float* pp = a.partial + (qg * a.splits + split) * (D + 2);
-      pp[tid] = o;
-      if (tid == 0) {
-        pp[D] = m_run;
-        pp[D + 1] = l_run;
+    }
+  } else if (CLUSTER) {
+    // every split sends (acc, max, sum) to the rank-0 CTA of its cluster, which merges
+    cg::cluster_group cl = cg::this_cluster();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA of the cluster runs
+    float* dst = cl.map_shared_rank(part, 0) + (size_t)split * (D + 2);
+    if (tid < D) dst[tid] = o;
+    if (tid == 0) {
+      dst[D] = M;
+      dst[D + 1] = l;
+    }
+    cl.sync();
+    if (split == 0 && tid < D) {
+      float MM = -INFINITY;
+      for (int s = 0; s < a.splits; ++s) MM = fmaxf(MM, part[s * (D + 2) + D]);
+      float num = 0.f, den = 0.f;
+      for (int s = 0; s < a.splits; ++s) {
+        const float ms = part[s * (D + 2) + D];
+        const float w = ms == -INFINITY ? 0.f : exp2f(ms - MM);
+        num = fmaf(w, part[s * (D + 2) + tid], num);
+        den = fmaf(w, part[s * (D + 2) + D + 1], den);
       }
+      const float r = den > 0.f ? num / den : (den == den ? 0.f : den);
+      if (a.o_bf16)
+        static_cast<uint16_t*>(a.O)[qg * D + tid] = f32_to_bf16_bits(r);
+      else
+        static_cast<float*>(a.O)[qg * D + tid] = r;
+    }
+  } else if (tid < D) {
+    float* pp = a.partial + (qg * a.splits + split) * (D + 2);
+    pp[tid] = o;
+    if (tid == 0) {
+      pp[D] = M;
+      pp[D + 1] = l;
     }
   }
 }
@@ -337,6 +447,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* partial, int 
   constexpr int DPL = D / 32;
   const long long qg = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_release();
   if (qg >= total_q) return;
   const float* p = partial + qg * splits * (D + 2);
   float M = -INFINITY;
@@ -354,7 +466,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* partial, int 
   }
 #pragma unroll
   for (int e = 0; e < DPL; ++e) {
-    const float r = den > 0.f ? acc[e] / den : 0.f;
+    const float r = den > 0.f ? acc[e] / den : (den == den ? 0.f : den);
     const long long o = qg * D + lane * DPL + e;
     if (o_bf16)
       static_cast<uint16_t*>(O)[o] = f32_to_bf16_bits(r);
@@ -363,40 +475,76 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* partial, int 
   }
 }
 
+// Split plan.  Enough CTAs to put about two per SM; when the queries alone do not, a
+// query's leaves are split so that a split fits one stage (up to 8 splits, merged inside a
+// cluster).  Very few queries with long leaf lists use more splits (scratch path).
 AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam) {
   AttnPlan p{};
   const int D = t->desc.head_dim;
   const int E = t->desc.kv_dtype == ZHA_BF16 ? 2 : 4;
   const int row = D * E;
   const long long lb = t->desc.leaf_block;
-  const int ts_max = std::max(8, 32768 / (2 * row));
+  const int ts_max = std::max(8, 32768 / (2 * row));  // a stage of K + V rows: 32 KB
   const long long queries = (long long)t->desc.batch * q_heads * nq;
   const long long tok = (long long)beam * lb;
-  long long want = queries > 0 ? (2LL * t->sms + queries - 1) / queries : 1;
+  const long long want = queries > 0 ? (2LL * t->sms + queries - 1) / queries : 1;
   const long long maxs = std::max(1LL, std::min((long long)beam, (tok + ts_max - 1) / ts_max));
-  long long splits = std::max(1LL, std::min(want, maxs));
-  const int lps = (int)((beam + splits - 1) / splits);
+  long long splits;
+  if (want <= kMaxClusterSplits) {
+    splits = std::min<long long>(kMaxClusterSplits, std::max(want, maxs));
+    splits = std::min<long long>(splits, beam);
+    p.cluster = splits > 1;
+  } else {
+    splits = std::max(1LL, std::min(want, maxs));
+    p.cluster = false;
+  }
+  int lps = (int)((beam + splits - 1) / splits);
   splits = (beam + lps - 1) / lps;
+  if (splits <= 1) p.cluster = false;
   const long long item_tok = (long long)lps * lb;
   const int ts = (int)std::min<long long>(ts_max, (item_tok + 7) / 8 * 8);
   p.leaves_per_split = lps;
   p.splits = (int)splits;
   p.stage_tokens = ts;
   p.stages = item_tok > ts ? 2 : 1;
-  p.smem_bytes = attn_smem_layout(D, row, lps, ts, p.stages).total;
-  p.scratch_bytes = splits > 1 ? (size_t)queries * splits * (D + 2) * sizeof(float) : 0;
+  p.smem_bytes = attn_smem_layout(D, row, lps, ts, p.stages, p.cluster).total;
+  p.scratch_bytes = (splits > 1 && !p.cluster) ? (size_t)queries * splits * (D + 2) * sizeof(float) : 0;
   return p;
 }
 
 namespace {
-template <typename TKV, int D>
+template <typename TKV, int D, bool CLUSTER>
 cudaError_t run_attend(const AttnArgs& a, const AttnPlan& plan, cudaStream_t s) {
-  auto kern = attend_kernel<TKV, D>;
+  auto kern = attend_kernel<TKV, D, CLUSTER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)plan.smem_bytes);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)a.total_items, kAttnThreads, plan.smem_bytes, s>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.total_items);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = plan.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int nattr = 1;
+  if (CLUSTER) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)plan.splits;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    nattr = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = nattr;
+  e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <typename TKV, int D>
+cudaError_t run_attend_any(const AttnArgs& a, const AttnPlan& plan, cudaStream_t s) {
+  return plan.cluster ? run_attend<TKV, D, true>(a, plan, s) : run_attend<TKV, D, false>(a, plan, s);
 }
 }  // namespace
 
@@ -434,18 +582,22 @@ cudaError_t launch_attention(zha_tree* t, const AttnPlan& plan, const void* d_Q,
   a.total_items = queries * plan.splits;
   cudaError_t e;
   if (bf)
-    e = D == 128 ? run_attend<uint16_t, 128>(a, plan, stream) : run_attend<uint16_t, 64>(a, plan, stream);
+    e = D == 128 ? run_attend_any<uint16_t, 128>(a, plan, stream)
+                 : run_attend_any<uint16_t, 64>(a, plan, stream);
   else
-    e = D == 128 ? run_attend<float, 128>(a, plan, stream) : run_attend<float, 64>(a, plan, stream);
+    e = D == 128 ? run_attend_any<float, 128>(a, plan, stream)
+                 : run_attend_any<float, 64>(a, plan, stream);
   ++t->launches;
-  if (e != cudaSuccess || plan.splits == 1) return e;
+  if (e != cudaSuccess || plan.splits == 1 || plan.cluster) return e;
   const unsigned blocks = (unsigned)((queries + 3) / 4);
   if (D == 128)
-    combine_kernel<128><<<blocks, 128, 0, stream>>>(a.partial, plan.splits, d_O, a.o_bf16, queries);
+    e = launch_pdl(combine_kernel<128>, dim3(blocks), dim3(128), 0, stream,
+                   (const float*)a.partial, plan.splits, d_O, a.o_bf16, queries);
   else
-    combine_kernel<64><<<blocks, 128, 0, stream>>>(a.partial, plan.splits, d_O, a.o_bf16, queries);
+    e = launch_pdl(combine_kernel<64>, dim3(blocks), dim3(128), 0, stream,
+                   (const float*)a.partial, plan.splits, d_O, a.o_bf16, queries);
   ++t->launches;
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace zha

@@ -21,7 +21,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 256 * 1024;
+constexpr size_t kNoAllocScratchBytes = 128 * 1024;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchBytes];

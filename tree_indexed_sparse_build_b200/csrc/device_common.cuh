@@ -116,3 +116,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 }  // namespace zha
+
+namespace zha {
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still running;
+// pdl_wait() blocks until that kernel has completed and its writes are visible, so it
+// must precede the first read of anything an earlier kernel produced.
+// pdl_release() lets the next kernel in the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace zha

@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
   const int qi = warp / a.wpq, wq = warp - qi * a.wpq;
   const long long qg = (long long)blockIdx.x * a.qpc + qi;
   const bool valid = qg < a.total_queries;
+  pdl_wait();
+  pdl_release();
 
   unsigned long long* keys = route_smem + (size_t)qi * a.query_smem_words;
   int* surv_a = reinterpret_cast<int*>(keys + a.cmax);
@@ -378,6 +380,50 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
   }
 }
 
+// One warp: keep the top-min(beam, C) of keys[0, C) and write their node ids (cand) to
+// nxt in candidate order (and their scores to leaf_sc when `leaf`).  Keys and ids for
+// k = lane + 32 i, i < R, are held in registers; candidates past 32 R come from shared
+// memory.  Returns the number kept.
+template <int R>
+__device__ __forceinline__ int select_compact(const unsigned long long* keys, const int* cand, int C,
+                                              int beam, int lane, int* nxt, float* leaf_sc,
+                                              bool leaf) {
+  unsigned long long kr[R];
+  int cr[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int k = lane + 32 * i;
+    kr[i] = k < C ? keys[k] : 0ull;
+    cr[i] = k < C ? cand[k] : 0;
+  }
+  const unsigned long long T = C > beam ? select_threshold<R>(kr, keys, C, beam, lane) : 0ull;
+  int kept = 0;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const bool keep = lane + 32 * i < C && kr[i] >= T;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+      nxt[pos] = cr[i];
+      if (leaf) leaf_sc[pos] = key_score(kr[i]);
+    }
+    kept += __popc(bal);
+  }
+  for (int k0 = 32 * R; k0 < C; k0 += 32) {
+    const int k = k0 + lane;
+    const unsigned long long key = k < C ? keys[k] : 0ull;
+    const bool keep = k < C && key >= T;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+      nxt[pos] = cand[k];
+      if (leaf) leaf_sc[pos] = key_score(key);
+    }
+    kept += __popc(bal);
+  }
+  return kept;
+}
+
 // Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq, the query's warps
 // synchronised by CTA barriers.  Otherwise qpc queries per CTA with one warp each,
 // synchronised only within the warp.
@@ -405,6 +451,8 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
   auto group_sync = [&]() {
     if (WIDE) __syncthreads(); else __syncwarp();
   };
+  pdl_wait();
+  pdl_release();
 
   long long unit = 0;
   if (valid) {
@@ -501,36 +549,9 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
     }
     group_sync();
     if (wq == 0 && C > 0) {
-      unsigned long long kr[R];
-#pragma unroll
-      for (int i = 0; i < R; ++i) kr[i] = lane + 32 * i < C ? keys[lane + 32 * i] : 0ull;
-      const unsigned long long T = C > a.beam ? select_threshold<R>(kr, keys, C, a.beam, lane) : 0ull;
-      // ordered compaction of the keys >= T
-      int kept = 0;
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const int k = lane + 32 * i;
-        const bool keep = k < C && kr[i] >= T;
-        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-        if (keep) {
-          const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-          nxt[pos] = cand[k];
-          if (l == 0) leaf_sc[pos] = key_score(kr[i]);
-        }
-        kept += __popc(bal);
-      }
-      for (int k0 = 32 * R; k0 < C; k0 += 32) {
-        const int k = k0 + lane;
-        const unsigned long long key = k < C ? keys[k] : 0ull;
-        const bool keep = k < C && key >= T;
-        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-        if (keep) {
-          const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-          nxt[pos] = cand[k];
-          if (l == 0) leaf_sc[pos] = key_score(key);
-        }
-        kept += __popc(bal);
-      }
+      const int kept = C <= 64    ? select_compact<2>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
+                       : C <= 128 ? select_compact<4>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
+                                  : select_compact<R>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0);
       __syncwarp();
       if (a.trace && valid) {
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
@@ -561,7 +582,8 @@ cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size
   auto kern = route_tma_kernel<D, WIDE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<blocks, threads, smem, s>>>(a);
+  e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -571,7 +593,8 @@ cudaError_t run_route(const RouteArgs& a, unsigned blocks, int threads, size_t s
   auto kern = route_reg_kernel<D, U>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<blocks, threads, smem, s>>>(a);
+  e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 }  // namespace

@@ -53,6 +53,8 @@ __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassAr
   static_assert(LPR <= 32 && 32 % LPR == 0, "row must split evenly over a warp");
 
   extern __shared__ double smem_d[];
+  pdl_wait();
+  pdl_release();
   double* bufA = smem_d;                        // [chunk][D]
   double* bufB = smem_d + (size_t)a.chunk * D;  // [chunk / b][D]
 
@@ -198,6 +200,8 @@ __global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendP
   double* cur = reinterpret_cast<double*>(psm + a.fp64_off);
   double* nxt = cur + kPathMaxLeaves * D;
   uint64_t* bar = reinterpret_cast<uint64_t*>(psm + a.bar_off);
+  pdl_wait();
+  pdl_release();
 
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
@@ -282,7 +286,8 @@ cudaError_t launch_pass(const PassArgs& a, dim3 grid, size_t smem, cudaStream_t 
   auto kern = pyramid_pass_kernel<TIn, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kPassThreads, smem, s>>>(a);
+  e = launch_pdl(kern, grid, dim3(kPassThreads), smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -291,7 +296,8 @@ cudaError_t launch_path(const AppendPathArgs& a, unsigned grid, size_t smem, cud
   auto kern = append_path_kernel<TIn, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kPathThreads, smem, s>>>(a);
+  e = launch_pdl(kern, dim3(grid), dim3(kPathThreads), smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

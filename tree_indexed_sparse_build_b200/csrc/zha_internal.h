@@ -16,6 +16,24 @@ constexpr int kMaxCandidates = 4096;  // beam * branching bound for the route ke
 // Bits of the device error word.
 enum : unsigned { kDevErrTimeout = 1u, kDevErrBadLeaf = 2u };
 
+// Launch `kern` with programmatic stream serialization (see pdl_wait in
+// device_common.cuh): the kernel may begin while its predecessor drains.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 }  // namespace zha
 
 struct zha_tree {
@@ -56,6 +74,7 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
 struct AttnPlan {
   int leaves_per_split;
   int splits;
+  bool cluster;        // splits of a query merge inside one thread-block cluster
   int stage_tokens;
   int stages;          // smem buffers (1 or 2)
   size_t smem_bytes;
