@@ -49,8 +49,8 @@ CASES = [
     # > 2 queries per SM: one warp per query, several queries per CTA
     _wl("bf16_d128_narrow", 2, 2, 8, 128, 6000, "bf16", 8, 16, 8, 32, 111),
     _wl("f32_d64_narrow", 1, 2, 4, 64, 3000, "f32", 4, 8, 5, 80, 113),
-    # 38 .. 296 queries with long leaf lists: splits merged inside a thread-block cluster
-    _wl("bf16_d128_cluster", 4, 2, 8, 128, 9000, "bf16", 16, 32, 16, 2, 114),
+    # enough queries that a few splits per query fill the GPU: merged inside a cluster
+    _wl("bf16_d128_cluster", 4, 2, 8, 128, 9000, "bf16", 16, 32, 16, 4, 114),
     _wl("f32_d64_cluster", 2, 2, 8, 64, 3000, "f32", 4, 16, 8, 4, 115),
     # widest level (beam * b = 512 rows) too large to stage: register-batched route kernel
     _wl("bf16_d128_regpath", 1, 1, 2, 128, 20000, "bf16", 8, 4, 64, 2, 112),

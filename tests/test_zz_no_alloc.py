@@ -41,9 +41,9 @@ def _setup(w: Workload, dev, zha):
 @pytest.mark.parametrize("kv_dtype", ["bf16", "f32"])
 def test_noalloc_matches_caller_scratch_twice(kv_dtype):
     dev, zha = _need_gpu()
-    # few queries, 16 leaves of 32 tokens each: every query's leaves are split over many
-    # CTAs whose partials go through the fixed array (fp32 rows split finer: one batch)
-    w = Workload(name="noalloc", batch=2 if kv_dtype == "bf16" else 1, kv_heads=2, q_heads=8,
+    # few queries, 16 leaves of 32 tokens each: every query's leaves are split over more
+    # CTAs than a cluster holds, so their partials go through the fixed array
+    w = Workload(name="noalloc", batch=1, kv_heads=2, q_heads=8,
                  head_dim=128, seq_len=9000, kv_dtype=kv_dtype, branching=16, leaf_block=32,
                  beam=16, nq=1, seed=0x2A0F0)
     tree, K, V = _setup(w, dev, zha)
@@ -72,8 +72,8 @@ def test_noalloc_matches_caller_scratch_twice(kv_dtype):
 
 def test_noalloc_refuses_partials_beyond_capacity():
     dev, zha = _need_gpu()
-    # 36 queries with 16 leaves of 64 tokens each: eight splits per query whose partials
-    # (36 x 8 x 130 fp32) exceed the fixed array
+    # 36 queries with 16 leaves of 64 tokens each: sixteen splits per query whose partials
+    # (36 x 16 x 130 fp32) exceed the fixed array
     w = Workload(name="noalloc_big", batch=1, kv_heads=4, q_heads=36, head_dim=128,
                  seq_len=4096, kv_dtype="bf16", branching=16, leaf_block=64, beam=16, nq=1,
                  seed=0x2A0F1)

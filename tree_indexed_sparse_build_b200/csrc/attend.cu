@@ -78,12 +78,14 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int D, int row_bytes, int l
   o += (size_t)(lps + 1) * 4;
   s.pw = align_up(o, 16);  // per-warp softmax weights of one round [warps][16]
   o = s.pw + (size_t)kAttnWarps * 16 * 4;
-  s.accr = align_up(o, 16);
-  o = s.accr + (size_t)kAttnWarps * D * 4;
-  s.part = align_up(o, 16);  // cluster path, rank 0: the splits' partials [8][D + 2]
-  o = s.part + (cluster ? (size_t)kMaxClusterSplits * (D + 2) * 4 : 0);
   s.kv = align_up(o, 128);
-  s.total = s.kv + (size_t)nbuf * 2 * stage_tokens * row_bytes;
+  // After the last stage the stage buffers are free: the four warps' accumulators and, in
+  // the cluster path (rank 0), the splits' partials [8][D + 2] reuse them.
+  s.accr = s.kv;
+  s.part = s.kv + align_up((size_t)kAttnWarps * D * 4, 16);
+  const size_t tail = (s.part - s.kv) + (cluster ? (size_t)kMaxClusterSplits * (D + 2) * 4 : 0);
+  const size_t stages = (size_t)nbuf * 2 * stage_tokens * row_bytes;
+  s.total = s.kv + (stages > tail ? stages : tail);
   return s;
 }
 
@@ -175,9 +177,6 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
   const char* Vu = a.V + unit * a.kv_unit_stride;
   pdl_wait();
   pdl_release();
-  // cluster path: announce this CTA has started (waited on before any distributed
-  // shared-memory write into the rank-0 CTA)
-  if (CLUSTER && a.splits > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
   // Query slice into registers, 16-byte loads (four lanes per token: lane (tg = lane / 4,
   // sub = lane % 4) holds chunks 4 (j ^ par) + sub of q, par = tg & 1, so the two tokens of
@@ -358,6 +357,13 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
   }
 
   float o = 0.f, M = -INFINITY, l = 0.f;
+  // From here on this CTA no longer reads its stage buffers from the stage loop; in the
+  // cluster path announce it (the rank-0 CTA receives partials into those buffers once
+  // every CTA of the cluster has arrived).
+  if (CLUSTER && a.splits > 1) {
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  }
   if (failed) {
     // Give copies still in flight (the stage that timed out and the one after it) a
     // second bounded wait before the CTA's shared memory is released; the output of this
@@ -374,8 +380,10 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
     M = 0.f;
     l = __int_as_float(0x7fc00000);
   } else {
-    // merge the four warps' states
+    // merge the four warps' states (the accumulators reuse the stage buffers: wait until
+    // every warp is done with them)
     l_w = warp_sum(l_w);
+    __syncthreads();
 #pragma unroll
     for (int e = 0; e < DPL; ++e) accr[warp * D + lane * DPL + e] = acc[e];
     if (lane == 0) {
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
   } else if (CLUSTER) {
     // every split sends (acc, max, sum) to the rank-0 CTA of its cluster, which merges
     cg::cluster_group cl = cg::this_cluster();
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA of the cluster runs
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // all past their stages
     float* dst = cl.map_shared_rank(part, 0) + (size_t)split * (D + 2);
     if (tid < D) dst[tid] = o;
     if (tid == 0) {
@@ -475,29 +483,26 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* partial, int 
   }
 }
 
-// Split plan.  Enough CTAs to put about two per SM; when the queries alone do not, a
-// query's leaves are split so that a split fits one stage (up to 8 splits, merged inside a
-// cluster).  Very few queries with long leaf lists use more splits (scratch path).
+// Split plan.  Stages of 16 KB (K + V rows) in two buffers, so about six CTAs fit on an
+// SM; a query's leaves are split so the whole grid fills one wave of such CTAs (up to 8
+// splits, merged inside a cluster).  Very few queries with long leaf lists use more
+// splits, merged through caller scratch by combine_kernel.
 AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam) {
   AttnPlan p{};
   const int D = t->desc.head_dim;
   const int E = t->desc.kv_dtype == ZHA_BF16 ? 2 : 4;
   const int row = D * E;
   const long long lb = t->desc.leaf_block;
-  const int ts_max = std::max(8, 32768 / (2 * row));  // a stage of K + V rows: 32 KB
+  const int ts_max = std::max(8, 16384 / (2 * row));
   const long long queries = (long long)t->desc.batch * q_heads * nq;
   const long long tok = (long long)beam * lb;
-  const long long want = queries > 0 ? (2LL * t->sms + queries - 1) / queries : 1;
-  const long long maxs = std::max(1LL, std::min((long long)beam, (tok + ts_max - 1) / ts_max));
-  long long splits;
-  if (want <= kMaxClusterSplits) {
-    splits = std::min<long long>(kMaxClusterSplits, std::max(want, maxs));
-    splits = std::min<long long>(splits, beam);
-    p.cluster = splits > 1;
-  } else {
-    splits = std::max(1LL, std::min(want, maxs));
-    p.cluster = false;
-  }
+  const size_t cta_smem = attn_smem_layout(D, row, 64, ts_max, 2, true).total + 1024;
+  const long long per_sm = std::max<long long>(1, std::min<long long>(16, (227 * 1024) / cta_smem));
+  const long long slots = per_sm * t->sms;
+  const long long want = queries > 0 ? std::max(1LL, slots / queries) : 1;
+  const long long maxs = std::max(1LL, std::min((long long)beam, (tok + lb - 1) / lb));
+  long long splits = std::max(1LL, std::min(want, maxs));
+  p.cluster = splits > 1 && splits <= kMaxClusterSplits;
   int lps = (int)((beam + splits - 1) / splits);
   splits = (beam + lps - 1) / lps;
   if (splits <= 1) p.cluster = false;

@@ -60,7 +60,7 @@ constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
 // Shared-memory layout of one query in the staged kernel.
 struct RouteSmem {
-  size_t rows, keys, cand, surv_a, surv_b, leaf_sc, bar, total;
+  size_t rows, keys, cand, surv_a, surv_b, leaf_sc, red, bar, total;
 };
 __host__ __device__ inline size_t route_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam) {
@@ -78,6 +78,9 @@ __host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam
   o += (size_t)beam * 4;
   s.leaf_sc = o;
   o += (size_t)beam * 4;
+  o = route_align(o, 16);
+  s.red = o;  // per-warp partial results of the CTA-wide selection [3][16]
+  o += 3 * 16 * 4;
   o = route_align(o, 8);
   s.bar = o;
   o += 8;
@@ -424,6 +427,77 @@ __device__ __forceinline__ int select_compact(const unsigned long long* keys, co
   return kept;
 }
 
+// Whole-CTA variant for one query per CTA with C <= blockDim.x: thread t holds candidate t.
+// The threshold search counts with __syncthreads_count (one CTA barrier per bit); the kept
+// candidates are compacted in candidate order with per-warp ballots and a prefix over the
+// warps' counts.  Every thread of the CTA must call it.  Returns the number kept.
+__device__ __forceinline__ int select_compact_cta(const unsigned long long* keys, const int* cand,
+                                                  int C, int beam, int* nxt, float* leaf_sc,
+                                                  bool leaf, unsigned* red) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = (int)(blockDim.x >> 5);
+  const bool have = t < C;
+  const unsigned long long key = have ? keys[t] : 0ull;
+  const int node = have ? cand[t] : 0;
+  const uint32_t h = (uint32_t)(key >> 32);
+  unsigned long long T = 0ull;
+  if (C > beam) {
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, have ? h : 0u);
+    const uint32_t wmin = __reduce_min_sync(0xffffffffu, have ? h : 0xFFFFFFFFu);
+    if (lane == 0) {
+      red[warp] = wmax;
+      red[16 + warp] = wmin;
+    }
+    __syncthreads();
+    uint32_t hmax = 0u, hmin = 0xFFFFFFFFu;
+    for (int w = 0; w < nw; ++w) {
+      hmax = max(hmax, red[w]);
+      hmin = min(hmin, red[16 + w]);
+    }
+    const uint32_t diff = hmax ^ hmin;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t Th = top < 0 ? hmax : (top >= 31 ? 0u : (hmax & ~((2u << top) - 1u)));
+    bool done = false;
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t c = Th | (1u << bit);
+      const int cnt = __syncthreads_count(have && h >= c);
+      if (cnt >= beam) {
+        Th = c;
+        if (cnt == beam) {
+          done = true;
+          break;
+        }
+      }
+    }
+    if (done) {
+      T = (unsigned long long)Th << 32;
+    } else {
+      const int need = beam - __syncthreads_count(have && h > Th);
+      uint32_t Tl = 0u;
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t c = Tl | (1u << bit);
+        const int cnt = __syncthreads_count(have && h == Th && (uint32_t)key >= c);
+        if (cnt >= need) {
+          Tl = c;
+          if (cnt == need) break;
+        }
+      }
+      T = ((unsigned long long)Th << 32) | Tl;
+    }
+  }
+  const bool keep = have && key >= T;
+  const unsigned bal = __ballot_sync(0xffffffffu, keep);
+  if (lane == 0) red[32 + warp] = __popc(bal);
+  __syncthreads();
+  int pre = 0;
+  for (int w = 0; w < warp; ++w) pre += (int)red[32 + w];
+  if (keep) {
+    const int pos = pre + __popc(bal & ((1u << lane) - 1u));
+    nxt[pos] = node;
+    if (leaf) leaf_sc[pos] = key_score(key);
+  }
+  return min(C, beam);
+}
+
 // Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq, the query's warps
 // synchronised by CTA barriers.  Otherwise qpc queries per CTA with one warp each,
 // synchronised only within the warp.
@@ -447,6 +521,7 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
   int* surv_b = reinterpret_cast<int*>(base + Ls.surv_b);
   float* leaf_sc = reinterpret_cast<float*>(base + Ls.leaf_sc);
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + Ls.bar);
+  unsigned* red = reinterpret_cast<unsigned*>(base + Ls.red);
 
   auto group_sync = [&]() {
     if (WIDE) __syncthreads(); else __syncwarp();
@@ -548,7 +623,14 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
       }
     }
     group_sync();
-    if (wq == 0 && C > 0) {
+    if (WIDE && C > 64 && C <= 32 * nw) {  // C is the same for the whole CTA
+      const int kept = select_compact_cta(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red);
+      __syncthreads();
+      if (wq == 0 && a.trace && valid) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
+      }
+    } else if (wq == 0 && C > 0) {
       const int kept = C <= 64    ? select_compact<2>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
                        : C <= 128 ? select_compact<4>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
                                   : select_compact<R>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0);
