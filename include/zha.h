@@ -152,6 +152,22 @@ zha_status zha_sparse_attn_decode_noalloc(const zha_tree* tree, const void* d_Q,
                                           zha_dtype o_dtype, void* stream);
 size_t zha_noalloc_scratch_capacity(void);
 
+/* Route + attention of a decode step in one call: the results of zha_route followed by
+ * zha_sparse_attn_decode over the leaves it selected, computed by one kernel launch in
+ * which each query's warps route it and then attend over its leaves' tokens (no leaf
+ * list or partials pass through global memory).  Arguments as in those two calls:
+ *   d_leaf_idx    out [batch, q_heads, nq, beam] int32, required: the selected leaves
+ *   d_leaf_score  out, nullable: their scores
+ *   d_O           out [batch, q_heads, nq, head_dim] in o_dtype
+ * Same constraints (q_heads % kv_heads == 0, 1 <= beam <= 1024, beam * branching <= 4096,
+ * non-empty tree).  Needs no scratch.  When a query's widest level is too large to
+ * stage in shared memory (more than about 200 KB of summary rows), the call runs the
+ * route and the attention as two launches instead, with the same results; it returns
+ * ZHA_ERR_UNSUPPORTED if that attention would need scratch (use the two calls then). */
+zha_status zha_decode(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                      int beam, const void* d_K, const void* d_V, float scale, int* d_leaf_idx,
+                      float* d_leaf_score, void* d_O, zha_dtype o_dtype, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word:
  * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */
 zha_status zha_tree_check(zha_tree* tree, void* stream);

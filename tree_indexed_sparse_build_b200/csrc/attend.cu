@@ -29,6 +29,7 @@
 
 #include <algorithm>
 
+#include "attn_core.cuh"
 #include "device_common.cuh"
 #include "zha_internal.h"
 
@@ -38,7 +39,6 @@ namespace zha {
 
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = kAttnThreads / 32;
-constexpr int kMaxClusterSplits = 8;
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
 struct AttnArgs {
@@ -89,35 +89,6 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int D, int row_bytes, int l
   return s;
 }
 
-template <int D>
-__device__ __forceinline__ void load_v(const uint16_t* p, float* o) {
-  if constexpr (D / 32 == 4) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    o[0] = __uint_as_float(v.x << 16);
-    o[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    o[2] = __uint_as_float(v.y << 16);
-    o[3] = __uint_as_float(v.y & 0xFFFF0000u);
-  } else {
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
-    o[0] = __uint_as_float(v << 16);
-    o[1] = __uint_as_float(v & 0xFFFF0000u);
-  }
-}
-template <int D>
-__device__ __forceinline__ void load_v(const float* p, float* o) {
-  if constexpr (D / 32 == 4) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    o[0] = v.x;
-    o[1] = v.y;
-    o[2] = v.z;
-    o[3] = v.w;
-  } else {
-    const float2 v = *reinterpret_cast<const float2*>(p);
-    o[0] = v.x;
-    o[1] = v.y;
-  }
-}
-
 // Issue the bulk copies of stage `s` (tokens [s*TS, s*TS + TS) of the work item's token
 // sequence) into buffers kbuf/vbuf.  Called by all lanes of one warp: lane 0 registers the
 // stage's byte count on the barrier, then each lane copies the pieces of its leaves.
@@ -145,13 +116,11 @@ __device__ void issue_stage(const AttnArgs& a, const char* Ku, const char* Vu, c
 
 template <typename TKV, int D, bool CLUSTER>
 __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) {
-  constexpr int E = sizeof(TKV);
-  constexpr int ROWB = D * E;
-  constexpr int VEC = 16 / E;     // elements per 16-byte chunk
-  constexpr int NCH = ROWB / 16;  // 16-byte chunks per row
-  constexpr int CPL = NCH / 4;    // chunks per lane, four lanes per token
-  constexpr int DPL = D / 32;     // output dims per lane
-  static_assert(NCH % 8 == 0, "row must split into an even number of chunks per lane");
+  using S = AttnShape<TKV, D>;
+  constexpr int ROWB = S::ROWB;
+  constexpr int VEC = S::VEC;
+  constexpr int CPL = S::CPL;
+  constexpr int DPL = S::DPL;
 
   extern __shared__ __align__(128) unsigned char smem[];
   const AttnSmem L = attn_smem_layout(D, ROWB, a.lps, a.stage_tokens, a.nbuf, CLUSTER);
@@ -178,43 +147,9 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
   pdl_wait();
   pdl_release();
 
-  // Query slice into registers, 16-byte loads (four lanes per token: lane (tg = lane / 4,
-  // sub = lane % 4) holds chunks 4 (j ^ par) + sub of q, par = tg & 1, so the two tokens of
-  // a shared-memory phase read opposite bank halves).
-  const int sub = lane & 3, tg = lane >> 2, par = tg & 1;
+  // Query slice into registers (four lanes per token, see attn_core.cuh).
   float qv[CPL][VEC];
-  {
-    const unsigned char* qrow = static_cast<const unsigned char*>(a.Q) + qg * D * (a.q_bf16 ? 2 : 4);
-    if (a.q_bf16) {
-      // bf16 q: a 16-byte chunk of q holds 8 values; this lane's chunk c of VEC elements
-      // spans VEC * 2 bytes
-#pragma unroll
-      for (int j = 0; j < CPL; ++j) {
-        const int c = 4 * (j ^ par) + sub;
-#pragma unroll
-        for (int e = 0; e < VEC; e += 8) {
-          const uint4 v = ldg16(qrow + (size_t)(c * VEC + e) * 2);
-          float f[8];
-          Vec16<uint16_t>::to_f32(v, f);
-#pragma unroll
-          for (int k = 0; k < 8 && e + k < VEC; ++k) qv[j][e + k] = f[k];
-        }
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < CPL; ++j) {
-        const int c = 4 * (j ^ par) + sub;
-#pragma unroll
-        for (int e = 0; e < VEC; e += 4) {
-          const uint4 v = ldg16(qrow + (size_t)(c * VEC + e) * 4);
-          float f[4];
-          Vec16<float>::to_f32(v, f);
-#pragma unroll
-          for (int k = 0; k < 4 && e + k < VEC; ++k) qv[j][e + k] = f[k];
-        }
-      }
-    }
-  }
+  attn_load_q<TKV, D>(a.Q, a.q_bf16 != 0, qg, lane, qv);
   // Leaf list of this split, built by warp 0: valid leaves compacted in slot order, with
   // the prefix of their token counts (their offsets in the split's token sequence).
   if (warp == 0) {
@@ -294,61 +229,7 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
     const int cnt = min(TS, total - s * TS);
 
     // rounds of 64 tokens: this warp takes tokens t0 + tg and t0 + 32 + tg
-    for (int t0 = 8 * warp; t0 < cnt; t0 += 64) {
-      float sc[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int t = t0 + 32 * u + tg;
-        float d0 = 0.f, d1 = 0.f;
-        if (t < cnt) {
-          const unsigned char* row = Ks + (size_t)t * ROWB;
-#pragma unroll
-          for (int j = 0; j < CPL; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(row + (4 * (j ^ par) + sub) * 16);
-            float f[VEC];
-            Vec16<TKV>::to_f32(v, f);
-#pragma unroll
-            for (int e = 0; e < VEC; e += 2) {
-              d0 = fmaf(qv[j][e], f[e], d0);
-              d1 = fmaf(qv[j][e + 1], f[e + 1], d1);
-            }
-          }
-        }
-        float d = d0 + d1;
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        d += __shfl_xor_sync(0xffffffffu, d, 2);
-        sc[u] = t < cnt ? d * a.qk_scale : -INFINITY;
-      }
-      float mg = fmaxf(sc[0], sc[1]);
-      mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 4));
-      mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 8));
-      mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, 16));
-      const float m_new = fmaxf(m_w, mg);
-      const float alpha = m_w == -INFINITY ? 0.f : exp2f(m_w - m_new);
-      const float p0 = sc[0] == -INFINITY ? 0.f : exp2f(sc[0] - m_new);
-      const float p1 = sc[1] == -INFINITY ? 0.f : exp2f(sc[1] - m_new);
-      l_w = l_w * alpha + (sub == 0 ? p0 + p1 : 0.f);  // per lane; summed over the warp at the end
-      m_w = m_new;
-      if (sub == 0) {
-        pw[tg] = p0;
-        pw[8 + tg] = p1;
-      }
-      __syncwarp();
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] *= alpha;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int t = t0 + (j < 8 ? j : 24 + j);  // tokens t0 .. t0+7 and t0+32 .. t0+39
-        if (t < cnt) {
-          const float p = pw[j];
-          float v[DPL];
-          load_v<D>(reinterpret_cast<const TKV*>(Vs + (size_t)t * ROWB) + lane * DPL, v);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(p, v[e], acc[e]);
-        }
-      }
-      __syncwarp();
-    }
+    attn_tokens<TKV, D>(Ks, Vs, cnt, 8 * warp, 32, 64, qv, a.qk_scale, pw, m_w, l_w, acc, lane);
     if (a.nbuf == 1 && s + 1 < nstages) {
       __syncthreads();  // single buffer: everyone is done with it before it is refilled
       if (warp == 0)
@@ -368,8 +249,10 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
     // Give copies still in flight (the stage that timed out and the one after it) a
     // second bounded wait before the CTA's shared memory is released; the output of this
     // split is poisoned so the failure is visible besides the error word.
+    // (the first nbuf stages are issued up front, stage s + 1 only after stage s's barrier)
+    const int last_issued = min(max(failed_stage, a.nbuf - 1), nstages - 1);
     if (tid == 0) {
-      for (int s = failed_stage; s < min(failed_stage + a.nbuf, nstages); ++s) {
+      for (int s = failed_stage; s <= last_issued; ++s) {
         const int buf = a.nbuf == 2 ? (s & 1) : 0;
         const uint32_t parity = (uint32_t)((a.nbuf == 2 ? (s >> 1) : s) & 1);
         mbar_wait_bounded(&bar[buf], parity, a.err, kDevErrTimeout, kWaitCycles);
@@ -483,11 +366,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* partial, int 
   }
 }
 
-// Split plan.  Stages of 16 KB (K + V rows) in two buffers, so about six CTAs fit on an
+// Split plan (at most max_splits splits per query).  Stages of 16 KB (K + V rows) in two buffers, so about six CTAs fit on an
 // SM; a query's leaves are split so the whole grid fills one wave of such CTAs (up to 8
 // splits, merged inside a cluster).  Very few queries with long leaf lists use more
 // splits, merged through caller scratch by combine_kernel.
-AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam) {
+AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam, int max_splits) {
   AttnPlan p{};
   const int D = t->desc.head_dim;
   const int E = t->desc.kv_dtype == ZHA_BF16 ? 2 : 4;
@@ -501,7 +384,7 @@ AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam) {
   const long long slots = per_sm * t->sms;
   const long long want = queries > 0 ? std::max(1LL, slots / queries) : 1;
   const long long maxs = std::max(1LL, std::min((long long)beam, (tok + lb - 1) / lb));
-  long long splits = std::max(1LL, std::min(want, maxs));
+  long long splits = std::max(1LL, std::min(std::min(want, maxs), (long long)max_splits));
   p.cluster = splits > 1 && splits <= kMaxClusterSplits;
   int lps = (int)((beam + splits - 1) / splits);
   splits = (beam + lps - 1) / lps;

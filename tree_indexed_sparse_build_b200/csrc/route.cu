@@ -29,7 +29,9 @@
 // Fallback kernel (route_reg_kernel) for levels too wide to stage in shared memory:
 // the same selection, with candidate rows loaded into registers in batches.
 #include <algorithm>
+#include <type_traits>
 
+#include "attn_core.cuh"
 #include "device_common.cuh"
 #include "zha_internal.h"
 
@@ -54,20 +56,36 @@ struct RouteArgs {
   long long total_queries;
   unsigned* err;           // device error word (bounded waits)
   int query_smem_bytes;    // shared memory per query (staged kernel)
+  int rows_bytes;          // bytes of the candidate-row region per query
+  // fused attention (route_tma_kernel with TKV != NoKV)
+  const char* K;
+  const char* V;
+  long long kv_unit_stride;  // bytes
+  long long lb, N;
+  float qk_scale;            // scale * log2(e)
+  int stage_tokens;          // tokens per stage buffer (two buffers in the row region)
+  void* O;
+  int o_bf16;
 };
+
+struct NoKV {};  // route only: no attention epilogue
 
 constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
 // Shared-memory layout of one query in the staged kernel.
 struct RouteSmem {
-  size_t rows, keys, cand, surv_a, surv_b, leaf_sc, red, bar, total;
+  size_t rows, keys, cand, surv_a, surv_b, leaf_sc, red, pw, bar, total;
 };
 __host__ __device__ inline size_t route_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
-__host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam) {
+__host__ __device__ inline size_t route_rows_bytes(int D, int cmax) { return (size_t)cmax * D * 4; }
+// rows_bytes >= route_rows_bytes(D, cmax); a fused decode may ask for more room to stage
+// K/V, and for 16 floats of softmax weights per attending warp (pw_warps).
+__host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam, size_t rows_bytes,
+                                                       int pw_warps) {
   RouteSmem s;
   size_t o = 0;
-  s.rows = o;   // candidate summary rows, fp32 [cmax][D]
-  o += (size_t)cmax * D * 4;
+  s.rows = o;   // candidate summary rows, fp32 [cmax][D]; K/V stage buffers after the route
+  o += rows_bytes;
   s.keys = o;   // candidate keys [cmax]
   o += (size_t)cmax * 8;
   s.cand = o;   // candidate node ids [cmax]
@@ -81,9 +99,11 @@ __host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam
   o = route_align(o, 16);
   s.red = o;  // per-warp partial results of the CTA-wide selection [3][16]
   o += 3 * 16 * 4;
+  s.pw = o;   // fused attention: per-warp softmax weights of one round [pw_warps][16]
+  o += (size_t)pw_warps * 16 * 4;
   o = route_align(o, 8);
-  s.bar = o;
-  o += 8;
+  s.bar = o;  // two mbarriers: level copies / stage buffer 0, stage buffer 1
+  o += 16;
   s.total = route_align(o, 128);
   return s;
 }
@@ -501,8 +521,17 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
 // Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq, the query's warps
 // synchronised by CTA barriers.  Otherwise qpc queries per CTA with one warp each,
 // synchronised only within the warp.
-template <int D, bool WIDE>
+//
+// With TKV = the KV storage type (not NoKV) the kernel is the fused decode: once the
+// last level is selected, the query's warps attend over the tokens of its leaves.  The
+// candidate-row region, free after the leaf-level scoring, becomes two K/V stage buffers
+// filled by one bulk copy per leaf piece (K and V) on the two mbarriers; the warps run
+// the online softmax of attn_core.cuh over each stage, merge their states through shared
+// memory and write O.  No leaf list goes through global memory and nothing is launched
+// between the route and the attention.
+template <int D, bool WIDE, typename TKV>
 __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const RouteArgs a) {
+  constexpr bool ATTEND = !std::is_same<TKV, NoKV>::value;
   constexpr int CPL = D / 16;  // 16-byte chunks of a row per lane (4 lanes per row)
   constexpr int R = 8;         // candidate keys held per lane in the selecting warp
   extern __shared__ __align__(128) unsigned char rsm[];
@@ -512,7 +541,8 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
   const int nw = WIDE ? (int)(blockDim.x >> 5) : 1;
   const long long qg = (long long)blockIdx.x * (WIDE ? 1 : a.qpc) + qi;
   const bool valid = qg < a.total_queries;
-  const RouteSmem Ls = route_smem_layout(D, a.cmax, a.beam);
+  const RouteSmem Ls =
+      route_smem_layout(D, a.cmax, a.beam, (size_t)a.rows_bytes, ATTEND ? (WIDE ? a.wpq : 1) : 0);
   unsigned char* base = rsm + (size_t)qi * a.query_smem_bytes;
   const float* rows = reinterpret_cast<const float*>(base + Ls.rows);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + Ls.keys);
@@ -537,7 +567,8 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
   }
   const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
   if (wq == 0 && lane == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    if (ATTEND) mbar_init(&bar[1], 1);
     fence_mbar_init();
     surv_a[0] = 0;  // the root
   }
@@ -646,27 +677,154 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
     cur = nxt;
     nxt = tmp;
   }
-  if (valid && wq == 0) {
+  if (valid && wq == 0 && a.leaf_idx) {
     int* out = a.leaf_idx + qg * a.beam;
     for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
-    if (a.leaf_score) {
-      float* os = a.leaf_score + qg * a.beam;
-      for (int k = lane; k < a.beam; k += 32)
-        os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
+  }
+  if (valid && wq == 0 && a.leaf_score) {
+    float* os = a.leaf_score + qg * a.beam;
+    for (int k = lane; k < a.beam; k += 32) os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
+  }
+  if constexpr (ATTEND) {
+    using S = AttnShape<TKV, D>;
+    constexpr int ROWB = S::ROWB;
+    const int TS = a.stage_tokens;
+    const int lb = (int)a.lb;
+    unsigned char* sb = base + Ls.rows;  // stage buffer b: K rows at sb + 2 b TS ROWB, V after
+    const size_t stage_bytes = (size_t)TS * ROWB;
+    // Tokens of the selected leaves in slot order.  Only leaf n0 - 1 can hold fewer than
+    // lb tokens, and survivors ascend, so it can only be the last one.
+    int total = 0;
+    if (m > 0) {
+      const long long last = cur[m - 1];
+      total = (m - 1) * lb + (int)(min(last * a.lb + a.lb, a.N) - last * a.lb);
+    }
+    const int nst = (total + TS - 1) / TS;
+    const char* Ku = a.K + unit * a.kv_unit_stride;
+    const char* Vu = a.V + unit * a.kv_unit_stride;
+    // Stage st covers tokens [st TS, min(st TS + TS, total)) in buffer st & 1; the lanes of
+    // warp 0 each copy the K and V pieces of some of its leaves.
+    auto issue = [&](int st) {
+      const int b = st & 1;
+      unsigned char* kb = sb + (size_t)b * 2 * stage_bytes;
+      const int w0 = st * TS, w1 = min(w0 + TS, total);
+      if (lane == 0) mbar_arrive_expect_tx(&bar[b], (uint32_t)(2 * (w1 - w0) * ROWB));
+      __syncwarp();
+      fence_proxy_async_smem();
+      for (int j = w0 / lb + lane; j <= (w1 - 1) / lb; j += 32) {
+        const int p0 = j * lb;
+        const int a0 = max(p0, w0), a1 = min(p0 + lb, w1);
+        const long long row = (long long)cur[j] * a.lb + (a0 - p0);
+        const uint32_t bytes = (uint32_t)((a1 - a0) * ROWB);
+        bulk_copy_g2s(kb + (size_t)(a0 - w0) * ROWB, Ku + row * ROWB, bytes, &bar[b]);
+        bulk_copy_g2s(kb + stage_bytes + (size_t)(a0 - w0) * ROWB, Vu + row * ROWB, bytes, &bar[b]);
+      }
+    };
+    // phase of the wait for stage st: bar[0] carries on from the route's level copies
+    auto phase = [&](int st) -> uint32_t { return ((st & 1) ? 0u : parity) ^ (uint32_t)((st >> 1) & 1); };
+    if (wq == 0 && nst > 0) {
+      issue(0);
+      if (nst > 1) issue(1);
+    }
+    float qa[S::CPL][S::VEC];
+    if (valid) attn_load_q<TKV, D>(a.Q, a.q_bf16 != 0, qg, lane, qa);
+    float* pw = reinterpret_cast<float*>(base + Ls.pw) + wq * 16;
+    float m_w = -INFINITY, l_w = 0.f;
+    float acc[S::DPL];
+#pragma unroll
+    for (int e = 0; e < S::DPL; ++e) acc[e] = 0.f;
+    int fail_st = -1;
+    for (int st = 0; st < nst; ++st) {
+      const int b = st & 1;
+      const bool ok = mbar_wait_bounded(&bar[b], phase(st), a.err, kDevErrTimeout, kRouteWaitCycles);
+      // the stage is visible to every warp, and every warp is done with stage st - 1, whose
+      // buffer the copy of stage st + 1 now reuses
+      const bool bad = WIDE ? (__syncthreads_or(!ok) != 0) : __any_sync(0xffffffffu, !ok);
+      if (bad) {
+        fail_st = st;
+        break;
+      }
+      if (wq == 0 && st >= 1 && st + 1 < nst) issue(st + 1);
+      const unsigned char* Ks = sb + (size_t)b * 2 * stage_bytes;
+      attn_tokens<TKV, D>(Ks, Ks + stage_bytes, min(TS, total - st * TS), 8 * wq, 8 * nw, 16 * nw, qa,
+                          a.qk_scale, pw, m_w, l_w, acc, lane);
+    }
+    if (fail_st >= 0) {
+      // let the copies in flight land before the CTA's shared memory is released; the
+      // query's output is poisoned so the failure shows besides the error word
+      // (stages 0 and 1 are issued up front, stage st + 1 only after stage st's barrier)
+      const int last_issued = min(max(fail_st, 1), nst - 1);
+      if (wq == 0 && lane == 0)
+        for (int st = fail_st; st <= last_issued; ++st)
+          mbar_wait_bounded(&bar[st & 1], phase(st), a.err, kDevErrTimeout, kRouteWaitCycles);
+      if (valid && wq == 0)
+        for (int e = lane; e < D; e += 32) {
+          if (a.o_bf16)
+            static_cast<uint16_t*>(a.O)[qg * D + e] = 0x7FC0u;
+          else
+            static_cast<float*>(a.O)[qg * D + e] = __int_as_float(0x7fc00000);
+        }
+      return;
+    }
+    l_w = warp_sum(l_w);
+    if (WIDE) {
+      // merge the warps' states; the accumulators reuse the stage buffers
+      float* accr = reinterpret_cast<float*>(sb);
+      float* redf = reinterpret_cast<float*>(red);
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < S::DPL; ++e) accr[wq * D + lane * S::DPL + e] = acc[e];
+      if (lane == 0) {
+        redf[wq] = m_w;
+        redf[16 + wq] = l_w;
+      }
+      __syncthreads();
+      for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float M = -INFINITY;
+        for (int w = 0; w < nw; ++w) M = fmaxf(M, redf[w]);
+        float o = 0.f, l = 0.f;
+        for (int w = 0; w < nw; ++w) {
+          const float sw = redf[w] == -INFINITY ? 0.f : exp2f(redf[w] - M);
+          o = fmaf(sw, accr[w * D + d], o);
+          l = fmaf(sw, redf[16 + w], l);
+        }
+        const float r = l > 0.f ? o / l : 0.f;
+        if (a.o_bf16)
+          static_cast<uint16_t*>(a.O)[qg * D + d] = f32_to_bf16_bits(r);
+        else
+          static_cast<float*>(a.O)[qg * D + d] = r;
+      }
+    } else if (valid) {
+#pragma unroll
+      for (int e = 0; e < S::DPL; ++e) {
+        const float r = l_w > 0.f ? acc[e] / l_w : 0.f;
+        const long long o = qg * D + lane * S::DPL + e;
+        if (a.o_bf16)
+          static_cast<uint16_t*>(a.O)[o] = f32_to_bf16_bits(r);
+        else
+          static_cast<float*>(a.O)[o] = r;
+      }
     }
   }
 }
 
 namespace {
-template <int D, bool WIDE>
+template <int D, bool WIDE, typename TKV>
 cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
                           cudaStream_t s) {
-  auto kern = route_tma_kernel<D, WIDE>;
+  auto kern = route_tma_kernel<D, WIDE, TKV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <bool WIDE, typename TKV>
+cudaError_t run_route_tma_d(int D, const RouteArgs& a, unsigned blocks, int threads, size_t smem,
+                            cudaStream_t s) {
+  return D == 128 ? run_route_tma<128, WIDE, TKV>(a, blocks, threads, smem, s)
+                  : run_route_tma<64, WIDE, TKV>(a, blocks, threads, smem, s);
 }
 
 template <int D, int U>
@@ -679,11 +837,12 @@ cudaError_t run_route(const RouteArgs& a, unsigned blocks, int threads, size_t s
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
-}  // namespace
 
-cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads,
-                         int nq, int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
-                         cudaStream_t stream) {
+constexpr size_t kRouteSmemCap = 200 * 1024;  // staged kernel: shared memory per query
+
+// Arguments common to the route and the fused decode.
+RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                     int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace) {
   RouteArgs a{};
   const int D = t->desc.head_dim;
   a.Q = d_Q;
@@ -710,29 +869,56 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   a.leaf_score = d_leaf_score;
   a.trace = d_trace;
   a.err = t->d_err;
+  return a;
+}
+
+// Launch shape of the staged kernel.  Wide (at most two queries per SM): one query per
+// CTA, enough warps for the widest level (and, fused, for the attention tokens).
+// Narrow: up to 8 queries per CTA, one warp each.
+struct StagedShape {
+  bool wide;
+  unsigned blocks;
+  int threads;
+  size_t smem;
+};
+StagedShape staged_shape(const zha_tree* t, RouteArgs& a, size_t per_query, int attn_warps) {
+  StagedShape sh{};
+  sh.wide = a.total_queries <= 2LL * t->sms;
+  if (sh.wide) {
+    const long long want = std::max<long long>((a.cmax + 31) / 32, attn_warps);
+    a.wpq = (int)std::max(1LL, std::min<long long>(kRouteMaxWarps, want));
+    a.qpc = 1;
+    sh.blocks = (unsigned)a.total_queries;
+    sh.threads = 32 * a.wpq;
+    sh.smem = per_query;
+  } else {
+    a.wpq = 1;
+    a.qpc = (int)std::max<size_t>(1, std::min<size_t>(8, (96 * 1024) / per_query));
+    sh.blocks = (unsigned)((a.total_queries + a.qpc - 1) / a.qpc);
+    sh.threads = 32 * a.qpc;
+    sh.smem = per_query * a.qpc;
+  }
+  return sh;
+}
+}  // namespace
+
+cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads,
+                         int nq, int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
+                         cudaStream_t stream) {
+  RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, d_trace);
+  const int D = t->desc.head_dim;
+  const long long cmax = a.cmax;
   cudaError_t e;
 
   // Staged kernel when a query's widest level fits in shared memory.
-  const size_t per_query = route_smem_layout(D, (int)cmax, beam).total;
-  constexpr size_t kSmemCap = 200 * 1024;
-  if (per_query <= kSmemCap) {
+  a.rows_bytes = (int)route_rows_bytes(D, a.cmax);
+  const size_t per_query = route_smem_layout(D, a.cmax, beam, a.rows_bytes, 0).total;
+  if (per_query <= kRouteSmemCap) {
     a.query_smem_bytes = (int)per_query;
-    const bool wide = a.total_queries <= 2LL * t->sms;
-    if (wide) {
-      const int wpq = (int)std::max(1LL, std::min<long long>(kRouteMaxWarps, (cmax + 31) / 32));  // 8 rows per warp step, two steps in flight
-      a.wpq = wpq;
-      a.qpc = 1;
-      const unsigned blocks = (unsigned)a.total_queries;
-      e = D == 128 ? run_route_tma<128, true>(a, blocks, 32 * wpq, per_query, stream)
-                   : run_route_tma<64, true>(a, blocks, 32 * wpq, per_query, stream);
-    } else {
-      const int qpc = (int)std::max<size_t>(1, std::min<size_t>(8, (96 * 1024) / per_query));
-      a.wpq = 1;
-      a.qpc = qpc;
-      const unsigned blocks = (unsigned)((a.total_queries + qpc - 1) / qpc);
-      e = D == 128 ? run_route_tma<128, false>(a, blocks, 32 * qpc, per_query * qpc, stream)
-                   : run_route_tma<64, false>(a, blocks, 32 * qpc, per_query * qpc, stream);
-    }
+    // 8 rows per warp step, two steps in flight
+    const StagedShape sh = staged_shape(t, a, per_query, 0);
+    e = sh.wide ? run_route_tma_d<true, NoKV>(D, a, sh.blocks, sh.threads, sh.smem, stream)
+                : run_route_tma_d<false, NoKV>(D, a, sh.blocks, sh.threads, sh.smem, stream);
     ++t->launches;
     return e;
   }
@@ -756,6 +942,63 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   const unsigned blocks = (unsigned)((a.total_queries + a.qpc - 1) / a.qpc);
   e = D == 128 ? run_route<128, kU128>(a, blocks, threads, smem, stream)
                : run_route<64, kU64>(a, blocks, threads, smem, stream);
+  ++t->launches;
+  return e;
+}
+
+// Fused route + attention (one launch).  Row region per query: the widest level's rows,
+// or more when the attention wants bigger stages (wide: up to 128 KB, so a long leaf list
+// streams in a few large stages; narrow: up to 32 KB, so several queries still share an
+// SM), and never less than two stages of 8 tokens.
+DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
+  DecodePlan p{};
+  const int D = t->desc.head_dim;
+  const int row = D * (t->desc.kv_dtype == ZHA_BF16 ? 2 : 4);
+  const long long queries = (long long)t->desc.batch * q_heads * nq;
+  const bool wide = queries <= 2LL * t->sms;
+  long long cmax = 1;
+  for (int l = 0; l < t->L; ++l)
+    cmax = std::max(cmax, std::min(std::min((long long)beam, t->n[l + 1]) * t->desc.branching, t->n[l]));
+  const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
+  const size_t route_rows = route_rows_bytes(D, (int)cmax);
+  const size_t want = (size_t)4 * row * (size_t)((tokens + 1) / 2);
+  const size_t cap = wide ? 128 * 1024 : 32 * 1024;
+  size_t rows = std::max(route_rows, std::min(want, cap));
+  rows = std::max(rows, (size_t)4 * 8 * row);
+  p.stage_tokens = (int)(rows / (4 * row)) / 8 * 8;
+  p.rows_bytes = rows;
+  p.attn_warps = wide ? (int)std::min<long long>(kRouteMaxWarps, (tokens + 31) / 32) : 1;
+  p.smem_per_query = route_smem_layout(D, (int)cmax, beam, rows, wide ? kRouteMaxWarps : 1).total;
+  p.fused = p.smem_per_query <= kRouteSmemCap;
+  return p;
+}
+
+cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
+                          int q_heads, int nq, int beam, const void* d_K, const void* d_V,
+                          float scale, int* d_leaf_idx, float* d_leaf_score, void* d_O,
+                          zha_dtype o_dtype, cudaStream_t stream) {
+  RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, nullptr);
+  const int D = t->desc.head_dim;
+  const bool bf = t->desc.kv_dtype == ZHA_BF16;
+  a.rows_bytes = (int)p.rows_bytes;
+  a.K = static_cast<const char*>(d_K);
+  a.V = static_cast<const char*>(d_V);
+  a.kv_unit_stride = t->desc.capacity_tokens * D * (bf ? 2LL : 4LL);
+  a.lb = t->desc.leaf_block;
+  a.N = t->N;
+  a.qk_scale = scale * 1.4426950408889634f;
+  a.stage_tokens = p.stage_tokens;
+  a.O = d_O;
+  a.o_bf16 = o_dtype == ZHA_BF16;
+  a.query_smem_bytes = (int)p.smem_per_query;  // weight area sized for 16 warps when wide
+  const StagedShape sh = staged_shape(t, a, p.smem_per_query, p.attn_warps);
+  cudaError_t e;
+  if (bf)
+    e = sh.wide ? run_route_tma_d<true, uint16_t>(D, a, sh.blocks, sh.threads, sh.smem, stream)
+                : run_route_tma_d<false, uint16_t>(D, a, sh.blocks, sh.threads, sh.smem, stream);
+  else
+    e = sh.wide ? run_route_tma_d<true, float>(D, a, sh.blocks, sh.threads, sh.smem, stream)
+                : run_route_tma_d<false, float>(D, a, sh.blocks, sh.threads, sh.smem, stream);
   ++t->launches;
   return e;
 }

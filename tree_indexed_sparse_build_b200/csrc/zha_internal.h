@@ -70,6 +70,21 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
                          int nq, int beam, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
                          cudaStream_t stream);
 
+// Fused route + attention (route.cu): one launch routes each query and attends over its
+// leaves.  fused == false when a query's widest level does not fit the staged kernel.
+struct DecodePlan {
+  bool fused;
+  size_t rows_bytes;      // candidate-row / K-V stage region per query
+  int stage_tokens;       // tokens per stage buffer (two buffers)
+  int attn_warps;         // warps per query the attention wants (wide launches)
+  size_t smem_per_query;
+};
+DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam);
+cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
+                          int q_heads, int nq, int beam, const void* d_K, const void* d_V,
+                          float scale, int* d_leaf_idx, float* d_leaf_score, void* d_O,
+                          zha_dtype o_dtype, cudaStream_t stream);
+
 // Attention (attend.cu).
 struct AttnPlan {
   int leaves_per_split;
@@ -80,7 +95,8 @@ struct AttnPlan {
   size_t smem_bytes;
   size_t scratch_bytes;
 };
-AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam);
+constexpr int kMaxClusterSplits = 8;  // splits of one query merged inside a cluster
+AttnPlan plan_attention(const zha_tree* t, int q_heads, int nq, int beam, int max_splits = 1 << 30);
 cudaError_t launch_attention(zha_tree* t, const AttnPlan& plan, const void* d_Q,
                              zha_dtype q_dtype, int q_heads, int nq, const void* d_K,
                              const void* d_V, const int* d_leaf_idx, int beam, float scale,
