@@ -182,10 +182,13 @@ def kernel_traffic(kernel: str):
     try:
         with open(path) as f:
             rec = json.load(f).get(kernel)
-        src = os.path.join(ROOT, "tree_indexed_sparse_build_b200", "csrc", rec["source"])
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
-                return None
+        srcs = rec["source"] if isinstance(rec["source"], list) else [rec["source"]]
+        h = hashlib.sha256()
+        for name in srcs:  # the kernel's source files, hashed in the listed order
+            with open(os.path.join(ROOT, "tree_indexed_sparse_build_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["sha256"]:
+            return None
         return rec["dram_bytes_per_launch"]
     except Exception:
         return None
@@ -198,13 +201,15 @@ def _graph_events(n):
     return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
 
-def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
+def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call=False):
     """128K decode steps: append 1 token + route + attend, one CUDA graph per step.
 
-    Timed pass (the bench value): steps W .. W+K-1, each graph bracketed by a start and an
-    end event only.  Kernel pass (per-call times for the roofline): steps W+K .. W+2K-1
-    with events between the calls as well (extra graph nodes between the kernels cost a
-    few microseconds, which is why they stay out of the timed pass).
+    The route and the attention run as one fused launch (zha_decode), or, with two_call,
+    as zha_route followed by zha_sparse_attn_decode.  Timed pass (the bench value): steps
+    W .. W+K-1, each graph bracketed by a start and an end event only.  Kernel pass
+    (per-call times for the roofline): steps W+K .. W+2K-1 with events between the calls as
+    well (extra graph nodes between the kernels cost a few microseconds, which is why they
+    stay out of the timed pass).
     """
     import torch
     from tree_indexed_sparse_build_b200 import synth, zha
@@ -225,23 +230,27 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
     traces = [torch.empty((B, Hq, nq, Ls[s], beam), dtype=torch.int32, device=dev)
               for s in range(2 * K)]
     Ow = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
+    Iw = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=dev)
     for s in range(W):
         tree.append(Kd, N + s + 1)
-        i, _, _ = tree.route(Qd[s], beam)
-        tree.attend(Qd[s], Kd, Vd, i, beam, w.scale, O=Ow)
+        zha.zha_decode(tree.handle, Qd[s], beam, Kd, Vd, w.scale, Iw, Ow)
     torch.cuda.synchronize()
 
+    def route_attend(Q, ix, out, tr):
+        if two_call:
+            zha.zha_route(tree.handle, Q, beam, ix, None, tr)
+            zha.zha_sparse_attn_decode(tree.handle, Q, Kd, Vd, ix, beam, w.scale, out, scratch)
+        else:
+            zha.zha_decode(tree.handle, Q, beam, Kd, Vd, w.scale, ix, out, None, tr)
+
     def one_step(s, e):
-        """Step W+s; e = [start, end] or [start, after append, after route, end]."""
+        """Step W+s; e = [start, end] or [start, after append, end]."""
         st = W + s
         e[0].record()
         zha.zha_tree_append(tree.handle, Kd, N + st + 1)
-        if len(e) == 4:
+        if len(e) == 3:
             e[1].record()
-        zha.zha_route(tree.handle, Qd[st], beam, idx[s], None, traces[s])
-        if len(e) == 4:
-            e[2].record()
-        zha.zha_sparse_attn_decode(tree.handle, Qd[st], Kd, Vd, idx[s], beam, w.scale, O[s], scratch)
+        route_attend(Qd[st], idx[s], O[s], traces[s])
         e[-1].record()
 
     def make(nev):
@@ -280,14 +289,14 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
     # kernel pass
     inner, graphs2 = [], []
     if eager:
-        inner = [make(4) for _ in range(K)]
+        inner = [make(3) for _ in range(K)]
         for s in range(K):
             flush.zero_()
             one_step(K + s, inner[s])
         torch.cuda.synchronize()
     else:
         for s in range(K):
-            e = make(4)
+            e = make(3)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
                 one_step(K + s, e)
@@ -299,8 +308,7 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
             graphs2[s].replay()
         torch.cuda.synchronize()
     t_app = np.array([inner[s][0].elapsed_time(inner[s][1]) for s in range(K)])
-    t_rte = np.array([inner[s][1].elapsed_time(inner[s][2]) for s in range(K)])
-    t_att = np.array([inner[s][2].elapsed_time(inner[s][3]) for s in range(K)])
+    t_dec = np.array([inner[s][1].elapsed_time(inner[s][2]) for s in range(K)])
     assert tree.check() == zha.ZHA_OK, "device error word set during the timed steps"
 
     idx_n, tr_n = idx.cpu().numpy(), [t.cpu().numpy() for t in traces]
@@ -312,7 +320,7 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
         for k in acc:
             acc[k] += pb[k] / K
     del graphs, graphs2
-    res = {"step_ms": t_step, "append_ms": t_app, "route_ms": t_rte, "attend_ms": t_att,
+    res = {"step_ms": t_step, "append_ms": t_app, "decode_ms": t_dec,
            "queries_per_step": B * Hq * nq, "launches_per_step": launches, "clocks": smp.summary(),
            **acc}
 
@@ -333,8 +341,7 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False):
         Vd[:, :, pos].copy_(hv[:, :, s], non_blocking=True)
         qbuf.copy_(hq[s], non_blocking=True)
         tree.append(Kd, pos + 1)
-        zha.zha_route(tree.handle, qbuf, beam, ibuf)
-        zha.zha_sparse_attn_decode(tree.handle, qbuf, Kd, Vd, ibuf, beam, w.scale, obuf, scratch)
+        route_attend(qbuf, ibuf, obuf, None)
         if out_slot is not None:
             ho[out_slot].copy_(obuf, non_blocking=True)
         torch.cuda.current_stream().synchronize()
@@ -384,17 +391,20 @@ def run_1m(W, K, rank, dev, flush, eager=False):
         scratch = tree.scratch_for(w.q_heads, nq, beam, dev)
 
         def one_step(e):
-            """route + attend; e = [start, end] or [start, after route, end]."""
+            """e = [start, end]: the fused call (zha_decode); e = [start, after route, end]:
+            zha_route then zha_sparse_attn_decode, for the per-call breakdown."""
             e[0].record()
-            zha.zha_route(tree.handle, Q, beam, idx, None, tr)
-            if len(e) == 3:
+            if len(e) == 2:
+                zha.zha_decode(tree.handle, Q, beam, Kd, Vd, w.scale, idx, O, None, tr)
+            else:
+                zha.zha_route(tree.handle, Q, beam, idx, None, tr)
                 e[1].record()
-            zha.zha_sparse_attn_decode(tree.handle, Q, Kd, Vd, idx, beam, w.scale, O, scratch)
+                zha.zha_sparse_attn_decode(tree.handle, Q, Kd, Vd, idx, beam, w.scale, O, scratch)
             e[-1].record()
 
         runs = {}
-        l0 = tree.launches
-        for nev in (2, 3):  # timed (start/end only), then per-call times
+        for nev in (2, 3):  # fused (the bench figure), then the two-call breakdown
+            l0 = tree.launches
             if eager:
                 e = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
                 runs[nev] = (e, (lambda e=e: one_step(e)))
@@ -404,9 +414,10 @@ def run_1m(W, K, rank, dev, flush, eager=False):
                 with torch.cuda.graph(g, stream=torch.cuda.Stream(), capture_error_mode="thread_local"):
                     one_step(e)
                 runs[nev] = (e, g.replay, g)
-        launches = (tree.launches - l0) // 2
+            if nev == 2:
+                launches = tree.launches - l0
         times = {}
-        for nev in (2, 3):
+        for nev in (3, 2):
             e, run = runs[nev][0], runs[nev][1]
             for _ in range(W):
                 run()
@@ -433,7 +444,7 @@ def run_1m(W, K, rank, dev, flush, eager=False):
 
 def run_build_256k(W, K, dev, flush):
     """256K cache: build from scratch, append 4,096 tokens in one call, route + attend 64
-    queries per head."""
+    queries per head (one zha_decode call)."""
     import torch
     from tree_indexed_sparse_build_b200 import synth, workloads, zha
 
@@ -458,8 +469,7 @@ def run_build_256k(W, K, dev, flush):
         ev[3].record()
         flush.zero_()
         ev[4].record()
-        idx, _, _ = tree.route(Qd, w.beam)
-        tree.attend(Qd, Kd, Vd, idx, w.beam, w.scale)
+        tree.decode(Qd, Kd, Vd, w.beam, w.scale)
         ev[5].record()
         torch.cuda.synchronize()
         if it >= W:
@@ -549,6 +559,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-1m", action="store_true")
     ap.add_argument("--no-build", action="store_true")
+    ap.add_argument("--two-call", action="store_true",
+                    help="decode steps as zha_route + zha_sparse_attn_decode instead of zha_decode")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--eager", action="store_true",
                     help="launch the same kernels without CUDA graphs (for profilers)")
@@ -601,7 +613,7 @@ def main():
 
     barrier()
     torch.cuda.synchronize()
-    r = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager)
+    r = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager, two_call=args.two_call)
     torch.cuda.synchronize()
     barrier()
 
@@ -609,17 +621,16 @@ def main():
     step_ms = max_over_ranks(float(r["step_ms"].mean()))
     qps = r["queries_per_step"] * world / (step_ms * 1e-3)
     e2e_ms = max_over_ranks(r["e2e_ms_per_step"])
-    kern = {}
-    for name, ms_key, b_key in (("route", "route_ms", "route_bytes"),
-                                ("attend", "attend_ms", "attend_bytes")):
-        ms = float(r[ms_key].mean())
-        kern[name] = {"ms": ms, "bytes": int(r[b_key]), "gbs": r[b_key] / (ms * 1e-3) / 1e9}
-    kern["append"] = {"ms": float(r["append_ms"].mean())}
-    dom = max(("route", "attend"), key=lambda k: kern[k]["ms"])
-    dom_kernel = {"route": "route_tma_kernel", "attend": "attend_kernel"}[dom]
+    # route + attention: one fused launch (route_tma_kernel with its attention epilogue), or
+    # the two calls' combined time with --two-call
+    dec_ms = float(r["decode_ms"].mean())
     ra_bytes = r["route_bytes"] + r["attend_bytes"]
-    ra_ms = float((r["route_ms"] + r["attend_ms"]).mean())
-
+    dom_kernel = "route_tma_kernel+attend_kernel" if args.two_call else "route_tma_kernel (fused decode)"
+    kern = {"decode": {"ms": dec_ms, "bytes": int(ra_bytes), "gbs": ra_bytes / (dec_ms * 1e-3) / 1e9,
+                       "route_bytes": int(r["route_bytes"]), "attend_bytes": int(r["attend_bytes"])},
+            "append": {"ms": float(r["append_ms"].mean())}}
+    dom = "decode"
+    ra_ms = dec_ms
     line = {
         "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -627,7 +638,8 @@ def main():
         "config": workload_config(w),
         "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": kern[dom]["gbs"],
                      "peak": peak, "unit": "GB/s", "frac": kern[dom]["gbs"] / peak,
-                     "traffic": kernel_traffic(dom_kernel), "peak_source": peak_kind,
+                     "traffic": None if args.two_call else kernel_traffic("decode_fused"),
+                     "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": kern[dom]["bytes"]},
         "route_attend": {"gbs": ra_bytes / (ra_ms * 1e-3) / 1e9, "frac": ra_bytes / (ra_ms * 1e-3) / 1e9 / peak,
                          "ms": ra_ms, "bytes": int(ra_bytes)},
@@ -638,6 +650,7 @@ def main():
                 "d2h_bytes_per_step": r["d2h_bytes_per_step"]},
         "gpu_launches": int(round(r["launches_per_step"] * K)),
         "launch_mode": "eager" if args.eager else "cuda_graph_per_step",
+        "decode_call": "zha_route + zha_sparse_attn_decode" if args.two_call else "zha_decode (fused)",
         "clocks": r["clocks"],
     }
 

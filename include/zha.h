@@ -158,6 +158,7 @@ size_t zha_noalloc_scratch_capacity(void);
  * list or partials pass through global memory).  Arguments as in those two calls:
  *   d_leaf_idx    out [batch, q_heads, nq, beam] int32, required: the selected leaves
  *   d_leaf_score  out, nullable: their scores
+ *   d_trace       out, nullable: the nodes kept per level, as in zha_route
  *   d_O           out [batch, q_heads, nq, head_dim] in o_dtype
  * Same constraints (q_heads % kv_heads == 0, 1 <= beam <= 1024, beam * branching <= 4096,
  * non-empty tree).  Needs no scratch.  When a query's widest level is too large to
@@ -166,7 +167,8 @@ size_t zha_noalloc_scratch_capacity(void);
  * ZHA_ERR_UNSUPPORTED if that attention would need scratch (use the two calls then). */
 zha_status zha_decode(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
                       int beam, const void* d_K, const void* d_V, float scale, int* d_leaf_idx,
-                      float* d_leaf_score, void* d_O, zha_dtype o_dtype, void* stream);
+                      float* d_leaf_score, int* d_trace, void* d_O, zha_dtype o_dtype,
+                      void* stream);
 
 /* Synchronizes `stream`, then reads and clears the device error word:
  * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */

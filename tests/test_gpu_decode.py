@@ -36,17 +36,21 @@ def test_decode_matches_route_and_oracle(dev, w):
     from tree_indexed_sparse_build_b200 import zha
     tree, (Qn, Kn, Vn), (Q, K, V) = _setup(w, dev)
     tree.build(K, w.seq_len)
-    ridx, rsc, _ = tree.route(Q, w.beam, scores=True)
+    ridx, rsc, rtr = tree.route(Q, w.beam, scores=True, trace=True)
     l0 = tree.launches
-    O, idx, sc = tree.decode(Q, K, V, w.beam, w.scale, out_dtype=_odt(w), scores=True)
+    O, idx, sc, tr = tree.decode(Q, K, V, w.beam, w.scale, out_dtype=_odt(w), scores=True, trace=True)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_OK
     assert torch.equal(idx, ridx)
+    assert torch.equal(tr, rtr)
     assert torch.equal(sc.nan_to_num(-7.0), rsc.nan_to_num(-7.0))
-    checked, ill, bad = _route_compare(tree, w, Qn, Kn, idx, None, w.seq_len)
+    checked, ill, bad = _route_compare(tree, w, Qn, Kn, idx, tr, w.seq_len)
     assert checked > 0
     _attend_check(w, Qn, Kn, Vn, O, idx.cpu().numpy().astype(np.int64), w.seq_len)
     launches = tree.launches - l0
+    # one launch whenever the plan fuses (the wide cases and the short-leaf narrow one)
+    if w.name in ("f32_d64_b2", "bf16_d128_b16_splits", "bf16_d128_narrow_lb4"):
+        assert launches == 1
     print(f"{w.name}: launches {launches}, well-conditioned {checked}, ill {ill} ({bad} differ)")
 
 

@@ -54,6 +54,8 @@ CASES = [
     _wl("f32_d64_cluster", 2, 2, 8, 64, 3000, "f32", 4, 16, 8, 4, 115),
     # widest level (beam * b = 512 rows) too large to stage: register-batched route kernel
     _wl("bf16_d128_regpath", 1, 1, 2, 128, 20000, "bf16", 8, 4, 64, 2, 112),
+    # many queries with short leaf lists (the 1M shape): narrow launch, attention fused
+    _wl("bf16_d128_narrow_lb4", 1, 2, 16, 128, 20001, "bf16", 8, 4, 8, 32, 116),
 ]
 
 

@@ -946,10 +946,13 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   return e;
 }
 
-// Fused route + attention (one launch).  Row region per query: the widest level's rows,
-// or more when the attention wants bigger stages (wide: up to 128 KB, so a long leaf list
-// streams in a few large stages; narrow: up to 32 KB, so several queries still share an
-// SM), and never less than two stages of 8 tokens.
+// Fused route + attention (one launch).  Wide launches (one query per CTA): the row
+// region grows up to 128 KB when the attention wants bigger stages, so a long leaf list
+// streams in a few large stages.  Narrow launches (several queries per SM): the row region
+// stays the route's own, since a larger one would cut the queries resident per SM, and the
+// call is fused only when the query's tokens then fit in at most two stages; otherwise
+// fused = false and the route and the attention run as two launches.  Stages hold at
+// least 8 tokens.
 DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
   DecodePlan p{};
   const int D = t->desc.head_dim;
@@ -961,23 +964,22 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
     cmax = std::max(cmax, std::min(std::min((long long)beam, t->n[l + 1]) * t->desc.branching, t->n[l]));
   const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
   const size_t route_rows = route_rows_bytes(D, (int)cmax);
-  const size_t want = (size_t)4 * row * (size_t)((tokens + 1) / 2);
-  const size_t cap = wide ? 128 * 1024 : 32 * 1024;
-  size_t rows = std::max(route_rows, std::min(want, cap));
+  const size_t want = (size_t)4 * row * (size_t)((tokens + 1) / 2);  // two stages
+  size_t rows = wide ? std::max(route_rows, std::min(want, (size_t)128 * 1024)) : route_rows;
   rows = std::max(rows, (size_t)4 * 8 * row);
   p.stage_tokens = (int)(rows / (4 * row)) / 8 * 8;
   p.rows_bytes = rows;
   p.attn_warps = wide ? (int)std::min<long long>(kRouteMaxWarps, (tokens + 31) / 32) : 1;
   p.smem_per_query = route_smem_layout(D, (int)cmax, beam, rows, wide ? kRouteMaxWarps : 1).total;
-  p.fused = p.smem_per_query <= kRouteSmemCap;
+  p.fused = p.smem_per_query <= kRouteSmemCap && (wide || 2LL * p.stage_tokens >= tokens);
   return p;
 }
 
 cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
                           int q_heads, int nq, int beam, const void* d_K, const void* d_V,
-                          float scale, int* d_leaf_idx, float* d_leaf_score, void* d_O,
-                          zha_dtype o_dtype, cudaStream_t stream) {
-  RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, nullptr);
+                          float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
+                          void* d_O, zha_dtype o_dtype, cudaStream_t stream) {
+  RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, d_trace);
   const int D = t->desc.head_dim;
   const bool bf = t->desc.kv_dtype == ZHA_BF16;
   a.rows_bytes = (int)p.rows_bytes;

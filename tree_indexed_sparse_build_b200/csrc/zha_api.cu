@@ -175,7 +175,8 @@ zha_status zha_sparse_attn_decode(const zha_tree* t, const void* d_Q, zha_dtype 
 
 zha_status zha_decode(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
                       int beam, const void* d_K, const void* d_V, float scale, int* d_leaf_idx,
-                      float* d_leaf_score, void* d_O, zha_dtype o_dtype, void* stream) {
+                      float* d_leaf_score, int* d_trace, void* d_O, zha_dtype o_dtype,
+                      void* stream) {
   if (!t || !dtype_ok(q_dtype) || !dtype_ok(o_dtype) || q_heads < 1 || nq < 0)
     return ZHA_ERR_INVALID_ARG;
   if (q_heads % t->desc.kv_heads != 0) return ZHA_ERR_INVALID_ARG;
@@ -186,19 +187,20 @@ zha_status zha_decode(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int
   if (nq == 0) return ZHA_OK;
   if (!d_Q || !d_K || !d_V || !d_leaf_idx || !d_O) return ZHA_ERR_INVALID_ARG;
   if (!aligned(d_Q, 16) || !aligned(d_K, 16) || !aligned(d_V, 16) || !aligned(d_O, 16) ||
-      !aligned(d_leaf_idx, 4) || (d_leaf_score && !aligned(d_leaf_score, 4)))
+      !aligned(d_leaf_idx, 4) || (d_leaf_score && !aligned(d_leaf_score, 4)) ||
+      (d_trace && !aligned(d_trace, 4)))
     return ZHA_ERR_INVALID_ARG;
   zha_tree* tm = const_cast<zha_tree*>(t);  // only the launch counter moves
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const DecodePlan dp = plan_decode(t, q_heads, nq, beam);
   if (dp.fused)
     return cuda_status(launch_decode(tm, dp, d_Q, q_dtype, q_heads, nq, beam, d_K, d_V, scale,
-                                     d_leaf_idx, d_leaf_score, d_O, o_dtype, s));
+                                     d_leaf_idx, d_leaf_score, d_trace, d_O, o_dtype, s));
   // Levels too wide for the staged kernel: route, then attention with splits merged
   // inside clusters (no scratch).
   const AttnPlan ap = plan_attention(t, q_heads, nq, beam, kMaxClusterSplits);
   if (ap.smem_bytes > 227 * 1024 || ap.scratch_bytes > 0) return ZHA_ERR_UNSUPPORTED;
-  cudaError_t e = launch_route(tm, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, nullptr, s);
+  cudaError_t e = launch_route(tm, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, d_trace, s);
   if (e != cudaSuccess) return ZHA_ERR_CUDA;
   return cuda_status(launch_attention(tm, ap, d_Q, q_dtype, q_heads, nq, d_K, d_V, d_leaf_idx, beam,
                                       scale, d_O, o_dtype, nullptr, s));

@@ -82,8 +82,8 @@ struct DecodePlan {
 DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam);
 cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
                           int q_heads, int nq, int beam, const void* d_K, const void* d_V,
-                          float scale, int* d_leaf_idx, float* d_leaf_score, void* d_O,
-                          zha_dtype o_dtype, cudaStream_t stream);
+                          float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
+                          void* d_O, zha_dtype o_dtype, cudaStream_t stream);
 
 // Attention (attend.cu).
 struct AttnPlan {

@@ -68,7 +68,8 @@ def lib() -> ctypes.CDLL:
             "zha_sparse_attn_decode_noalloc": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _I,
                                                     ctypes.c_float, _P, _I, _P]),
             "zha_noalloc_scratch_capacity": (_SZ, []),
-            "zha_decode": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, _P, _I, _P]),
+            "zha_decode": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P, _I,
+                                _P]),
             "zha_tree_check": (_I, [_P, _P]),
             "zha_tree_seq_len": (_LL, [_P]),
             "zha_tree_levels": (_I, [_P]),
@@ -182,12 +183,12 @@ def zha_sparse_attn_decode_noalloc(handle, Q: torch.Tensor, K: torch.Tensor, V: 
 
 def zha_decode(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: torch.Tensor, scale: float,
                leaf_idx: torch.Tensor, O: torch.Tensor, leaf_score: torch.Tensor | None = None,
-               stream=None) -> None:
+               trace: torch.Tensor | None = None, stream=None) -> None:
     """Route + attention in one call (one launch when the levels fit shared memory)."""
     B, Hq, nq, _ = Q.shape
     _check(lib().zha_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
-                            scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(O), dtype_code(O.dtype),
-                            _stream(stream)), "zha_decode")
+                            scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _ptr(O),
+                            dtype_code(O.dtype), _stream(stream)), "zha_decode")
 
 
 def zha_noalloc_scratch_capacity() -> int:
@@ -311,14 +312,18 @@ class Tree:
         return O
 
     def decode(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, beam: int, scale: float,
-               out_dtype: torch.dtype = torch.bfloat16, scores: bool = False, stream=None):
-        """Route + attention in one call; returns (O, leaf_idx, leaf_score or None)."""
+               out_dtype: torch.dtype = torch.bfloat16, scores: bool = False, trace: bool = False,
+               stream=None):
+        """Route + attention in one call; returns (O, leaf_idx, leaf_score or None), plus the
+        per-level trace when trace=True."""
         B, Hq, nq, d = Q.shape
         idx = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=Q.device)
         sc = torch.empty((B, Hq, nq, beam), dtype=torch.float32, device=Q.device) if scores else None
+        tr = (torch.empty((B, Hq, nq, max(self.levels, 1), beam), dtype=torch.int32, device=Q.device)
+              if trace else None)
         O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
-        zha_decode(self.handle, Q, beam, K, V, scale, idx, O, sc, stream)
-        return O, idx, sc
+        zha_decode(self.handle, Q, beam, K, V, scale, idx, O, sc, tr, stream)
+        return (O, idx, sc, tr) if trace else (O, idx, sc)
 
     def check(self, stream=None) -> int:
         return zha_tree_check(self.handle, stream)
