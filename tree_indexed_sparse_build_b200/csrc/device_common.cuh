@@ -119,6 +119,38 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 
 namespace zha {
 
+// Named CTA barriers over a group of warps: barrier `id` (1..15) with `nthreads` threads (a
+// multiple of 32, every thread of the group arrives).  Used when several queries share a
+// CTA and each query owns a group of warps.
+__device__ __forceinline__ void group_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Number of threads of the group with p true (a barrier as well).
+__device__ __forceinline__ int group_count(int id, int nthreads, bool p) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.popc.u32 %0, %2, %3, q;\n\t}"
+      : "=r"(r)
+      : "r"((int)p), "r"(id), "r"(nthreads)
+      : "memory");
+  return r;
+}
+// True if p holds for any thread of the group (a barrier as well).
+__device__ __forceinline__ bool group_any(int id, int nthreads, bool p) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred q, o;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred o, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, o;\n\t}"
+      : "=r"(r)
+      : "r"((int)p), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialization may start while the previous kernel in the stream is still running;
 // pdl_wait() blocks until that kernel has completed and its writes are visible, so it

@@ -447,14 +447,69 @@ __device__ __forceinline__ int select_compact(const unsigned long long* keys, co
   return kept;
 }
 
-// Whole-CTA variant for one query per CTA with C <= blockDim.x: thread t holds candidate t.
-// The threshold search counts with __syncthreads_count (one CTA barrier per bit); the kept
+// Rank selection for small levels (C <= 64 nw, at most two candidates per thread of the
+// query's nw warps): a key is kept iff fewer than `beam` keys of the level are greater
+// (keys are distinct, so exactly min(C, beam) are kept).  Each thread counts for its
+// candidates k = t and t + 32 nw against every key, reading two keys per 16-byte
+// shared-memory load; no barrier per bit, and every warp of the query takes part.  The
+// kept candidates are compacted in candidate order by per-warp ballots.  keys must be
+// 16-byte aligned.  Every thread of the group must call it.  Returns the number kept.
+__device__ __forceinline__ int select_rank_group(const unsigned long long* keys, const int* cand,
+                                                 int C, int beam, int* nxt, float* leaf_sc,
+                                                 bool leaf, unsigned* red, int wq, int lane, int nw,
+                                                 int bar_id) {
+  const int nt = 32 * nw;
+  int kept_before = 0;  // kept candidates of earlier passes
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int k = 32 * wq + lane + pass * nt;
+    if (pass == 1 && C <= nt) break;  // C is the same for the whole group
+    const bool have = k < C;
+    const unsigned long long key = have ? keys[k] : 0ull;
+    int rank = 0;
+    if (have && C > beam) {
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
+      int j = 0;
+#pragma unroll 4
+      for (; j + 1 < C; j += 2) {
+        const ulonglong2 v = k2[j >> 1];
+        rank += (v.x > key ? 1 : 0) + (v.y > key ? 1 : 0);
+      }
+      if (j < C) rank += keys[j] > key ? 1 : 0;
+    }
+    const bool keep = have && rank < beam;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (nw > 1) {
+      if (lane == 0) red[32 + wq] = __popc(bal);
+      group_sync(bar_id, nt);
+    }
+    int pre = kept_before, all = kept_before;
+    for (int w = 0; w < nw; ++w) {
+      const int c = nw > 1 ? (int)red[32 + w] : __popc(bal);
+      if (w < wq) pre += c;
+      all += c;
+    }
+    if (keep) {
+      const int pos = pre + __popc(bal & ((1u << lane) - 1u));
+      nxt[pos] = cand[k];
+      if (leaf) leaf_sc[pos] = key_score(key);
+    }
+    if (nw > 1) group_sync(bar_id, nt);  // red is reused by the next pass
+    kept_before = all;
+  }
+  return min(C, beam);
+}
+
+// Warp-group variant for a query owning nw warps (C <= 32 nw): thread t = 32 wq + lane of
+// the group holds candidate t.  The threshold search counts with a group barrier reduction
+// (named barrier bar_id over the group's 32 nw threads; one barrier per bit); the kept
 // candidates are compacted in candidate order with per-warp ballots and a prefix over the
-// warps' counts.  Every thread of the CTA must call it.  Returns the number kept.
-__device__ __forceinline__ int select_compact_cta(const unsigned long long* keys, const int* cand,
-                                                  int C, int beam, int* nxt, float* leaf_sc,
-                                                  bool leaf, unsigned* red) {
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = (int)(blockDim.x >> 5);
+// warps' counts.  Every thread of the group must call it.  Returns the number kept.
+__device__ __forceinline__ int select_compact_group(const unsigned long long* keys, const int* cand,
+                                                    int C, int beam, int* nxt, float* leaf_sc,
+                                                    bool leaf, unsigned* red, int wq, int lane,
+                                                    int nw, int bar_id) {
+  const int t = 32 * wq + lane, nt = 32 * nw;
   const bool have = t < C;
   const unsigned long long key = have ? keys[t] : 0ull;
   const int node = have ? cand[t] : 0;
@@ -464,10 +519,10 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
     const uint32_t wmax = __reduce_max_sync(0xffffffffu, have ? h : 0u);
     const uint32_t wmin = __reduce_min_sync(0xffffffffu, have ? h : 0xFFFFFFFFu);
     if (lane == 0) {
-      red[warp] = wmax;
-      red[16 + warp] = wmin;
+      red[wq] = wmax;
+      red[16 + wq] = wmin;
     }
-    __syncthreads();
+    group_sync(bar_id, nt);
     uint32_t hmax = 0u, hmin = 0xFFFFFFFFu;
     for (int w = 0; w < nw; ++w) {
       hmax = max(hmax, red[w]);
@@ -479,7 +534,7 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
     bool done = false;
     for (int bit = top; bit >= 0; --bit) {
       const uint32_t c = Th | (1u << bit);
-      const int cnt = __syncthreads_count(have && h >= c);
+      const int cnt = group_count(bar_id, nt, have && h >= c);
       if (cnt >= beam) {
         Th = c;
         if (cnt == beam) {
@@ -491,11 +546,11 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
     if (done) {
       T = (unsigned long long)Th << 32;
     } else {
-      const int need = beam - __syncthreads_count(have && h > Th);
+      const int need = beam - group_count(bar_id, nt, have && h > Th);
       uint32_t Tl = 0u;
       for (int bit = 31; bit >= 0; --bit) {
         const uint32_t c = Tl | (1u << bit);
-        const int cnt = __syncthreads_count(have && h == Th && (uint32_t)key >= c);
+        const int cnt = group_count(bar_id, nt, have && h == Th && (uint32_t)key >= c);
         if (cnt >= need) {
           Tl = c;
           if (cnt == need) break;
@@ -506,10 +561,10 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
   }
   const bool keep = have && key >= T;
   const unsigned bal = __ballot_sync(0xffffffffu, keep);
-  if (lane == 0) red[32 + warp] = __popc(bal);
-  __syncthreads();
+  if (lane == 0) red[32 + wq] = __popc(bal);
+  group_sync(bar_id, nt);
   int pre = 0;
-  for (int w = 0; w < warp; ++w) pre += (int)red[32 + w];
+  for (int w = 0; w < wq; ++w) pre += (int)red[32 + w];
   if (keep) {
     const int pos = pre + __popc(bal & ((1u << lane) - 1u));
     nxt[pos] = node;
@@ -518,9 +573,9 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
   return min(C, beam);
 }
 
-// Staged routing.  WIDE: one query per CTA, blockDim.x = 32 * wpq, the query's warps
-// synchronised by CTA barriers.  Otherwise qpc queries per CTA with one warp each,
-// synchronised only within the warp.
+// Staged routing.  qpc queries per CTA, wpq warps per query (blockDim.x = 32 qpc wpq).
+// GROUPED (wpq > 1): the warps of query qi synchronise on named barrier 1 + qi; otherwise
+// each query is one warp, synchronised only within the warp.
 //
 // With TKV = the KV storage type (not NoKV) the kernel is the fused decode: once the
 // last level is selected, the query's warps attend over the tokens of its leaves.  The
@@ -529,20 +584,23 @@ __device__ __forceinline__ int select_compact_cta(const unsigned long long* keys
 // the online softmax of attn_core.cuh over each stage, merge their states through shared
 // memory and write O.  No leaf list goes through global memory and nothing is launched
 // between the route and the attention.
-template <int D, bool WIDE, typename TKV>
-__global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const RouteArgs a) {
+// NARROW instantiations are built for CTAs of at most 8 warps, three per SM (register cap).
+template <int D, bool GROUPED, typename TKV, bool NARROW>
+__global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3 : 1)
+    route_tma_kernel(const RouteArgs a) {
   constexpr bool ATTEND = !std::is_same<TKV, NoKV>::value;
   constexpr int CPL = D / 16;  // 16-byte chunks of a row per lane (4 lanes per row)
   constexpr int R = 8;         // candidate keys held per lane in the selecting warp
   extern __shared__ __align__(128) unsigned char rsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qi = WIDE ? 0 : warp;
-  const int wq = WIDE ? warp : 0;
-  const int nw = WIDE ? (int)(blockDim.x >> 5) : 1;
-  const long long qg = (long long)blockIdx.x * (WIDE ? 1 : a.qpc) + qi;
+  const int nw = GROUPED ? a.wpq : 1;  // warps of this query
+  const int qi = warp / nw;
+  const int wq = warp - qi * nw;
+  const int bar_id = 1 + qi, bar_n = 32 * nw;
+  const long long qg = (long long)blockIdx.x * a.qpc + qi;
   const bool valid = qg < a.total_queries;
   const RouteSmem Ls =
-      route_smem_layout(D, a.cmax, a.beam, (size_t)a.rows_bytes, ATTEND ? (WIDE ? a.wpq : 1) : 0);
+      route_smem_layout(D, a.cmax, a.beam, (size_t)a.rows_bytes, ATTEND ? nw : 0);
   unsigned char* base = rsm + (size_t)qi * a.query_smem_bytes;
   const float* rows = reinterpret_cast<const float*>(base + Ls.rows);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + Ls.keys);
@@ -553,8 +611,8 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + Ls.bar);
   unsigned* red = reinterpret_cast<unsigned*>(base + Ls.red);
 
-  auto group_sync = [&]() {
-    if (WIDE) __syncthreads(); else __syncwarp();
+  auto qsync = [&]() {  // all warps of this query
+    if (GROUPED) group_sync(bar_id, bar_n); else __syncwarp();
   };
   pdl_wait();
   pdl_release();
@@ -572,7 +630,7 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
     fence_mbar_init();
     surv_a[0] = 0;  // the root
   }
-  group_sync();
+  qsync();
 
   // Four lanes per row: lane (rg = lane / 4, sub = lane % 4) reads chunks 4 (j ^ par) + sub,
   // par = rg & 1, so the two rows of a shared-memory phase use opposite bank halves.
@@ -615,13 +673,13 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
       }
     }
     const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
-    const bool failed = WIDE ? (__syncthreads_or(!ok) != 0) : __any_sync(0xffffffffu, !ok);
+    const bool failed = GROUPED ? group_any(bar_id, bar_n, !ok) : __any_sync(0xffffffffu, !ok);
     if (failed) {
       if (wq == 0 && lane == 0 && C > 0)  // let the copies land before the CTA exits
         mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
       return;  // the whole group leaves together
     }
-    if (!WIDE) __syncwarp();  // candidate ids written by other lanes
+    if (!GROUPED) __syncwarp();  // candidate ids written by other lanes
     if (C > 0) parity ^= 1u;
 
     // score: rows r = 8 (wq + nw t) + rg, two rows per lane in flight
@@ -653,10 +711,19 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
         if (sub == 0 && r < C) keys[r] = route_key(s, cand[r]);
       }
     }
-    group_sync();
-    if (WIDE && C > 64 && C <= 32 * nw) {  // C is the same for the whole CTA
-      const int kept = select_compact_cta(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red);
-      __syncthreads();
+    qsync();
+    if (C > 0 && C <= 128 && C <= 64 * nw) {  // C is the same for the whole group
+      const int kept =
+          select_rank_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red, wq, lane, nw, bar_id);
+      qsync();
+      if (wq == 0 && a.trace && valid) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
+      }
+    } else if (GROUPED && C <= 32 * nw) {
+      const int kept =
+          select_compact_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red, wq, lane, nw, bar_id);
+      group_sync(bar_id, bar_n);
       if (wq == 0 && a.trace && valid) {
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
         for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
@@ -672,7 +739,7 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
       }
     }
     m = min(C, a.beam);
-    group_sync();
+    qsync();
     int* tmp = cur;
     cur = nxt;
     nxt = tmp;
@@ -739,7 +806,7 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
       const bool ok = mbar_wait_bounded(&bar[b], phase(st), a.err, kDevErrTimeout, kRouteWaitCycles);
       // the stage is visible to every warp, and every warp is done with stage st - 1, whose
       // buffer the copy of stage st + 1 now reuses
-      const bool bad = WIDE ? (__syncthreads_or(!ok) != 0) : __any_sync(0xffffffffu, !ok);
+      const bool bad = GROUPED ? group_any(bar_id, bar_n, !ok) : __any_sync(0xffffffffu, !ok);
       if (bad) {
         fail_st = st;
         break;
@@ -767,19 +834,19 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
       return;
     }
     l_w = warp_sum(l_w);
-    if (WIDE) {
+    if (GROUPED) {
       // merge the warps' states; the accumulators reuse the stage buffers
       float* accr = reinterpret_cast<float*>(sb);
       float* redf = reinterpret_cast<float*>(red);
-      __syncthreads();
+      group_sync(bar_id, bar_n);
 #pragma unroll
       for (int e = 0; e < S::DPL; ++e) accr[wq * D + lane * S::DPL + e] = acc[e];
       if (lane == 0) {
         redf[wq] = m_w;
         redf[16 + wq] = l_w;
       }
-      __syncthreads();
-      for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      group_sync(bar_id, bar_n);
+      for (int d = 32 * wq + lane; d < D && valid; d += bar_n) {
         float M = -INFINITY;
         for (int w = 0; w < nw; ++w) M = fmaxf(M, redf[w]);
         float o = 0.f, l = 0.f;
@@ -809,10 +876,10 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_tma_kernel(const Ro
 }
 
 namespace {
-template <int D, bool WIDE, typename TKV>
+template <int D, bool GROUPED, typename TKV, bool NARROW>
 cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
                           cudaStream_t s) {
-  auto kern = route_tma_kernel<D, WIDE, TKV>;
+  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
@@ -820,11 +887,21 @@ cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size
   return cudaGetLastError();
 }
 
-template <bool WIDE, typename TKV>
-cudaError_t run_route_tma_d(int D, const RouteArgs& a, unsigned blocks, int threads, size_t smem,
-                            cudaStream_t s) {
-  return D == 128 ? run_route_tma<128, WIDE, TKV>(a, blocks, threads, smem, s)
-                  : run_route_tma<64, WIDE, TKV>(a, blocks, threads, smem, s);
+template <typename TKV>
+cudaError_t run_route_tma_d(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                            int threads, size_t smem, cudaStream_t s) {
+  if (narrow) {
+    if (grouped)
+      return D == 128 ? run_route_tma<128, true, TKV, true>(a, blocks, threads, smem, s)
+                      : run_route_tma<64, true, TKV, true>(a, blocks, threads, smem, s);
+    return D == 128 ? run_route_tma<128, false, TKV, true>(a, blocks, threads, smem, s)
+                    : run_route_tma<64, false, TKV, true>(a, blocks, threads, smem, s);
+  }
+  if (grouped)
+    return D == 128 ? run_route_tma<128, true, TKV, false>(a, blocks, threads, smem, s)
+                    : run_route_tma<64, true, TKV, false>(a, blocks, threads, smem, s);
+  return D == 128 ? run_route_tma<128, false, TKV, false>(a, blocks, threads, smem, s)
+                  : run_route_tma<64, false, TKV, false>(a, blocks, threads, smem, s);
 }
 
 template <int D, int U>
@@ -872,11 +949,21 @@ RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int 
   return a;
 }
 
+// Warps per query in narrow launches: enough that each warp scores about 16 rows of the
+// widest level (at most 4).
+#ifndef ZHA_NARROW_WPQ
+#define ZHA_NARROW_WPQ 0  // 0: by the widest level; else a fixed count (1, 2 or 4)
+#endif
+int narrow_wpq(long long cmax) {
+  if (ZHA_NARROW_WPQ > 0) return ZHA_NARROW_WPQ;
+  return (int)std::min<long long>(4, std::max<long long>(1, (cmax + 15) / 16));
+}
+
 // Launch shape of the staged kernel.  Wide (at most two queries per SM): one query per
 // CTA, enough warps for the widest level (and, fused, for the attention tokens).
-// Narrow: up to 8 queries per CTA, one warp each.
+// Narrow: up to 8 warps per CTA, narrow_wpq warps per query.
 struct StagedShape {
-  bool wide;
+  bool wide, grouped;
   unsigned blocks;
   int threads;
   size_t smem;
@@ -889,15 +976,15 @@ StagedShape staged_shape(const zha_tree* t, RouteArgs& a, size_t per_query, int 
     a.wpq = (int)std::max(1LL, std::min<long long>(kRouteMaxWarps, want));
     a.qpc = 1;
     sh.blocks = (unsigned)a.total_queries;
-    sh.threads = 32 * a.wpq;
     sh.smem = per_query;
   } else {
-    a.wpq = 1;
-    a.qpc = (int)std::max<size_t>(1, std::min<size_t>(8, (96 * 1024) / per_query));
+    a.wpq = narrow_wpq(a.cmax);
+    a.qpc = (int)std::max<size_t>(1, std::min<size_t>(8 / a.wpq, (96 * 1024) / per_query));
     sh.blocks = (unsigned)((a.total_queries + a.qpc - 1) / a.qpc);
-    sh.threads = 32 * a.qpc;
     sh.smem = per_query * a.qpc;
   }
+  sh.threads = 32 * a.wpq * a.qpc;
+  sh.grouped = a.wpq > 1;
   return sh;
 }
 }  // namespace
@@ -917,8 +1004,7 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
     a.query_smem_bytes = (int)per_query;
     // 8 rows per warp step, two steps in flight
     const StagedShape sh = staged_shape(t, a, per_query, 0);
-    e = sh.wide ? run_route_tma_d<true, NoKV>(D, a, sh.blocks, sh.threads, sh.smem, stream)
-                : run_route_tma_d<false, NoKV>(D, a, sh.blocks, sh.threads, sh.smem, stream);
+    e = run_route_tma_d<NoKV>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream);
     ++t->launches;
     return e;
   }
@@ -970,7 +1056,8 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
   p.stage_tokens = (int)(rows / (4 * row)) / 8 * 8;
   p.rows_bytes = rows;
   p.attn_warps = wide ? (int)std::min<long long>(kRouteMaxWarps, (tokens + 31) / 32) : 1;
-  p.smem_per_query = route_smem_layout(D, (int)cmax, beam, rows, wide ? kRouteMaxWarps : 1).total;
+  p.smem_per_query =
+      route_smem_layout(D, (int)cmax, beam, rows, wide ? kRouteMaxWarps : narrow_wpq(cmax)).total;
   p.fused = p.smem_per_query <= kRouteSmemCap && (wide || 2LL * p.stage_tokens >= tokens);
   return p;
 }
@@ -996,11 +1083,9 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
   const StagedShape sh = staged_shape(t, a, p.smem_per_query, p.attn_warps);
   cudaError_t e;
   if (bf)
-    e = sh.wide ? run_route_tma_d<true, uint16_t>(D, a, sh.blocks, sh.threads, sh.smem, stream)
-                : run_route_tma_d<false, uint16_t>(D, a, sh.blocks, sh.threads, sh.smem, stream);
+    e = run_route_tma_d<uint16_t>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream);
   else
-    e = sh.wide ? run_route_tma_d<true, float>(D, a, sh.blocks, sh.threads, sh.smem, stream)
-                : run_route_tma_d<false, float>(D, a, sh.blocks, sh.threads, sh.smem, stream);
+    e = run_route_tma_d<float>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream);
   ++t->launches;
   return e;
 }
