@@ -59,6 +59,22 @@ def level_counts(N: int, lb: int, b: int) -> list[int]:
     return out
 
 
+def append_bytes(N_new: int, lb: int, b: int, d: int, kv_bytes: int, units: int) -> int:
+    """Algorithmic bytes of a one-leaf append that ends at N_new tokens: per unit, the
+    touched leaf's tokens and, at every level above, the stored children of the path node
+    are read; the L + 1 path rows (fp32) are written."""
+    counts = level_counts(N_new, lb, b)
+    L = len(counts) - 1
+    leaf = (N_new - 1) // lb
+    per_unit = (N_new - leaf * lb) * d * kv_bytes
+    node = leaf
+    for lvl in range(1, L + 1):
+        node //= b
+        per_unit += (min(node * b + b, counts[lvl - 1]) - node * b) * d * 4
+    per_unit += (L + 1) * d * 4
+    return per_unit * units
+
+
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -201,15 +217,16 @@ def _graph_events(n):
     return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
 
-def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call=False):
+def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="step"):
     """128K decode steps: append 1 token + route + attend, one CUDA graph per step.
 
-    The route and the attention run as one fused launch (zha_decode), or, with two_call,
-    as zha_route followed by zha_sparse_attn_decode.  Timed pass (the bench value): steps
-    W .. W+K-1, each graph bracketed by a start and an end event only.  Kernel pass
-    (per-call times for the roofline): steps W+K .. W+2K-1 with events between the calls as
-    well (extra graph nodes between the kernels cost a few microseconds, which is why they
-    stay out of the timed pass).
+    mode "step": one zha_decode_step launch per step (append, route and attention fused);
+    "decode": zha_tree_append then zha_decode; "two_call": zha_tree_append, zha_route,
+    zha_sparse_attn_decode.  Timed pass (the bench value): steps W .. W+K-1, each graph
+    bracketed by a start and an end event only.  Kernel pass (per-call times for the
+    roofline): steps W+K .. W+2K-1, with an event after the append as well in the modes that
+    launch it separately (extra graph nodes between the kernels cost a few microseconds,
+    which is why they stay out of the timed pass).
     """
     import torch
     from tree_indexed_sparse_build_b200 import synth, zha
@@ -232,12 +249,18 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call
     Ow = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
     Iw = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=dev)
     for s in range(W):
-        tree.append(Kd, N + s + 1)
-        zha.zha_decode(tree.handle, Qd[s], beam, Kd, Vd, w.scale, Iw, Ow)
+        zha.zha_decode_step(tree.handle, Kd, Vd, N + s + 1, Qd[s], beam, w.scale, Iw, Ow)
     torch.cuda.synchronize()
 
-    def route_attend(Q, ix, out, tr):
-        if two_call:
+    def decode_call(new_n, Q, ix, out, tr, e=None):
+        """The step's calls; e: record an event between the append and the rest."""
+        if mode == "step":
+            zha.zha_decode_step(tree.handle, Kd, Vd, new_n, Q, beam, w.scale, ix, out, None, tr)
+            return
+        zha.zha_tree_append(tree.handle, Kd, new_n)
+        if e is not None:
+            e.record()
+        if mode == "two_call":
             zha.zha_route(tree.handle, Q, beam, ix, None, tr)
             zha.zha_sparse_attn_decode(tree.handle, Q, Kd, Vd, ix, beam, w.scale, out, scratch)
         else:
@@ -247,10 +270,7 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call
         """Step W+s; e = [start, end] or [start, after append, end]."""
         st = W + s
         e[0].record()
-        zha.zha_tree_append(tree.handle, Kd, N + st + 1)
-        if len(e) == 3:
-            e[1].record()
-        route_attend(Qd[st], idx[s], O[s], traces[s])
+        decode_call(N + st + 1, Qd[st], idx[s], O[s], traces[s], e[1] if len(e) == 3 else None)
         e[-1].record()
 
     def make(nev):
@@ -287,16 +307,17 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call
     t_step = np.array([outer[s][0].elapsed_time(outer[s][1]) for s in range(K)])
 
     # kernel pass
+    n_in = 2 if mode == "step" else 3
     inner, graphs2 = [], []
     if eager:
-        inner = [make(3) for _ in range(K)]
+        inner = [make(n_in) for _ in range(K)]
         for s in range(K):
             flush.zero_()
             one_step(K + s, inner[s])
         torch.cuda.synchronize()
     else:
         for s in range(K):
-            e = make(3)
+            e = make(n_in)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
                 one_step(K + s, e)
@@ -307,17 +328,23 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call
             flush.zero_()
             graphs2[s].replay()
         torch.cuda.synchronize()
-    t_app = np.array([inner[s][0].elapsed_time(inner[s][1]) for s in range(K)])
-    t_dec = np.array([inner[s][1].elapsed_time(inner[s][2]) for s in range(K)])
+    if mode == "step":  # one launch: append, route and attention together
+        t_dec = np.array([inner[s][0].elapsed_time(inner[s][1]) for s in range(K)])
+        t_app = np.zeros(K)
+    else:
+        t_app = np.array([inner[s][0].elapsed_time(inner[s][1]) for s in range(K)])
+        t_dec = np.array([inner[s][1].elapsed_time(inner[s][2]) for s in range(K)])
     assert tree.check() == zha.ZHA_OK, "device error word set during the timed steps"
 
     idx_n, tr_n = idx.cpu().numpy(), [t.cpu().numpy() for t in traces]
-    acc = {"route_bytes": 0, "attend_bytes": 0, "summaries_per_query": 0.0, "keys_per_query": 0.0}
+    acc = {"route_bytes": 0, "attend_bytes": 0, "summaries_per_query": 0.0, "keys_per_query": 0.0,
+           "append_bytes": 0}
     for s in range(K, 2 * K):  # the kernel pass's calls, whose times the roofline uses
         Nst = N + W + s + 1
+        acc["append_bytes"] += append_bytes(Nst, w.leaf_block, w.branching, d, 2, w.units) / K
         pb = path_bytes(idx_n[s], tr_n[s], level_counts(Nst, w.leaf_block, w.branching), Nst,
                         w.leaf_block, w.branching, d, 2, w.group, 2)
-        for k in acc:
+        for k in pb:
             acc[k] += pb[k] / K
     del graphs, graphs2
     res = {"step_ms": t_step, "append_ms": t_app, "decode_ms": t_dec,
@@ -340,8 +367,7 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, two_call
         Kd[:, :, pos].copy_(hk[:, :, s], non_blocking=True)
         Vd[:, :, pos].copy_(hv[:, :, s], non_blocking=True)
         qbuf.copy_(hq[s], non_blocking=True)
-        tree.append(Kd, pos + 1)
-        route_attend(qbuf, ibuf, obuf, None)
+        decode_call(pos + 1, qbuf, ibuf, obuf, None)
         if out_slot is not None:
             ho[out_slot].copy_(obuf, non_blocking=True)
         torch.cuda.current_stream().synchronize()
@@ -559,8 +585,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-1m", action="store_true")
     ap.add_argument("--no-build", action="store_true")
-    ap.add_argument("--two-call", action="store_true",
-                    help="decode steps as zha_route + zha_sparse_attn_decode instead of zha_decode")
+    ap.add_argument("--mode", choices=["step", "decode", "two_call"], default="step",
+                    help="decode step calls: zha_decode_step (one launch); zha_tree_append + "
+                         "zha_decode; zha_tree_append + zha_route + zha_sparse_attn_decode")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--eager", action="store_true",
                     help="launch the same kernels without CUDA graphs (for profilers)")
@@ -613,7 +640,7 @@ def main():
 
     barrier()
     torch.cuda.synchronize()
-    r = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager, two_call=args.two_call)
+    r = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager, mode=args.mode)
     torch.cuda.synchronize()
     barrier()
 
@@ -621,15 +648,20 @@ def main():
     step_ms = max_over_ranks(float(r["step_ms"].mean()))
     qps = r["queries_per_step"] * world / (step_ms * 1e-3)
     e2e_ms = max_over_ranks(r["e2e_ms_per_step"])
-    # route + attention: one fused launch (route_tma_kernel with its attention epilogue), or
-    # the two calls' combined time with --two-call
+    # the dominant launch: append + route + attention in one kernel (mode "step"), route +
+    # attention in one kernel (mode "decode"), or the route and attention calls together
     dec_ms = float(r["decode_ms"].mean())
-    ra_bytes = r["route_bytes"] + r["attend_bytes"]
-    dom_kernel = "route_tma_kernel+attend_kernel" if args.two_call else "route_tma_kernel (fused decode)"
-    kern = {"decode": {"ms": dec_ms, "bytes": int(ra_bytes), "gbs": ra_bytes / (dec_ms * 1e-3) / 1e9,
-                       "route_bytes": int(r["route_bytes"]), "attend_bytes": int(r["attend_bytes"])},
-            "append": {"ms": float(r["append_ms"].mean())}}
+    fused_append = args.mode == "step"
+    dec_bytes = r["route_bytes"] + r["attend_bytes"] + (r["append_bytes"] if fused_append else 0)
+    dom_kernel = {"step": "route_tma_kernel (fused append + decode)",
+                  "decode": "route_tma_kernel (fused decode)",
+                  "two_call": "route_tma_kernel + attend_kernel"}[args.mode]
+    kern = {"decode": {"ms": dec_ms, "bytes": int(dec_bytes), "gbs": dec_bytes / (dec_ms * 1e-3) / 1e9,
+                       "route_bytes": int(r["route_bytes"]), "attend_bytes": int(r["attend_bytes"]),
+                       "append_bytes": int(r["append_bytes"]), "includes_append": fused_append},
+            "append": {"ms": float(r["append_ms"].mean()), "separate_launch": not fused_append}}
     dom = "decode"
+    ra_bytes = r["route_bytes"] + r["attend_bytes"]
     ra_ms = dec_ms
     line = {
         "metric": METRIC, "value": qps, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
@@ -638,7 +670,7 @@ def main():
         "config": workload_config(w),
         "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": kern[dom]["gbs"],
                      "peak": peak, "unit": "GB/s", "frac": kern[dom]["gbs"] / peak,
-                     "traffic": None if args.two_call else kernel_traffic("decode_fused"),
+                     "traffic": kernel_traffic({"step": "decode_step_fused", "decode": "decode_fused"}.get(args.mode, "")),
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": kern[dom]["bytes"]},
         "route_attend": {"gbs": ra_bytes / (ra_ms * 1e-3) / 1e9, "frac": ra_bytes / (ra_ms * 1e-3) / 1e9 / peak,
@@ -650,7 +682,9 @@ def main():
                 "d2h_bytes_per_step": r["d2h_bytes_per_step"]},
         "gpu_launches": int(round(r["launches_per_step"] * K)),
         "launch_mode": "eager" if args.eager else "cuda_graph_per_step",
-        "decode_call": "zha_route + zha_sparse_attn_decode" if args.two_call else "zha_decode (fused)",
+        "decode_call": {"step": "zha_decode_step (append + route + attention, one launch)",
+                        "decode": "zha_tree_append + zha_decode",
+                        "two_call": "zha_tree_append + zha_route + zha_sparse_attn_decode"}[args.mode],
         "clocks": r["clocks"],
     }
 

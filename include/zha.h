@@ -170,6 +170,20 @@ zha_status zha_decode(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, 
                       float* d_leaf_score, int* d_trace, void* d_O, zha_dtype o_dtype,
                       void* stream);
 
+/* One decode step: zha_tree_append(tree, d_K, new_seq_len) followed by zha_decode(...) over
+ * the extended cache, with the same results.  When the appended tokens all fall into one
+ * leaf (a step of one token, say) and the decode runs one query per CTA (at most two queries
+ * per SM), both happen in a single kernel launch: every CTA recomputes the leaf-to-root path
+ * of its unit with the append's arithmetic, one CTA per unit stores it, and the route uses
+ * the recomputed rows.  Otherwise the append and the decode are launched one after the other.
+ * The caller has written rows [seq_len, new_seq_len) of K and V.  Argument checks as in both
+ * calls (new_seq_len >= seq_len, <= capacity_tokens, > 0); on a host-side error nothing is
+ * launched and the tree is unchanged. */
+zha_status zha_decode_step(zha_tree* tree, const void* d_K, const void* d_V, long long new_seq_len,
+                           const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
+                           float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                           zha_dtype o_dtype, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word:
  * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */
 zha_status zha_tree_check(zha_tree* tree, void* stream);

@@ -56,6 +56,8 @@ CASES = [
     _wl("bf16_d128_regpath", 1, 1, 2, 128, 20000, "bf16", 8, 4, 64, 2, 112),
     # many queries with short leaf lists (the 1M shape): narrow launch, attention fused
     _wl("bf16_d128_narrow_lb4", 1, 2, 16, 128, 20001, "bf16", 8, 4, 8, 32, 116),
+    # odd number of queries (the last CTA is partly empty), d 64, one warp per query
+    _wl("bf16_d64_narrow_odd", 1, 3, 3, 64, 2000, "bf16", 4, 8, 4, 101, 117),
 ]
 
 

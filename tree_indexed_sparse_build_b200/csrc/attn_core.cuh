@@ -111,7 +111,7 @@ __device__ __forceinline__ void attn_tokens(const unsigned char* Ks, const unsig
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int t = t0 + off * u + tg;
-      float d0 = 0.f, d1 = 0.f;
+      float2 d01 = make_float2(0.f, 0.f);  // even / odd dims, updated by packed FMAs
       if (t < cnt) {
         const unsigned char* row = Ks + (size_t)t * S::ROWB;
 #pragma unroll
@@ -120,13 +120,11 @@ __device__ __forceinline__ void attn_tokens(const unsigned char* Ks, const unsig
           float f[S::VEC];
           Vec16<TKV>::to_f32(v, f);
 #pragma unroll
-          for (int e = 0; e < S::VEC; e += 2) {
-            d0 = fmaf(qv[j][e], f[e], d0);
-            d1 = fmaf(qv[j][e + 1], f[e + 1], d1);
-          }
+          for (int e = 0; e < S::VEC; e += 2)
+            d01 = __ffma2_rn(make_float2(qv[j][e], qv[j][e + 1]), make_float2(f[e], f[e + 1]), d01);
         }
       }
-      float d = d0 + d1;
+      float d = d01.x + d01.y;
       d += __shfl_xor_sync(0xffffffffu, d, 1);
       d += __shfl_xor_sync(0xffffffffu, d, 2);
       sc[u] = t < cnt ? d * qk_scale : -INFINITY;
@@ -156,7 +154,12 @@ __device__ __forceinline__ void attn_tokens(const unsigned char* Ks, const unsig
         float v[S::DPL];
         attn_load_v<D>(reinterpret_cast<const TKV*>(Vs + (size_t)t * S::ROWB) + lane * S::DPL, v);
 #pragma unroll
-        for (int e = 0; e < S::DPL; ++e) acc[e] = fmaf(p, v[e], acc[e]);
+        for (int e = 0; e < S::DPL; e += 2) {
+          const float2 r = __ffma2_rn(make_float2(p, p), make_float2(v[e], v[e + 1]),
+                                      make_float2(acc[e], acc[e + 1]));
+          acc[e] = r.x;
+          acc[e + 1] = r.y;
+        }
       }
     }
     __syncwarp();

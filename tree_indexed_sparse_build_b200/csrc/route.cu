@@ -32,249 +32,13 @@
 #include <type_traits>
 
 #include "attn_core.cuh"
+#include "decode_append.cuh"
+#include "decode_attn.cuh"
 #include "device_common.cuh"
+#include "route_common.cuh"
 #include "zha_internal.h"
 
 namespace zha {
-
-constexpr int kRouteMaxWarps = 16;
-
-struct RouteArgs {
-  const void* Q;
-  int q_bf16;
-  int q_heads, nq, group, kv_heads;
-  const float* pyr;
-  long long pyr_unit_stride;  // floats
-  long long off[kMaxLevels];
-  long long n[kMaxLevels];
-  int L, b, beam, cmax;
-  int wpq, qpc;           // warps per query, queries per CTA
-  int query_smem_words;   // 8-byte words of shared memory per query
-  int* leaf_idx;
-  float* leaf_score;
-  int* trace;
-  long long total_queries;
-  unsigned* err;           // device error word (bounded waits)
-  int query_smem_bytes;    // shared memory per query (staged kernel)
-  int rows_bytes;          // bytes of the candidate-row region per query
-  // fused attention (route_tma_kernel with TKV != NoKV)
-  const char* K;
-  const char* V;
-  long long kv_unit_stride;  // bytes
-  long long lb, N;
-  float qk_scale;            // scale * log2(e)
-  int stage_tokens;          // tokens per stage buffer (two buffers in the row region)
-  void* O;
-  int o_bf16;
-};
-
-struct NoKV {};  // route only: no attention epilogue
-
-constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
-
-// Shared-memory layout of one query in the staged kernel.
-struct RouteSmem {
-  size_t rows, keys, cand, surv_a, surv_b, leaf_sc, red, pw, bar, total;
-};
-__host__ __device__ inline size_t route_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
-__host__ __device__ inline size_t route_rows_bytes(int D, int cmax) { return (size_t)cmax * D * 4; }
-// rows_bytes >= route_rows_bytes(D, cmax); a fused decode may ask for more room to stage
-// K/V, and for 16 floats of softmax weights per attending warp (pw_warps).
-__host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam, size_t rows_bytes,
-                                                       int pw_warps) {
-  RouteSmem s;
-  size_t o = 0;
-  s.rows = o;   // candidate summary rows, fp32 [cmax][D]; K/V stage buffers after the route
-  o += rows_bytes;
-  s.keys = o;   // candidate keys [cmax]
-  o += (size_t)cmax * 8;
-  s.cand = o;   // candidate node ids [cmax]
-  o += (size_t)cmax * 4;
-  s.surv_a = o;
-  o += (size_t)beam * 4;
-  s.surv_b = o;
-  o += (size_t)beam * 4;
-  s.leaf_sc = o;
-  o += (size_t)beam * 4;
-  o = route_align(o, 16);
-  s.red = o;  // per-warp partial results of the CTA-wide selection [3][16]
-  o += 3 * 16 * 4;
-  s.pw = o;   // fused attention: per-warp softmax weights of one round [pw_warps][16]
-  o += (size_t)pw_warps * 16 * 4;
-  o = route_align(o, 8);
-  s.bar = o;  // two mbarriers: level copies / stage buffer 0, stage buffer 1
-  o += 16;
-  s.total = route_align(o, 128);
-  return s;
-}
-
-__device__ __forceinline__ unsigned long long route_key(float s, int node) {
-  s = s + 0.0f;  // -0 -> +0 so equal scores tie exactly
-  const uint32_t u = __float_as_uint(s);
-  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return ((unsigned long long)ord << 32) | (uint32_t)(~(uint32_t)node);
-}
-__device__ __forceinline__ int key_node(unsigned long long k) { return (int)(~(uint32_t)k); }
-__device__ __forceinline__ float key_score(unsigned long long k) {
-  const uint32_t ord = (uint32_t)(k >> 32);
-  const uint32_t u = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
-  return __uint_as_float(u);
-}
-
-// Threshold T with exactly `beam` of keys[0, C) >= T (C > beam; keys distinct), found by
-// one warp.  kr holds this lane's keys k = lane + 32 i (i < R; 0 past C), keys beyond 32 R
-// are read from shared memory.  Binary search on the score word, one bit per step, with
-// the warp-wide count taken from ballots; it starts below the common prefix of the
-// largest and smallest score word and stops as soon as exactly `beam` keys remain.  If
-// the whole score word ties at the boundary, the same search runs on the index word of
-// the tied keys (larger index word = lower node index = kept first).
-template <int R>
-__device__ unsigned long long select_threshold(const unsigned long long (&kr)[R],
-                                               const unsigned long long* keys, int C, int beam,
-                                               int lane) {
-  uint32_t h[R];
-  uint32_t lmax = 0u, lmin = 0xFFFFFFFFu;
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    h[i] = (uint32_t)(kr[i] >> 32);
-    if (lane + 32 * i < C) {
-      lmax = max(lmax, h[i]);
-      lmin = min(lmin, h[i]);
-    }
-  }
-  const bool tail = C > 32 * R;
-  for (int k = lane + 32 * R; k < C; k += 32) {
-    const uint32_t x = (uint32_t)(keys[k] >> 32);
-    lmax = max(lmax, x);
-    lmin = min(lmin, x);
-  }
-  const uint32_t hmax = __reduce_max_sync(0xffffffffu, lmax);
-  const uint32_t hmin = __reduce_min_sync(0xffffffffu, lmin);
-  const uint32_t diff = hmax ^ hmin;
-  const int top = diff ? 31 - __clz(diff) : -1;
-  // T <= hmin, so count(>= T) == C > beam holds before the first step.
-  uint32_t T = top < 0 ? hmax : (top >= 31 ? 0u : (hmax & ~((2u << top) - 1u)));
-#pragma unroll 1
-  for (int bit = top; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    unsigned cnt = 0;
-#pragma unroll
-    for (int i = 0; i < R; ++i) cnt += __popc(__ballot_sync(0xffffffffu, h[i] >= cand));
-    if (tail) {
-      unsigned t = 0;
-      for (int k = lane + 32 * R; k < C; k += 32) t += (uint32_t)(keys[k] >> 32) >= cand ? 1u : 0u;
-      cnt += __reduce_add_sync(0xffffffffu, t);
-    }
-    if (cnt >= (unsigned)beam) {
-      T = cand;
-      if (cnt == (unsigned)beam) return (unsigned long long)T << 32;
-    }
-  }
-  // Ties on the score word T: keep every larger score and the `need` tied keys with the
-  // largest index words.
-  unsigned gt = 0;
-#pragma unroll
-  for (int i = 0; i < R; ++i) gt += __popc(__ballot_sync(0xffffffffu, h[i] > T));
-  if (tail) {
-    unsigned t = 0;
-    for (int k = lane + 32 * R; k < C; k += 32) t += (uint32_t)(keys[k] >> 32) > T ? 1u : 0u;
-    gt += __reduce_add_sync(0xffffffffu, t);
-  }
-  const unsigned need = (unsigned)beam - gt;
-  uint32_t Tl = 0u;
-#pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = Tl | (1u << bit);
-    unsigned cnt = 0;
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-      cnt += __popc(__ballot_sync(0xffffffffu, h[i] == T && (uint32_t)kr[i] >= cand && lane + 32 * i < C));
-    if (tail) {
-      unsigned t = 0;
-      for (int k = lane + 32 * R; k < C; k += 32) {
-        const unsigned long long key = keys[k];
-        t += ((uint32_t)(key >> 32) == T && (uint32_t)key >= cand) ? 1u : 0u;
-      }
-      cnt += __reduce_add_sync(0xffffffffu, t);
-    }
-    if (cnt >= need) {
-      Tl = cand;
-      if (cnt == need) break;
-    }
-  }
-  return ((unsigned long long)T << 32) | Tl;
-}
-
-// The beam-th largest of keys[0, C) (C > beam; keys distinct).  Binary search on the
-// score word first (cached in registers, one bit per step, warp-wide counts), stopping as
-// soon as exactly `beam` keys are at or above the threshold; only when scores tie at the
-// threshold does it continue on the index word, read from shared memory.
-__device__ unsigned long long kth_largest_key(const unsigned long long* keys, int C, int beam,
-                                              int lane) {
-  constexpr int R = 8;  // score words cached per lane (C <= 256 needs no shared reads)
-  uint32_t hi[R];
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    const int k = lane + 32 * i;
-    hi[i] = k < C ? (uint32_t)(keys[k] >> 32) : 0u;
-  }
-  // Every key's score word lies in [hmin, hmax]; their common leading bits are fixed.
-  uint32_t lmax = 0u, lmin = 0xFFFFFFFFu;
-#pragma unroll
-  for (int i = 0; i < R; ++i)
-    if (lane + 32 * i < C) {
-      lmax = max(lmax, hi[i]);
-      lmin = min(lmin, hi[i]);
-    }
-  for (int k = lane + 32 * R; k < C; k += 32) {
-    const uint32_t h = (uint32_t)(keys[k] >> 32);
-    lmax = max(lmax, h);
-    lmin = min(lmin, h);
-  }
-  const uint32_t hmax = __reduce_max_sync(0xffffffffu, lmax);
-  const uint32_t hmin = __reduce_min_sync(0xffffffffu, lmin);
-  const uint32_t diff = hmax ^ hmin;
-  const int top = diff ? 31 - __clz(diff) : -1;  // highest bit where scores differ
-  // T <= hmin, so count(>= T) == C > beam holds before the first step.
-  uint32_t T = top < 0 ? hmax : (top >= 31 ? 0u : (hmax & ~((2u << top) - 1u)));
-#pragma unroll 1
-  for (int bit = top; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    unsigned cnt = 0;
-#pragma unroll
-    for (int i = 0; i < R; ++i) cnt += hi[i] >= cand ? 1u : 0u;
-    for (int k = lane + 32 * R; k < C; k += 32) cnt += (uint32_t)(keys[k] >> 32) >= cand ? 1u : 0u;
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= (unsigned)beam) {
-      T = cand;
-      if (cnt == (unsigned)beam) return (unsigned long long)T << 32;
-    }
-  }
-  // Scores tie at T: keep every key with a larger score and the `need` tied keys with
-  // the largest index words (= lowest node indices).
-  unsigned gt = 0;
-#pragma unroll
-  for (int i = 0; i < R; ++i) gt += hi[i] > T ? 1u : 0u;
-  for (int k = lane + 32 * R; k < C; k += 32) gt += (uint32_t)(keys[k] >> 32) > T ? 1u : 0u;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const unsigned need = (unsigned)beam - gt;
-  uint32_t Tl = 0u;
-#pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = Tl | (1u << bit);
-    unsigned cnt = 0;
-    for (int k = lane; k < C; k += 32) {
-      const unsigned long long key = keys[k];
-      cnt += ((uint32_t)(key >> 32) == T && (uint32_t)key >= cand) ? 1u : 0u;
-    }
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= need) {
-      Tl = cand;
-      if (cnt == need) break;
-    }
-  }
-  return ((unsigned long long)T << 32) | Tl;
-}
 
 template <int D, int U>
 __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const RouteArgs a) {
@@ -403,176 +167,6 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
   }
 }
 
-// One warp: keep the top-min(beam, C) of keys[0, C) and write their node ids (cand) to
-// nxt in candidate order (and their scores to leaf_sc when `leaf`).  Keys and ids for
-// k = lane + 32 i, i < R, are held in registers; candidates past 32 R come from shared
-// memory.  Returns the number kept.
-template <int R>
-__device__ __forceinline__ int select_compact(const unsigned long long* keys, const int* cand, int C,
-                                              int beam, int lane, int* nxt, float* leaf_sc,
-                                              bool leaf) {
-  unsigned long long kr[R];
-  int cr[R];
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    const int k = lane + 32 * i;
-    kr[i] = k < C ? keys[k] : 0ull;
-    cr[i] = k < C ? cand[k] : 0;
-  }
-  const unsigned long long T = C > beam ? select_threshold<R>(kr, keys, C, beam, lane) : 0ull;
-  int kept = 0;
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    const bool keep = lane + 32 * i < C && kr[i] >= T;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-      nxt[pos] = cr[i];
-      if (leaf) leaf_sc[pos] = key_score(kr[i]);
-    }
-    kept += __popc(bal);
-  }
-  for (int k0 = 32 * R; k0 < C; k0 += 32) {
-    const int k = k0 + lane;
-    const unsigned long long key = k < C ? keys[k] : 0ull;
-    const bool keep = k < C && key >= T;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = kept + __popc(bal & ((1u << lane) - 1u));
-      nxt[pos] = cand[k];
-      if (leaf) leaf_sc[pos] = key_score(key);
-    }
-    kept += __popc(bal);
-  }
-  return kept;
-}
-
-// Rank selection for small levels (C <= 64 nw, at most two candidates per thread of the
-// query's nw warps): a key is kept iff fewer than `beam` keys of the level are greater
-// (keys are distinct, so exactly min(C, beam) are kept).  Each thread counts for its
-// candidates k = t and t + 32 nw against every key, reading two keys per 16-byte
-// shared-memory load; no barrier per bit, and every warp of the query takes part.  The
-// kept candidates are compacted in candidate order by per-warp ballots.  keys must be
-// 16-byte aligned.  Every thread of the group must call it.  Returns the number kept.
-__device__ __forceinline__ int select_rank_group(const unsigned long long* keys, const int* cand,
-                                                 int C, int beam, int* nxt, float* leaf_sc,
-                                                 bool leaf, unsigned* red, int wq, int lane, int nw,
-                                                 int bar_id) {
-  const int nt = 32 * nw;
-  int kept_before = 0;  // kept candidates of earlier passes
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int k = 32 * wq + lane + pass * nt;
-    if (pass == 1 && C <= nt) break;  // C is the same for the whole group
-    const bool have = k < C;
-    const unsigned long long key = have ? keys[k] : 0ull;
-    int rank = 0;
-    if (have && C > beam) {
-      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
-      int j = 0;
-#pragma unroll 4
-      for (; j + 1 < C; j += 2) {
-        const ulonglong2 v = k2[j >> 1];
-        rank += (v.x > key ? 1 : 0) + (v.y > key ? 1 : 0);
-      }
-      if (j < C) rank += keys[j] > key ? 1 : 0;
-    }
-    const bool keep = have && rank < beam;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (nw > 1) {
-      if (lane == 0) red[32 + wq] = __popc(bal);
-      group_sync(bar_id, nt);
-    }
-    int pre = kept_before, all = kept_before;
-    for (int w = 0; w < nw; ++w) {
-      const int c = nw > 1 ? (int)red[32 + w] : __popc(bal);
-      if (w < wq) pre += c;
-      all += c;
-    }
-    if (keep) {
-      const int pos = pre + __popc(bal & ((1u << lane) - 1u));
-      nxt[pos] = cand[k];
-      if (leaf) leaf_sc[pos] = key_score(key);
-    }
-    if (nw > 1) group_sync(bar_id, nt);  // red is reused by the next pass
-    kept_before = all;
-  }
-  return min(C, beam);
-}
-
-// Warp-group variant for a query owning nw warps (C <= 32 nw): thread t = 32 wq + lane of
-// the group holds candidate t.  The threshold search counts with a group barrier reduction
-// (named barrier bar_id over the group's 32 nw threads; one barrier per bit); the kept
-// candidates are compacted in candidate order with per-warp ballots and a prefix over the
-// warps' counts.  Every thread of the group must call it.  Returns the number kept.
-__device__ __forceinline__ int select_compact_group(const unsigned long long* keys, const int* cand,
-                                                    int C, int beam, int* nxt, float* leaf_sc,
-                                                    bool leaf, unsigned* red, int wq, int lane,
-                                                    int nw, int bar_id) {
-  const int t = 32 * wq + lane, nt = 32 * nw;
-  const bool have = t < C;
-  const unsigned long long key = have ? keys[t] : 0ull;
-  const int node = have ? cand[t] : 0;
-  const uint32_t h = (uint32_t)(key >> 32);
-  unsigned long long T = 0ull;
-  if (C > beam) {
-    const uint32_t wmax = __reduce_max_sync(0xffffffffu, have ? h : 0u);
-    const uint32_t wmin = __reduce_min_sync(0xffffffffu, have ? h : 0xFFFFFFFFu);
-    if (lane == 0) {
-      red[wq] = wmax;
-      red[16 + wq] = wmin;
-    }
-    group_sync(bar_id, nt);
-    uint32_t hmax = 0u, hmin = 0xFFFFFFFFu;
-    for (int w = 0; w < nw; ++w) {
-      hmax = max(hmax, red[w]);
-      hmin = min(hmin, red[16 + w]);
-    }
-    const uint32_t diff = hmax ^ hmin;
-    const int top = diff ? 31 - __clz(diff) : -1;
-    uint32_t Th = top < 0 ? hmax : (top >= 31 ? 0u : (hmax & ~((2u << top) - 1u)));
-    bool done = false;
-    for (int bit = top; bit >= 0; --bit) {
-      const uint32_t c = Th | (1u << bit);
-      const int cnt = group_count(bar_id, nt, have && h >= c);
-      if (cnt >= beam) {
-        Th = c;
-        if (cnt == beam) {
-          done = true;
-          break;
-        }
-      }
-    }
-    if (done) {
-      T = (unsigned long long)Th << 32;
-    } else {
-      const int need = beam - group_count(bar_id, nt, have && h > Th);
-      uint32_t Tl = 0u;
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t c = Tl | (1u << bit);
-        const int cnt = group_count(bar_id, nt, have && h == Th && (uint32_t)key >= c);
-        if (cnt >= need) {
-          Tl = c;
-          if (cnt == need) break;
-        }
-      }
-      T = ((unsigned long long)Th << 32) | Tl;
-    }
-  }
-  const bool keep = have && key >= T;
-  const unsigned bal = __ballot_sync(0xffffffffu, keep);
-  if (lane == 0) red[32 + wq] = __popc(bal);
-  group_sync(bar_id, nt);
-  int pre = 0;
-  for (int w = 0; w < wq; ++w) pre += (int)red[32 + w];
-  if (keep) {
-    const int pos = pre + __popc(bal & ((1u << lane) - 1u));
-    nxt[pos] = node;
-    if (leaf) leaf_sc[pos] = key_score(key);
-  }
-  return min(C, beam);
-}
-
 // Staged routing.  qpc queries per CTA, wpq warps per query (blockDim.x = 32 qpc wpq).
 // GROUPED (wpq > 1): the warps of query qi synchronise on named barrier 1 + qi; otherwise
 // each query is one warp, synchronised only within the warp.
@@ -585,7 +179,9 @@ __device__ __forceinline__ int select_compact_group(const unsigned long long* ke
 // memory and write O.  No leaf list goes through global memory and nothing is launched
 // between the route and the attention.
 // NARROW instantiations are built for CTAs of at most 8 warps, three per SM (register cap).
-template <int D, bool GROUPED, typename TKV, bool NARROW>
+// APPEND (fused decode, one query per CTA): the kernel first extends the tree by the
+// tokens appended to one leaf (decode_append.cuh).
+template <int D, bool GROUPED, typename TKV, bool NARROW, bool APPEND = false>
 __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3 : 1)
     route_tma_kernel(const RouteArgs a) {
   constexpr bool ATTEND = !std::is_same<TKV, NoKV>::value;
@@ -624,11 +220,28 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
   }
   const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
+  // fused append: the path region after the query's route region
+  unsigned char* pb = base + a.path_smem_off;
+  PathSmem Ps{};
+  if (APPEND) Ps = path_smem_layout(D, D * (int)sizeof(TKV), (int)a.lb, a.b, a.L);
+  uint64_t* pbar = reinterpret_cast<uint64_t*>(pb + Ps.bar);
   if (wq == 0 && lane == 0) {
     mbar_init(&bar[0], 1);
-    if (ATTEND) mbar_init(&bar[1], 1);
+    if (ATTEND)
+      for (int i = 0; i < a.attn_nbuf; ++i) {
+        if (i > 0) mbar_init(&bar[i], 1);  // "full" (bar[0] serves the route first)
+        mbar_init(&bar[3 + i], nw);        // "empty": one arrival per warp
+      }
+    if (APPEND) mbar_init(pbar, 1);
     fence_mbar_init();
     surv_a[0] = 0;  // the root
+    if constexpr (APPEND) {
+      if (valid) {
+        fence_proxy_async_smem();
+        path_issue<TKV, D>(Ps, pb, a.K + unit * a.kv_unit_stride, pyr_u, a.off, a.n, a.b, a.L,
+                           a.path_leaf, a.path_tokens, a.lb, pbar);
+      }
+    }
   }
   qsync();
 
@@ -657,7 +270,24 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         const int nc = (int)min((long long)a.b, a.n[l] - node0);
         bulk_copy_g2s((void*)(rows + (size_t)j * a.b * D), S + node0 * D, (uint32_t)nc * D * 4, bar);
       }
-      for (int k = lane; k < C; k += 32) cand[k] = a.b * cur[k / a.b] + k % a.b;
+      for (int j = lane; j < m; j += 32) {  // survivor j's children are candidates j b ..
+        const int node0 = a.b * cur[j];
+        const int nc = min(a.b, C - j * a.b);
+        for (int i = 0; i < nc; ++i) cand[j * a.b + i] = node0 + i;
+      }
+    }
+    if (APPEND && wq == 0) {
+      // candidate slot of the path node at this level: its parent is a survivor j, and the
+      // parent's children are candidates j b .. j b + b - 1
+      const long long* node = reinterpret_cast<const long long*>(pb + Ps.node);
+      int* kpos = reinterpret_cast<int*>(pb + Ps.kpos);
+      int found = -1;
+      for (int j0 = 0; j0 < m; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned hit = __ballot_sync(0xffffffffu, j < m && valid && cur[j] == node[l + 1]);
+        if (hit && found < 0) found = j0 + __ffs(hit) - 1;
+      }
+      if (lane == 0) kpos[0] = found < 0 ? -1 : (int)(found * a.b + (node[l] - a.b * node[l + 1]));
     }
     if (l == a.L - 1 && valid) {  // load q while the first level is in flight
       const long long qo = qg * D;
@@ -672,6 +302,25 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         qv[j] = make_float4(f[0], f[1], f[2], f[3]);
       }
     }
+    if (APPEND && l == a.L - 1) {
+      // the path rows, while the first level's copies are in flight
+      const bool pok = !valid || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+      const bool pfail = GROUPED ? group_any(bar_id, bar_n, !pok) : __any_sync(0xffffffffu, !pok);
+      if (pfail) {
+        if (wq == 0 && lane == 0) {  // let all copies land before the CTA exits
+          mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+          if (C > 0) mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+        }
+        return;
+      }
+      if constexpr (APPEND) {
+        if (valid) {
+          const bool writer = (qg % a.nq) == 0 && ((qg / a.nq) % a.q_heads) % a.group == 0;
+          path_compute<TKV, D>(Ps, pb, const_cast<float*>(pyr_u), a.off, a.n, a.b, a.L, a.path_tokens,
+                               writer, 32 * wq + lane, bar_n, qsync);
+        }
+      }
+    }
     const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
     const bool failed = GROUPED ? group_any(bar_id, bar_n, !ok) : __any_sync(0xffffffffu, !ok);
     if (failed) {
@@ -681,30 +330,39 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     }
     if (!GROUPED) __syncwarp();  // candidate ids written by other lanes
     if (C > 0) parity ^= 1u;
+    if (APPEND) {
+      // the staged row of the path node may predate the append: use the recomputed one
+      const int k = *reinterpret_cast<const int*>(pb + Ps.kpos);
+      if (k >= 0) {
+        const float* pf = reinterpret_cast<const float*>(pb + Ps.pf) + (size_t)l * D;
+        float* dst = const_cast<float*>(rows) + (size_t)k * D;
+        for (int e = 32 * wq + lane; e < D; e += bar_n) dst[e] = pf[e];
+        qsync();
+      }
+    }
 
     // score: rows r = 8 (wq + nw t) + rg, two rows per lane in flight
     for (int r0 = 8 * wq; r0 < C; r0 += 16 * nw) {
-      float acc[2][4];
+      // four running sums per row (dims 4c + e for e = 0..3), updated pairwise by packed FMAs
+      float2 acc[2][2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int r = r0 + 8 * nw * u + rg;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[u][e] = 0.f;
+        acc[u][0] = make_float2(0.f, 0.f);
+        acc[u][1] = make_float2(0.f, 0.f);
         if (r < C) {
           const float4* row = reinterpret_cast<const float4*>(rows + (size_t)r * D);
 #pragma unroll
           for (int j = 0; j < CPL; ++j) {
             const float4 v = row[4 * (j ^ par) + sub];
-            acc[u][0] = fmaf(qv[j].x, v.x, acc[u][0]);
-            acc[u][1] = fmaf(qv[j].y, v.y, acc[u][1]);
-            acc[u][2] = fmaf(qv[j].z, v.z, acc[u][2]);
-            acc[u][3] = fmaf(qv[j].w, v.w, acc[u][3]);
+            acc[u][0] = __ffma2_rn(make_float2(qv[j].x, qv[j].y), make_float2(v.x, v.y), acc[u][0]);
+            acc[u][1] = __ffma2_rn(make_float2(qv[j].z, qv[j].w), make_float2(v.z, v.w), acc[u][1]);
           }
         }
       }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        float s = (acc[u][0] + acc[u][1]) + (acc[u][2] + acc[u][3]);
+        float s = (acc[u][0].x + acc[u][0].y) + (acc[u][1].x + acc[u][1].y);
         s += __shfl_xor_sync(0xffffffffu, s, 1);
         s += __shfl_xor_sync(0xffffffffu, s, 2);
         const int r = r0 + 8 * nw * u + rg;
@@ -720,9 +378,9 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
         for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
       }
-    } else if (GROUPED && C <= 32 * nw) {
-      const int kept =
-          select_compact_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red, wq, lane, nw, bar_id);
+    } else if (GROUPED && C <= 32 * nw) {  // radix selection over the group
+      const int kept = select_radix_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red,
+                                          reinterpret_cast<unsigned*>(base + Ls.hist), wq, lane, nw, bar_id);
       group_sync(bar_id, bar_n);
       if (wq == 0 && a.trace && valid) {
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
@@ -754,132 +412,39 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   }
   if constexpr (ATTEND) {
     using S = AttnShape<TKV, D>;
-    constexpr int ROWB = S::ROWB;
-    const int TS = a.stage_tokens;
-    const int lb = (int)a.lb;
-    unsigned char* sb = base + Ls.rows;  // stage buffer b: K rows at sb + 2 b TS ROWB, V after
-    const size_t stage_bytes = (size_t)TS * ROWB;
-    // Tokens of the selected leaves in slot order.  Only leaf n0 - 1 can hold fewer than
-    // lb tokens, and survivors ascend, so it can only be the last one.
-    int total = 0;
-    if (m > 0) {
-      const long long last = cur[m - 1];
-      total = (m - 1) * lb + (int)(min(last * a.lb + a.lb, a.N) - last * a.lb);
-    }
-    const int nst = (total + TS - 1) / TS;
-    const char* Ku = a.K + unit * a.kv_unit_stride;
-    const char* Vu = a.V + unit * a.kv_unit_stride;
-    // Stage st covers tokens [st TS, min(st TS + TS, total)) in buffer st & 1; the lanes of
-    // warp 0 each copy the K and V pieces of some of its leaves.
-    auto issue = [&](int st) {
-      const int b = st & 1;
-      unsigned char* kb = sb + (size_t)b * 2 * stage_bytes;
-      const int w0 = st * TS, w1 = min(w0 + TS, total);
-      if (lane == 0) mbar_arrive_expect_tx(&bar[b], (uint32_t)(2 * (w1 - w0) * ROWB));
-      __syncwarp();
-      fence_proxy_async_smem();
-      for (int j = w0 / lb + lane; j <= (w1 - 1) / lb; j += 32) {
-        const int p0 = j * lb;
-        const int a0 = max(p0, w0), a1 = min(p0 + lb, w1);
-        const long long row = (long long)cur[j] * a.lb + (a0 - p0);
-        const uint32_t bytes = (uint32_t)((a1 - a0) * ROWB);
-        bulk_copy_g2s(kb + (size_t)(a0 - w0) * ROWB, Ku + row * ROWB, bytes, &bar[b]);
-        bulk_copy_g2s(kb + stage_bytes + (size_t)(a0 - w0) * ROWB, Vu + row * ROWB, bytes, &bar[b]);
-      }
-    };
-    // phase of the wait for stage st: bar[0] carries on from the route's level copies
-    auto phase = [&](int st) -> uint32_t { return ((st & 1) ? 0u : parity) ^ (uint32_t)((st >> 1) & 1); };
-    if (wq == 0 && nst > 0) {
-      issue(0);
-      if (nst > 1) issue(1);
-    }
+    StagedAttn sa;
+    sa.leaves = cur;
+    sa.lb = (int)a.lb;
+    sa.total = leaf_tokens(cur, m, a.lb, a.N);
+    sa.TS = a.stage_tokens;
+    sa.nbuf = a.attn_nbuf;
+    sa.sb = base + Ls.rows;  // the candidate rows (and the append path) are no longer needed
+    sa.bars = bar;
+    sa.empty = bar + 3;
+    sa.ph0 = parity;  // bar[0] carries on from the route's level copies
+    sa.Ku = a.K + unit * a.kv_unit_stride;
+    sa.Vu = a.V + unit * a.kv_unit_stride;
+    sa.qk_scale = a.qk_scale;
+    sa.O = a.O;
+    sa.o_bf16 = a.o_bf16;
+    sa.err = a.err;
+    sa.wait_cycles = kRouteWaitCycles;
+    const int nst = (sa.total + sa.TS - 1) / sa.TS;
+    if (wq == 0)
+      for (int st = 0; st < min(nst, sa.nbuf); ++st)
+        attn_issue_stage<S::ROWB>(cur, sa.lb, sa.total, sa.TS, st, sa.nbuf, sa.sb, sa.Ku, sa.Vu, bar, lane);
     float qa[S::CPL][S::VEC];
     if (valid) attn_load_q<TKV, D>(a.Q, a.q_bf16 != 0, qg, lane, qa);
     float* pw = reinterpret_cast<float*>(base + Ls.pw) + wq * 16;
-    float m_w = -INFINITY, l_w = 0.f;
-    float acc[S::DPL];
-#pragma unroll
-    for (int e = 0; e < S::DPL; ++e) acc[e] = 0.f;
-    int fail_st = -1;
-    for (int st = 0; st < nst; ++st) {
-      const int b = st & 1;
-      const bool ok = mbar_wait_bounded(&bar[b], phase(st), a.err, kDevErrTimeout, kRouteWaitCycles);
-      // the stage is visible to every warp, and every warp is done with stage st - 1, whose
-      // buffer the copy of stage st + 1 now reuses
-      const bool bad = GROUPED ? group_any(bar_id, bar_n, !ok) : __any_sync(0xffffffffu, !ok);
-      if (bad) {
-        fail_st = st;
-        break;
-      }
-      if (wq == 0 && st >= 1 && st + 1 < nst) issue(st + 1);
-      const unsigned char* Ks = sb + (size_t)b * 2 * stage_bytes;
-      attn_tokens<TKV, D>(Ks, Ks + stage_bytes, min(TS, total - st * TS), 8 * wq, 8 * nw, 16 * nw, qa,
-                          a.qk_scale, pw, m_w, l_w, acc, lane);
-    }
-    if (fail_st >= 0) {
-      // let the copies in flight land before the CTA's shared memory is released; the
-      // query's output is poisoned so the failure shows besides the error word
-      // (stages 0 and 1 are issued up front, stage st + 1 only after stage st's barrier)
-      const int last_issued = min(max(fail_st, 1), nst - 1);
-      if (wq == 0 && lane == 0)
-        for (int st = fail_st; st <= last_issued; ++st)
-          mbar_wait_bounded(&bar[st & 1], phase(st), a.err, kDevErrTimeout, kRouteWaitCycles);
-      if (valid && wq == 0)
-        for (int e = lane; e < D; e += 32) {
-          if (a.o_bf16)
-            static_cast<uint16_t*>(a.O)[qg * D + e] = 0x7FC0u;
-          else
-            static_cast<float*>(a.O)[qg * D + e] = __int_as_float(0x7fc00000);
-        }
-      return;
-    }
-    l_w = warp_sum(l_w);
-    if (GROUPED) {
-      // merge the warps' states; the accumulators reuse the stage buffers
-      float* accr = reinterpret_cast<float*>(sb);
-      float* redf = reinterpret_cast<float*>(red);
-      group_sync(bar_id, bar_n);
-#pragma unroll
-      for (int e = 0; e < S::DPL; ++e) accr[wq * D + lane * S::DPL + e] = acc[e];
-      if (lane == 0) {
-        redf[wq] = m_w;
-        redf[16 + wq] = l_w;
-      }
-      group_sync(bar_id, bar_n);
-      for (int d = 32 * wq + lane; d < D && valid; d += bar_n) {
-        float M = -INFINITY;
-        for (int w = 0; w < nw; ++w) M = fmaxf(M, redf[w]);
-        float o = 0.f, l = 0.f;
-        for (int w = 0; w < nw; ++w) {
-          const float sw = redf[w] == -INFINITY ? 0.f : exp2f(redf[w] - M);
-          o = fmaf(sw, accr[w * D + d], o);
-          l = fmaf(sw, redf[16 + w], l);
-        }
-        const float r = l > 0.f ? o / l : 0.f;
-        if (a.o_bf16)
-          static_cast<uint16_t*>(a.O)[qg * D + d] = f32_to_bf16_bits(r);
-        else
-          static_cast<float*>(a.O)[qg * D + d] = r;
-      }
-    } else if (valid) {
-#pragma unroll
-      for (int e = 0; e < S::DPL; ++e) {
-        const float r = l_w > 0.f ? acc[e] / l_w : 0.f;
-        const long long o = qg * D + lane * S::DPL + e;
-        if (a.o_bf16)
-          static_cast<uint16_t*>(a.O)[o] = f32_to_bf16_bits(r);
-        else
-          static_cast<float*>(a.O)[o] = r;
-      }
-    }
+    attend_staged<TKV, D>(sa, qg, valid, qa, pw, reinterpret_cast<float*>(red), wq, nw, lane, bar_id);
   }
 }
 
 namespace {
-template <int D, bool GROUPED, typename TKV, bool NARROW>
+template <int D, bool GROUPED, typename TKV, bool NARROW, bool APPEND = false>
 cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
                           cudaStream_t s) {
-  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW>;
+  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW, APPEND>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
@@ -889,7 +454,16 @@ cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size
 
 template <typename TKV>
 cudaError_t run_route_tma_d(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
-                            int threads, size_t smem, cudaStream_t s) {
+                            int threads, size_t smem, cudaStream_t s, bool append = false) {
+  if constexpr (!std::is_same<TKV, NoKV>::value) {
+    if (append) {  // fused one-leaf append: wide launches only
+      if (grouped)
+        return D == 128 ? run_route_tma<128, true, TKV, false, true>(a, blocks, threads, smem, s)
+                        : run_route_tma<64, true, TKV, false, true>(a, blocks, threads, smem, s);
+      return D == 128 ? run_route_tma<128, false, TKV, false, true>(a, blocks, threads, smem, s)
+                      : run_route_tma<64, false, TKV, false, true>(a, blocks, threads, smem, s);
+    }
+  }
   if (narrow) {
     if (grouped)
       return D == 128 ? run_route_tma<128, true, TKV, true>(a, blocks, threads, smem, s)
@@ -916,6 +490,7 @@ cudaError_t run_route(const RouteArgs& a, unsigned blocks, int threads, size_t s
 }
 
 constexpr size_t kRouteSmemCap = 200 * 1024;  // staged kernel: shared memory per query
+constexpr size_t kCtaSmemCap = 227 * 1024;    // dynamic shared memory of one CTA
 
 // Arguments common to the route and the fused decode.
 RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
@@ -928,6 +503,7 @@ RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int 
   a.nq = nq;
   a.kv_heads = t->desc.kv_heads;
   a.group = q_heads / t->desc.kv_heads;
+  a.head_dim = D;
   a.pyr = t->pyr;
   a.pyr_unit_stride = t->unit_rows * D;
   for (int l = 0; l <= t->L; ++l) {
@@ -997,8 +573,8 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   const long long cmax = a.cmax;
   cudaError_t e;
 
-  // Staged kernel when a query's widest level fits in shared memory.
   a.rows_bytes = (int)route_rows_bytes(D, a.cmax);
+  // Staged kernel when a query's widest level fits in shared memory.
   const size_t per_query = route_smem_layout(D, a.cmax, beam, a.rows_bytes, 0).total;
   if (per_query <= kRouteSmemCap) {
     a.query_smem_bytes = (int)per_query;
@@ -1032,13 +608,15 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   return e;
 }
 
-// Fused route + attention (one launch).  Wide launches (one query per CTA): the row
-// region grows up to 128 KB when the attention wants bigger stages, so a long leaf list
-// streams in a few large stages.  Narrow launches (several queries per SM): the row region
+// Fused route + attention (one launch).  Wide launches (one query per CTA): the row region
+// grows so that the attention streams its leaves through up to three large stages in
+// flight together -- up to 192 KB when every CTA has an SM to itself, 96 KB when two share
+// one -- and, with an SM to itself, also holds the one-leaf append's path after the route's
+// rows (decode_append.cuh).  Narrow launches (several queries per SM): the row region
 // stays the route's own, since a larger one would cut the queries resident per SM, and the
 // call is fused only when the query's tokens then fit in at most two stages; otherwise
-// fused = false and the route and the attention run as two launches.  Stages hold at
-// least 8 tokens.
+// fused = false and the route and the attention run as two launches.  Stages hold a
+// multiple of 16 tokens (the attention's rounds), at least 16.
 DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
   DecodePlan p{};
   const int D = t->desc.head_dim;
@@ -1050,22 +628,36 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
     cmax = std::max(cmax, std::min(std::min((long long)beam, t->n[l + 1]) * t->desc.branching, t->n[l]));
   const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
   const size_t route_rows = route_rows_bytes(D, (int)cmax);
-  const size_t want = (size_t)4 * row * (size_t)((tokens + 1) / 2);  // two stages
-  size_t rows = wide ? std::max(route_rows, std::min(want, (size_t)128 * 1024)) : route_rows;
-  rows = std::max(rows, (size_t)4 * 8 * row);
-  p.stage_tokens = (int)(rows / (4 * row)) / 8 * 8;
+  if (!wide) {
+    p.nbuf = 2;
+    p.rows_bytes = std::max(route_rows, (size_t)4 * 8 * row);
+    p.stage_tokens = (int)(p.rows_bytes / (4 * row)) / 16 * 16;
+    p.attn_warps = 1;
+    p.smem_per_query = route_smem_layout(D, (int)cmax, beam, p.rows_bytes, narrow_wpq(cmax)).total;
+    p.fused = p.smem_per_query <= kRouteSmemCap && p.stage_tokens >= 16 && 2LL * p.stage_tokens >= tokens;
+    return p;
+  }
+  const bool own_sm = queries <= t->sms;
+  const size_t cap = own_sm ? 192 * 1024 : 96 * 1024;
+  size_t rows = std::min((size_t)2 * row * (size_t)tokens, cap);  // all the tokens, if they fit
+  rows = std::max(std::max(rows, route_rows), (size_t)4 * 16 * row);
+  p.path_bytes = path_smem_layout(D, row, (int)t->desc.leaf_block, t->desc.branching, t->L).total;
+  p.path_off = route_align(route_rows, 128);
+  if (own_sm) rows = std::max(rows, p.path_off + p.path_bytes);
+  p.nbuf = rows >= (size_t)3 * 2 * 16 * row ? 3 : 2;
+  p.stage_tokens = (int)(rows / ((size_t)p.nbuf * 2 * row)) / 16 * 16;
   p.rows_bytes = rows;
-  p.attn_warps = wide ? (int)std::min<long long>(kRouteMaxWarps, (tokens + 31) / 32) : 1;
-  p.smem_per_query =
-      route_smem_layout(D, (int)cmax, beam, rows, wide ? kRouteMaxWarps : narrow_wpq(cmax)).total;
-  p.fused = p.smem_per_query <= kRouteSmemCap && (wide || 2LL * p.stage_tokens >= tokens);
+  p.attn_warps = (int)std::min<long long>(kRouteMaxWarps, (tokens + 31) / 32);
+  p.smem_per_query = route_smem_layout(D, (int)cmax, beam, rows, kRouteMaxWarps).total;
+  p.fused = p.smem_per_query <= kCtaSmemCap;
+  p.append_ok = p.fused && own_sm;
   return p;
 }
 
 cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
                           int q_heads, int nq, int beam, const void* d_K, const void* d_V,
                           float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
-                          void* d_O, zha_dtype o_dtype, cudaStream_t stream) {
+                          void* d_O, zha_dtype o_dtype, cudaStream_t stream, long long append_leaf) {
   RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, d_trace);
   const int D = t->desc.head_dim;
   const bool bf = t->desc.kv_dtype == ZHA_BF16;
@@ -1077,15 +669,22 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
   a.N = t->N;
   a.qk_scale = scale * 1.4426950408889634f;
   a.stage_tokens = p.stage_tokens;
+  a.attn_nbuf = p.nbuf;
   a.O = d_O;
   a.o_bf16 = o_dtype == ZHA_BF16;
   a.query_smem_bytes = (int)p.smem_per_query;  // weight area sized for 16 warps when wide
-  const StagedShape sh = staged_shape(t, a, p.smem_per_query, p.attn_warps);
+  StagedShape sh = staged_shape(t, a, p.smem_per_query, p.attn_warps);
+  const bool append = append_leaf >= 0;
+  if (append) {  // the tree already has its new shape; the path region follows the route's
+    a.path_leaf = append_leaf;
+    a.path_tokens = (int)(std::min(append_leaf * a.lb + a.lb, t->N) - append_leaf * a.lb);
+    a.path_smem_off = (long long)p.path_off;  // inside the row region, after the route's rows
+  }
   cudaError_t e;
   if (bf)
-    e = run_route_tma_d<uint16_t>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream);
+    e = run_route_tma_d<uint16_t>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, append);
   else
-    e = run_route_tma_d<float>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream);
+    e = run_route_tma_d<float>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, append);
   ++t->launches;
   return e;
 }

@@ -206,6 +206,41 @@ zha_status zha_decode(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int
                                       scale, d_O, o_dtype, nullptr, s));
 }
 
+zha_status zha_decode_step(zha_tree* t, const void* d_K, const void* d_V, long long new_seq_len,
+                           const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
+                           float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                           zha_dtype o_dtype, void* stream) {
+  // the checks of both calls, before anything is launched or the tree changes
+  if (!t || new_seq_len < t->N || !dtype_ok(q_dtype) || !dtype_ok(o_dtype) || q_heads < 1 || nq < 0)
+    return ZHA_ERR_INVALID_ARG;
+  if (new_seq_len > t->desc.capacity_tokens) return ZHA_ERR_CAPACITY;
+  if (q_heads % t->desc.kv_heads != 0) return ZHA_ERR_INVALID_ARG;
+  if (beam < 1 || beam > kMaxBeam) return ZHA_ERR_INVALID_ARG;
+  if ((long long)beam * t->desc.branching > kMaxCandidates) return ZHA_ERR_UNSUPPORTED;
+  if (new_seq_len == 0 || !(scale == scale)) return ZHA_ERR_INVALID_ARG;
+  if (!d_Q || !d_K || !d_V || !d_leaf_idx || !d_O) return ZHA_ERR_INVALID_ARG;
+  if (!aligned(d_Q, 16) || !aligned(d_K, 16) || !aligned(d_V, 16) || !aligned(d_O, 16) ||
+      !aligned(d_leaf_idx, 4) || (d_leaf_score && !aligned(d_leaf_score, 4)) ||
+      (d_trace && !aligned(d_trace, 4)))
+    return ZHA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long lb = t->desc.leaf_block;
+  const bool one_leaf = t->N > 0 && new_seq_len > t->N && t->N / lb == (new_seq_len - 1) / lb;
+  if (one_leaf && nq > 0) {
+    zha_tree saved = *t;
+    set_shape(t, new_seq_len);
+    const DecodePlan dp = plan_decode(t, q_heads, nq, beam);
+    if (dp.append_ok)
+      return cuda_status(launch_decode(t, dp, d_Q, q_dtype, q_heads, nq, beam, d_K, d_V, scale, d_leaf_idx,
+                                       d_leaf_score, d_trace, d_O, o_dtype, s, (new_seq_len - 1) / lb));
+    *t = saved;  // not fusable: append, then decode
+  }
+  const zha_status st = zha_tree_append(t, d_K, new_seq_len, stream);
+  if (st != ZHA_OK) return st;
+  return zha_decode(t, d_Q, q_dtype, q_heads, nq, beam, d_K, d_V, scale, d_leaf_idx, d_leaf_score,
+                    d_trace, d_O, o_dtype, stream);
+}
+
 zha_status zha_tree_check(zha_tree* t, void* stream) {
   if (!t) return ZHA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

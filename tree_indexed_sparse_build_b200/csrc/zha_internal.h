@@ -72,18 +72,25 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
 
 // Fused route + attention (route.cu): one launch routes each query and attends over its
 // leaves.  fused == false when a query's widest level does not fit the staged kernel.
+// launch_decode with append_leaf >= 0: the launch also extends the tree by the tokens that
+// the caller appended to leaf append_leaf (the tree's host shape already updated;
+// requires append_ok).
 struct DecodePlan {
   bool fused;
   size_t rows_bytes;      // candidate-row / K-V stage region per query
-  int stage_tokens;       // tokens per stage buffer (two buffers)
+  int stage_tokens;       // tokens per stage buffer
+  int nbuf;               // stage buffers (2 or 3)
   int attn_warps;         // warps per query the attention wants (wide launches)
   size_t smem_per_query;
+  bool append_ok;         // a one-leaf append can ride along (wide launches)
+  size_t path_off, path_bytes;  // that append's region inside the row region
 };
 DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam);
 cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
                           int q_heads, int nq, int beam, const void* d_K, const void* d_V,
                           float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
-                          void* d_O, zha_dtype o_dtype, cudaStream_t stream);
+                          void* d_O, zha_dtype o_dtype, cudaStream_t stream,
+                          long long append_leaf = -1);
 
 // Attention (attend.cu).
 struct AttnPlan {

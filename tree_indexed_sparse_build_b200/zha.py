@@ -27,7 +27,7 @@ EXPORTED = [
     "zha_tree_check", "zha_tree_seq_len", "zha_tree_levels", "zha_tree_level_nodes",
     "zha_tree_level_offset", "zha_tree_unit_rows", "zha_tree_summaries", "zha_tree_launch_count",
     "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
-    "zha_decode",
+    "zha_decode", "zha_decode_step",
 ]
 
 
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
             "zha_noalloc_scratch_capacity": (_SZ, []),
             "zha_decode": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P, _I,
                                 _P]),
+            "zha_decode_step": (_I, [_P, _P, _P, _LL, _P, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P,
+                                     _P, _I, _P]),
             "zha_tree_check": (_I, [_P, _P]),
             "zha_tree_seq_len": (_LL, [_P]),
             "zha_tree_levels": (_I, [_P]),
@@ -189,6 +191,17 @@ def zha_decode(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: torch.Ten
     _check(lib().zha_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
                             scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _ptr(O),
                             dtype_code(O.dtype), _stream(stream)), "zha_decode")
+
+
+def zha_decode_step(handle, K: torch.Tensor, V: torch.Tensor, new_seq_len: int, Q: torch.Tensor,
+                    beam: int, scale: float, leaf_idx: torch.Tensor, O: torch.Tensor,
+                    leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
+                    stream=None) -> None:
+    """Append up to new_seq_len, then route + attention (one launch for one-leaf appends)."""
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_decode_step(handle, _ptr(K), _ptr(V), new_seq_len, _ptr(Q), dtype_code(Q.dtype),
+                                 Hq, nq, beam, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
+                                 _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_step")
 
 
 def zha_noalloc_scratch_capacity() -> int:
@@ -324,6 +337,29 @@ class Tree:
         O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
         zha_decode(self.handle, Q, beam, K, V, scale, idx, O, sc, tr, stream)
         return (O, idx, sc, tr) if trace else (O, idx, sc)
+
+    def levels_for(self, seq_len: int) -> int:
+        """Levels below the root of a tree over seq_len tokens (shape only)."""
+        n0 = -(-seq_len // self.desc.leaf_block)
+        L, span = 1, self.desc.branching
+        while span < n0:
+            span *= self.desc.branching
+            L += 1
+        return L if n0 > 0 else 0
+
+    def decode_step(self, K: torch.Tensor, V: torch.Tensor, new_seq_len: int, Q: torch.Tensor,
+                    beam: int, scale: float, out_dtype: torch.dtype = torch.bfloat16,
+                    trace: bool = False, stream=None):
+        """Append to new_seq_len, then route + attention; returns (O, leaf_idx[, trace])."""
+        B, Hq, nq, d = Q.shape
+        idx = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=Q.device)
+        O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
+        tr = None
+        if trace:
+            L = self.levels_for(new_seq_len)
+            tr = torch.empty((B, Hq, nq, L, beam), dtype=torch.int32, device=Q.device)
+        zha_decode_step(self.handle, K, V, new_seq_len, Q, beam, scale, idx, O, None, tr, stream)
+        return (O, idx, tr) if trace else (O, idx)
 
     def check(self, stream=None) -> int:
         return zha_tree_check(self.handle, stream)
