@@ -229,10 +229,10 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     which is why they stay out of the timed pass).
     """
     import torch
-    from tree_indexed_sparse_build_b200 import synth, zha
+    from tree_indexed_sparse_build_b200 import ranks, synth, zha
 
     N, cap = w.seq_len, w.seq_len + W + 2 * K
-    w = w.with_(seed=w.seed + 7919 * rank)
+    w = w.with_(seed=ranks.rank_seed(w.seed, rank))
     Qs = np.stack([synth.queries(w, step=s) for s in range(W + 2 * K)])
     Kn = synth.keys(w, capacity=cap)
     Vn = synth.values(w, capacity=cap)
@@ -393,10 +393,10 @@ def run_1m(W, K, rank, dev, flush, eager=False):
     """1M-token cache, 8 KV heads: route + attend with 64 queries per head (throughput)
     and with 1 query per head (single step)."""
     import torch
-    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+    from tree_indexed_sparse_build_b200 import ranks, synth, workloads, zha
 
     w = workloads.get("deep_1m")
-    w = w.with_(seed=w.seed + 7919 * rank)
+    w = w.with_(seed=ranks.rank_seed(w.seed, rank))
     nqt = workloads.THROUGHPUT_NQ
     Qn = synth.queries(w, nq=nqt)
     Kn = synth.keys(w, Q=Qn)
@@ -517,7 +517,8 @@ def run_build_256k(W, K, dev, flush):
 
 # ----------------------------------------------------------------------------- oracle arm
 
-def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), warmup: int = 0):
+def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), warmup: int = 0,
+                         start=None):
     """Time the fp64 oracle on decode steps of `w` for a few units (single thread).
 
     Setup (not timed): each sampled unit's tree over the first N tokens.  Timed: per step
@@ -551,6 +552,8 @@ def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), 
 
     for s in range(warmup):
         step(s)
+    if start is not None:  # threads of a host-parallel run begin their timed steps together
+        start.wait()
     t0 = time.perf_counter()
     nq = steps = 0
     per_step = []
@@ -562,6 +565,50 @@ def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), 
     el = time.perf_counter() - t0
     return {"value": nq / el, "queries": nq, "seconds": el, "steps": steps, "units": len(units),
             "per_step_s": per_step}
+
+
+def _host_parallel_worker(i, w, seconds, max_steps, start, out):
+    """One process of oracle_host_parallel: a single-unit replica of w (its own seed)."""
+    wi = w.with_(batch=1, kv_heads=1, q_heads=w.group, seed=w.seed + 104729 * (i + 1))
+    r = oracle_decode_sample(wi, seconds=seconds, max_steps=max_steps, units=(0,), start=start)
+    out.put((i, r["queries"], r["seconds"], r["steps"]))
+
+
+def oracle_host_parallel(w, seconds: float, max_steps: int):
+    """The fp64 oracle on every host core: one process per core (started with spawn, so it
+    is safe after CUDA initialisation), each a single-threaded oracle instance routing one
+    (batch, KV head) unit of w's shape with its own seed.  Setup (the unit's tree over the
+    first N tokens) is untimed; all processes then start together and run decode steps;
+    rate = all processes' queries / the slowest process's time."""
+    import multiprocessing as mp
+
+    cores = os.cpu_count() or 1
+    n = min(cores, 64)
+    ctx = mp.get_context("spawn")
+    start = ctx.Barrier(n)
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_host_parallel_worker, args=(i, w, seconds, max_steps, start, out))
+             for i in range(n)]
+    for p in procs:
+        p.start()
+    res = []
+    deadline = time.time() + 20 * seconds + 120
+    import queue as _queue
+    while len(res) < n:
+        try:
+            res.append(out.get(timeout=5))
+        except _queue.Empty:
+            if time.time() > deadline or any(p.exitcode not in (None, 0) for p in procs):
+                for p in procs:
+                    if p.is_alive():
+                        p.terminate()
+                raise RuntimeError("host-parallel oracle processes failed or timed out")
+    for p in procs:
+        p.join(timeout=60)
+    q = sum(r[1] for r in res)
+    t = max(r[2] for r in res)
+    return {"value": q / t, "queries": q, "seconds": t, "threads": n, "cores": cores,
+            "steps": min(r[3] for r in res)}
 
 
 # ----------------------------------------------------------------------------- main
@@ -594,11 +641,10 @@ def main():
     args = ap.parse_args()
     K, W = args.steps, args.warmup
 
-    from tree_indexed_sparse_build_b200 import workloads
+    from tree_indexed_sparse_build_b200 import ranks, workloads
     w = workloads.get("decode_128k")
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ri = ranks.rank_info()
+    rank, world, local = ri.rank, ri.world, ri.local
 
     if args.impl == "reference":
         if rank != 0:
@@ -626,15 +672,10 @@ def main():
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier(world)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return ranks.max_over_ranks(x, world, dev)
 
     sampler = lambda: ClockSampler(local)  # noqa: E731
 
@@ -646,7 +687,7 @@ def main():
 
     peak, peak_kind = hbm_peak()
     step_ms = max_over_ranks(float(r["step_ms"].mean()))
-    qps = r["queries_per_step"] * world / (step_ms * 1e-3)
+    qps = ranks.weak_scaling_rate(r["queries_per_step"], world, step_ms)
     e2e_ms = max_over_ranks(r["e2e_ms_per_step"])
     # the dominant launch: append + route + attention in one kernel (mode "step"), route +
     # attention in one kernel (mode "decode"), or the route and attention calls together
@@ -724,6 +765,17 @@ def main():
         except Exception as e:  # the baseline must never sink the GPU number
             line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle",
                                     "sample": f"failed: {e}"}
+        if args.cpu_seconds > 0:
+            try:
+                hp = oracle_host_parallel(w, seconds=args.cpu_seconds, max_steps=64)
+                line["cpu_baseline_host_parallel"] = {
+                    "value": hp["value"], "unit": UNIT, "cores": hp["threads"], "host_cores": hp["cores"],
+                    "kind": "oracle",
+                    "sample": f"{hp['threads']} processes, each one (batch, KV head) unit of "
+                              f"decode_128k's shape with its own seed, single-threaded fp64 C oracle, "
+                              f">= {hp['steps']} decode steps each"}
+            except Exception as e:
+                line["cpu_baseline_host_parallel"] = {"value": None, "sample": f"failed: {e}"}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
