@@ -515,6 +515,41 @@ def run_build_256k(W, K, dev, flush):
     return res
 
 
+def run_profile_case(case: str, W: int, K: int):
+    """A small case of a bench workload for ncu captures (eager launches, no graphs):
+    deep_1m_2kv = the 1M-token tree with 2 KV heads and 16 query heads (group 8, 64 queries
+    per head) instead of 8 and 64, so a capture holds about 1.5 GB on the device."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+
+    dev = torch.device("cuda", 0)
+    w = workloads.get("deep_1m").with_(kv_heads=2, q_heads=16)
+    nq = workloads.THROUGHPUT_NQ
+    Qn = synth.queries(w, nq=nq)
+    Kn = synth.keys(w, Q=Qn)
+    Vn = synth.values(w)
+    Kd, Vd, Q = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
+    del Kn, Vn
+    tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len, torch.bfloat16)
+    tree.build(Kd, w.seq_len)
+    idx = torch.empty((w.batch, w.q_heads, nq, w.beam), dtype=torch.int32, device=dev)
+    O = torch.empty((w.batch, w.q_heads, nq, w.head_dim), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for it in range(W + K):
+        flush.zero_()
+        e0.record()
+        zha.zha_decode(tree.handle, Q, w.beam, Kd, Vd, w.scale, idx, O)
+        e1.record()
+        torch.cuda.synchronize()
+        if it >= W:
+            ms.append(e0.elapsed_time(e1))
+    assert tree.check() == zha.ZHA_OK
+    tree.close()
+    return {"case": case, "queries": w.batch * w.q_heads * nq, "zha_decode_ms": float(np.mean(ms))}
+
+
 # ----------------------------------------------------------------------------- oracle arm
 
 def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), warmup: int = 0,
@@ -632,6 +667,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-1m", action="store_true")
     ap.add_argument("--no-build", action="store_true")
+    ap.add_argument("--profile-case", choices=["deep_1m_2kv"], default=None,
+                    help="run only a small case for ncu captures: the 1M-token tree at 2 of its "
+                         "8 KV heads (1,024 queries, 64 per head), zha_decode, eager launches")
     ap.add_argument("--mode", choices=["step", "decode", "two_call"], default="step",
                     help="decode step calls: zha_decode_step (one launch); zha_tree_append + "
                          "zha_decode; zha_tree_append + zha_route + zha_sparse_attn_decode")
@@ -661,6 +699,10 @@ def main():
                                            f"{w.group} query heads, single-threaded fp64 C oracle"},
                 "e2e": {"value": qps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
+        return
+
+    if args.profile_case:
+        print(json.dumps(run_profile_case(args.profile_case, W, K)))
         return
 
     import torch
