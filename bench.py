@@ -515,6 +515,51 @@ def run_build_256k(W, K, dev, flush):
     return res
 
 
+def run_causal(W, K, dev, flush):
+    """Causal (per-position) routing + attention, zha_decode_causal: (1) every position of a
+    1,024-token cache (tiny_fp32's tree: binary, 16-token leaves, beam 2) with the keys read
+    per query against dense causal attention; (2) 256 evenly spaced positions of every head of
+    the gqa_32k cache (b 8, 64-token leaves, beam 8)."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+
+    out = {}
+    cases = (("prefix_1024", workloads.get("tiny_fp32").with_(needles=0), 1024),
+             ("gqa_32k", workloads.get("gqa_32k").with_(needles=0), 256))
+    for name, w, npos in cases:
+        Qn = synth.queries(w, nq=npos)
+        Kn, Vn = synth.keys(w), synth.values(w)
+        dt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+        Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
+        del Kn, Vn
+        tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len, dt)
+        tree.build(Kd, w.seq_len)
+        pos = np.linspace(0, w.seq_len - 1, npos).round().astype(np.int64)
+        pos_d = torch.from_numpy(pos).to(dev)
+        idx = torch.empty((w.batch, w.q_heads, npos, w.beam), dtype=torch.int32, device=dev)
+        O = torch.empty((w.batch, w.q_heads, npos, w.head_dim), dtype=dt if name == "prefix_1024" else torch.bfloat16,
+                        device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ms = []
+        for it in range(W + K):
+            flush.zero_()
+            e0.record()
+            zha.zha_decode_causal(tree.handle, Qd, pos_d, w.beam, Kd, Vd, w.scale, idx, O)
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= W:
+                ms.append(e0.elapsed_time(e1))
+        assert tree.check() == zha.ZHA_OK
+        li = idx.cpu().numpy().astype(np.int64)
+        tok = np.where(li >= 0, np.minimum((li + 1) * w.leaf_block, pos[None, None, :, None] + 1)
+                       - li * w.leaf_block, 0).sum(axis=-1)
+        q = w.batch * w.q_heads * npos
+        out[name] = {"queries": q, "ms": float(np.mean(ms)), "qps": q / (np.mean(ms) * 1e-3),
+                     "keys_per_query": float(tok.mean()), "dense_keys_per_query": float((pos + 1).mean())}
+        tree.close()
+    return out
+
+
 def run_profile_case(case: str, W: int, K: int):
     """A small case of a bench workload for ncu captures (eager launches, no graphs):
     deep_1m_2kv = the 1M-token tree with 2 KV heads and 16 query heads (group 8, 64 queries
@@ -795,6 +840,7 @@ def main():
 
     if not args.no_build and rank == 0:
         line["build_256k"] = run_build_256k(W, K, dev, flush)
+        line["causal"] = run_causal(W, min(K, 10), dev, flush)
 
     if rank == 0 and world == 1:
         try:

@@ -184,6 +184,32 @@ zha_status zha_decode_step(zha_tree* tree, const void* d_K, const void* d_V, lon
                            float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
                            zha_dtype o_dtype, void* stream);
 
+/* Causal (per-position) routing, as a prefill visits every position: query i of every
+ * (batch, query head) routes over the tree of the prefix of tokens 0 .. d_positions[i] -- the
+ * tree zha_tree_build would make over those tokens alone -- with the rules of zha_route.
+ * That tree shares every node with the stored tree except its right edge (the ancestors of
+ * the leaf holding token d_positions[i]), which each query recomputes on chip from the
+ * cache and the stored rows; the stored tree is not changed.
+ *   d_K          the cache the tree was built over (the prefix's last leaf is re-read)
+ *   d_positions  [nq] int64, device: 0 <= position < seq_len; a position outside the tree
+ *                sets ZHA_ERR_DEVICE in the error word and that query routes nowhere
+ *                (leaves all -1)
+ *   d_trace      nullable: [batch, q_heads, nq, L, beam] with L = zha_tree_levels of the
+ *                whole tree; rows of levels at or above the prefix tree's depth are -1
+ * Other arguments, layouts and limits as in zha_route; nothing is allocated.
+ * ZHA_ERR_UNSUPPORTED when a query's widest level and the path do not fit shared memory. */
+zha_status zha_route_causal(const zha_tree* tree, const void* d_K, const void* d_Q, zha_dtype q_dtype,
+                            int q_heads, int nq, const long long* d_positions, int beam, int* d_leaf_idx,
+                            float* d_leaf_score, int* d_trace, void* stream);
+
+/* zha_route_causal followed by exact softmax attention of each query over the tokens of its
+ * leaves that lie in its prefix (t <= position), in one launch; O as in zha_decode.
+ * ZHA_ERR_UNSUPPORTED when the shape does not fit the fused kernel. */
+zha_status zha_decode_causal(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                             const long long* d_positions, int beam, const void* d_K, const void* d_V,
+                             float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                             zha_dtype o_dtype, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word:
  * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */
 zha_status zha_tree_check(zha_tree* tree, void* stream);

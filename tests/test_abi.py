@@ -74,6 +74,10 @@ def test_calls_reject_null_tree_on_host():
     assert lib.zha_sparse_attn_decode_noalloc(None, None, 1, 8, 1, None, None, None, 4,
                                               ctypes.c_float(0.1), None, 1, None) == \
         zha.ZHA_ERR_INVALID_ARG
+    assert lib.zha_route_causal(None, None, None, 1, 8, 1, None, 4, None, None, None, None) == \
+        zha.ZHA_ERR_INVALID_ARG
+    assert lib.zha_decode_causal(None, None, 1, 8, 1, None, 4, None, None, ctypes.c_float(0.1), None,
+                                 None, None, None, 1, None) == zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_tree_destroy(None) == zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_tree_check(None, None) == zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_tree_levels(None) == -1

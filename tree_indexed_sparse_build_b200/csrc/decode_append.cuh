@@ -19,9 +19,9 @@
 namespace zha {
 
 // Shared memory of the path, for head_dim D, token rows of row_bytes, leaf block lb,
-// branching b and L levels below the root.
+// branching b and (at most) L levels below the root.
 struct PathSmem {
-  size_t tok, sib, pv, pf, node, kpos, bar, total;
+  size_t tok, sib, pv, pf, node, kpos, qn, bar, total;
 };
 __host__ __device__ inline size_t path_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int lb, int b, int L) {
@@ -39,6 +39,8 @@ __host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int l
   o += (size_t)(L + 1) * 8;
   s.kpos = o;  // candidate slot of the path node at the current route level
   o += 8;
+  s.qn = o;    // causal routing: the prefix tree's node counts per level; its depth last
+  o += (size_t)kMaxLevels * 8;
   s.bar = o;
   o += 8;
   s.total = path_align(o, 128);

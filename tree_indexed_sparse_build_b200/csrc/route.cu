@@ -179,12 +179,21 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
 // memory and write O.  No leaf list goes through global memory and nothing is launched
 // between the route and the attention.
 // NARROW instantiations are built for CTAs of at most 8 warps, three per SM (register cap).
-// APPEND (fused decode, one query per CTA): the kernel first extends the tree by the
-// tokens appended to one leaf (decode_append.cuh).
-template <int D, bool GROUPED, typename TKV, bool NARROW, bool APPEND = false>
+// PATH (decode_append.cuh; needs TKV, the type of the K rows the path reads):
+//  kPathAppend (fused decode, one query per CTA) -- the kernel first extends the tree by
+//    the tokens appended to one leaf, and stores the path (one CTA per unit);
+//  kPathPrefix (causal routing) -- query qg routes over the tree of tokens 0 .. p, p =
+//    positions[qg % nq]: its own depth and node counts, and its prefix's right edge
+//    recomputed into shared memory (never stored).
+// With a KV type, the query then attends over its leaves unless O is null.
+template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH = kPathNone>
 __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3 : 1)
     route_tma_kernel(const RouteArgs a) {
   constexpr bool ATTEND = !std::is_same<TKV, NoKV>::value;
+  constexpr bool APPEND = PATH == kPathAppend;
+  constexpr bool PREFIX = PATH == kPathPrefix;
+  constexpr bool HASPATH = PATH != kPathNone;
+  static_assert(!HASPATH || ATTEND, "the path reads K rows of type TKV");
   constexpr int CPL = D / 16;  // 16-byte chunks of a row per lane (4 lanes per row)
   constexpr int R = 8;         // candidate keys held per lane in the selecting warp
   extern __shared__ __align__(128) unsigned char rsm[];
@@ -220,11 +229,35 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
   }
   const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
-  // fused append: the path region after the query's route region
+  // the path region (fused append or causal prefix)
   unsigned char* pb = base + a.path_smem_off;
   PathSmem Ps{};
-  if (APPEND) Ps = path_smem_layout(D, D * (int)sizeof(TKV), (int)a.lb, a.b, a.L);
+  if (HASPATH) Ps = path_smem_layout(D, D * (int)sizeof(TKV), (int)a.lb, a.b, a.L);
   uint64_t* pbar = reinterpret_cast<uint64_t*>(pb + Ps.bar);
+  // this query's tree: the whole tree, or (PREFIX) the tree of its prefix
+  long long Nq = a.N;
+  bool live = valid;  // a query with a position outside the tree routes nowhere
+  if constexpr (PREFIX) {
+    const long long pos = valid ? a.positions[qg % a.nq] : 0;
+    if (valid && (pos < 0 || pos >= a.N)) {
+      if (wq == 0 && lane == 0) atomicOr(a.err, kDevErrBadLeaf);
+      live = false;
+    }
+    Nq = live ? pos + 1 : 1;
+    if (wq == 0 && lane == 0) {
+      long long* qn = reinterpret_cast<long long*>(pb + Ps.qn);
+      qn[0] = (Nq + a.lb - 1) / a.lb;
+      int L = 0;
+      do {  // L = smallest L >= 1 with b^L >= n0
+        qn[L + 1] = (qn[L] + a.b - 1) / a.b;
+        ++L;
+      } while (qn[L] > 1);
+      qn[kMaxLevels - 1] = L;
+    }
+    qsync();
+  }
+  const long long* nl = PREFIX ? reinterpret_cast<const long long*>(pb + Ps.qn) : a.n;
+  const int Lq = PREFIX ? (int)nl[kMaxLevels - 1] : a.L;
   if (wq == 0 && lane == 0) {
     mbar_init(&bar[0], 1);
     if (ATTEND)
@@ -232,14 +265,16 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         if (i > 0) mbar_init(&bar[i], 1);  // "full" (bar[0] serves the route first)
         mbar_init(&bar[3 + i], nw);        // "empty": one arrival per warp
       }
-    if (APPEND) mbar_init(pbar, 1);
+    if (HASPATH) mbar_init(pbar, 1);
     fence_mbar_init();
     surv_a[0] = 0;  // the root
-    if constexpr (APPEND) {
-      if (valid) {
+    if constexpr (HASPATH) {
+      if (live) {
         fence_proxy_async_smem();
-        path_issue<TKV, D>(Ps, pb, a.K + unit * a.kv_unit_stride, pyr_u, a.off, a.n, a.b, a.L,
-                           a.path_leaf, a.path_tokens, a.lb, pbar);
+        const long long leaf = APPEND ? a.path_leaf : (Nq - 1) / a.lb;
+        const int ntok = APPEND ? a.path_tokens : (int)(Nq - leaf * a.lb);
+        path_issue<TKV, D>(Ps, pb, a.K + unit * a.kv_unit_stride, pyr_u, a.off, nl, a.b, Lq, leaf,
+                           ntok, a.lb, pbar);
       }
     }
   }
@@ -251,13 +286,13 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   float4 qv[CPL];
   int* cur = surv_a;
   int* nxt = surv_b;
-  int m = valid ? 1 : 0;
+  int m = live ? 1 : 0;
   uint32_t parity = 0;
-  for (int l = a.L - 1; l >= 0; --l) {
+  for (int l = Lq - 1; l >= 0; --l) {
     int C = 0;
     if (m > 0) {
       const long long last = cur[m - 1];
-      C = (m - 1) * a.b + (int)min((long long)a.b, a.n[l] - (long long)a.b * last);
+      C = (m - 1) * a.b + (int)min((long long)a.b, nl[l] - (long long)a.b * last);
     }
     const float* S = pyr_u + a.off[l] * D;
     if (wq == 0 && C > 0) {
@@ -267,7 +302,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       fence_proxy_async_smem();
       for (int j = lane; j < m; j += 32) {
         const long long node0 = (long long)a.b * cur[j];
-        const int nc = (int)min((long long)a.b, a.n[l] - node0);
+        const int nc = (int)min((long long)a.b, nl[l] - node0);
         bulk_copy_g2s((void*)(rows + (size_t)j * a.b * D), S + node0 * D, (uint32_t)nc * D * 4, bar);
       }
       for (int j = lane; j < m; j += 32) {  // survivor j's children are candidates j b ..
@@ -276,7 +311,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         for (int i = 0; i < nc; ++i) cand[j * a.b + i] = node0 + i;
       }
     }
-    if (APPEND && wq == 0) {
+    if (HASPATH && wq == 0) {
       // candidate slot of the path node at this level: its parent is a survivor j, and the
       // parent's children are candidates j b .. j b + b - 1
       const long long* node = reinterpret_cast<const long long*>(pb + Ps.node);
@@ -284,12 +319,12 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       int found = -1;
       for (int j0 = 0; j0 < m; j0 += 32) {
         const int j = j0 + lane;
-        const unsigned hit = __ballot_sync(0xffffffffu, j < m && valid && cur[j] == node[l + 1]);
+        const unsigned hit = __ballot_sync(0xffffffffu, j < m && live && cur[j] == node[l + 1]);
         if (hit && found < 0) found = j0 + __ffs(hit) - 1;
       }
       if (lane == 0) kpos[0] = found < 0 ? -1 : (int)(found * a.b + (node[l] - a.b * node[l + 1]));
     }
-    if (l == a.L - 1 && valid) {  // load q while the first level is in flight
+    if (l == Lq - 1 && valid) {  // load q while the first level is in flight
       const long long qo = qg * D;
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
@@ -302,22 +337,24 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         qv[j] = make_float4(f[0], f[1], f[2], f[3]);
       }
     }
-    if (APPEND && l == a.L - 1) {
+    if (HASPATH && l == Lq - 1) {
       // the path rows, while the first level's copies are in flight
-      const bool pok = !valid || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+      const bool pok = !live || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
       const bool pfail = GROUPED ? group_any(bar_id, bar_n, !pok) : __any_sync(0xffffffffu, !pok);
       if (pfail) {
         if (wq == 0 && lane == 0) {  // let all copies land before the CTA exits
-          mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+          if (live) mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
           if (C > 0) mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
         }
         return;
       }
-      if constexpr (APPEND) {
-        if (valid) {
-          const bool writer = (qg % a.nq) == 0 && ((qg / a.nq) % a.q_heads) % a.group == 0;
-          path_compute<TKV, D>(Ps, pb, const_cast<float*>(pyr_u), a.off, a.n, a.b, a.L, a.path_tokens,
-                               writer, 32 * wq + lane, bar_n, qsync);
+      if constexpr (HASPATH) {
+        if (live) {
+          // fused append: the first query of each unit stores the path
+          const bool writer = APPEND && (qg % a.nq) == 0 && ((qg / a.nq) % a.q_heads) % a.group == 0;
+          const int ntok = APPEND ? a.path_tokens : (int)(Nq - ((Nq - 1) / a.lb) * a.lb);
+          path_compute<TKV, D>(Ps, pb, const_cast<float*>(pyr_u), a.off, nl, a.b, Lq, ntok, writer,
+                               32 * wq + lane, bar_n, qsync);
         }
       }
     }
@@ -330,8 +367,9 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     }
     if (!GROUPED) __syncwarp();  // candidate ids written by other lanes
     if (C > 0) parity ^= 1u;
-    if (APPEND) {
-      // the staged row of the path node may predate the append: use the recomputed one
+    if (HASPATH) {
+      // the staged row of the path node may predate the append, or (prefix) cover tokens
+      // past the query's prefix: use the recomputed one
       const int k = *reinterpret_cast<const int*>(pb + Ps.kpos);
       if (k >= 0) {
         const float* pf = reinterpret_cast<const float*>(pb + Ps.pf) + (size_t)l * D;
@@ -402,6 +440,11 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     cur = nxt;
     nxt = tmp;
   }
+  if (PREFIX && valid && wq == 0 && a.trace)  // levels above this query's tree
+    for (int l = Lq; l < a.L; ++l) {
+      int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+      for (int k = lane; k < a.beam; k += 32) tr[k] = -1;
+    }
   if (valid && wq == 0 && a.leaf_idx) {
     int* out = a.leaf_idx + qg * a.beam;
     for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
@@ -411,11 +454,12 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     for (int k = lane; k < a.beam; k += 32) os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
   }
   if constexpr (ATTEND) {
+    if (a.O == nullptr) return;  // route only (the path needed the K type)
     using S = AttnShape<TKV, D>;
     StagedAttn sa;
     sa.leaves = cur;
     sa.lb = (int)a.lb;
-    sa.total = leaf_tokens(cur, m, a.lb, a.N);
+    sa.total = leaf_tokens(cur, m, a.lb, Nq);
     sa.TS = a.stage_tokens;
     sa.nbuf = a.attn_nbuf;
     sa.sb = base + Ls.rows;  // the candidate rows (and the append path) are no longer needed
@@ -441,10 +485,10 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
 }
 
 namespace {
-template <int D, bool GROUPED, typename TKV, bool NARROW, bool APPEND = false>
+template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH = kPathNone>
 cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
                           cudaStream_t s) {
-  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW, APPEND>;
+  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW, PATH>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
@@ -452,30 +496,35 @@ cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size
   return cudaGetLastError();
 }
 
-template <typename TKV>
-cudaError_t run_route_tma_d(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
-                            int threads, size_t smem, cudaStream_t s, bool append = false) {
-  if constexpr (!std::is_same<TKV, NoKV>::value) {
-    if (append) {  // fused one-leaf append: wide launches only
+template <typename TKV, int PATH>
+cudaError_t run_shape(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks, int threads,
+                      size_t smem, cudaStream_t s) {
+  if constexpr (PATH != kPathAppend) {  // the fused append runs in wide launches only
+    if (narrow) {
       if (grouped)
-        return D == 128 ? run_route_tma<128, true, TKV, false, true>(a, blocks, threads, smem, s)
-                        : run_route_tma<64, true, TKV, false, true>(a, blocks, threads, smem, s);
-      return D == 128 ? run_route_tma<128, false, TKV, false, true>(a, blocks, threads, smem, s)
-                      : run_route_tma<64, false, TKV, false, true>(a, blocks, threads, smem, s);
+        return D == 128 ? run_route_tma<128, true, TKV, true, PATH>(a, blocks, threads, smem, s)
+                        : run_route_tma<64, true, TKV, true, PATH>(a, blocks, threads, smem, s);
+      return D == 128 ? run_route_tma<128, false, TKV, true, PATH>(a, blocks, threads, smem, s)
+                      : run_route_tma<64, false, TKV, true, PATH>(a, blocks, threads, smem, s);
     }
-  }
-  if (narrow) {
-    if (grouped)
-      return D == 128 ? run_route_tma<128, true, TKV, true>(a, blocks, threads, smem, s)
-                      : run_route_tma<64, true, TKV, true>(a, blocks, threads, smem, s);
-    return D == 128 ? run_route_tma<128, false, TKV, true>(a, blocks, threads, smem, s)
-                    : run_route_tma<64, false, TKV, true>(a, blocks, threads, smem, s);
+  } else if (narrow) {
+    return cudaErrorNotSupported;
   }
   if (grouped)
-    return D == 128 ? run_route_tma<128, true, TKV, false>(a, blocks, threads, smem, s)
-                    : run_route_tma<64, true, TKV, false>(a, blocks, threads, smem, s);
-  return D == 128 ? run_route_tma<128, false, TKV, false>(a, blocks, threads, smem, s)
-                  : run_route_tma<64, false, TKV, false>(a, blocks, threads, smem, s);
+    return D == 128 ? run_route_tma<128, true, TKV, false, PATH>(a, blocks, threads, smem, s)
+                    : run_route_tma<64, true, TKV, false, PATH>(a, blocks, threads, smem, s);
+  return D == 128 ? run_route_tma<128, false, TKV, false, PATH>(a, blocks, threads, smem, s)
+                  : run_route_tma<64, false, TKV, false, PATH>(a, blocks, threads, smem, s);
+}
+
+template <typename TKV>
+cudaError_t run_route_tma_d(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                            int threads, size_t smem, cudaStream_t s, int path = kPathNone) {
+  if constexpr (!std::is_same<TKV, NoKV>::value) {
+    if (path == kPathAppend) return run_shape<TKV, kPathAppend>(D, grouped, narrow, a, blocks, threads, smem, s);
+    if (path == kPathPrefix) return run_shape<TKV, kPathPrefix>(D, grouped, narrow, a, blocks, threads, smem, s);
+  }
+  return run_shape<TKV, kPathNone>(D, grouped, narrow, a, blocks, threads, smem, s);
 }
 
 template <int D, int U>
@@ -630,7 +679,7 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
   const size_t route_rows = route_rows_bytes(D, (int)cmax);
   if (!wide) {
     p.nbuf = 2;
-    p.rows_bytes = std::max(route_rows, (size_t)4 * 8 * row);
+    p.rows_bytes = std::max(route_rows, (size_t)4 * 16 * row);  // two stages of 16 tokens at least
     p.stage_tokens = (int)(p.rows_bytes / (4 * row)) / 16 * 16;
     p.attn_warps = 1;
     p.smem_per_query = route_smem_layout(D, (int)cmax, beam, p.rows_bytes, narrow_wpq(cmax)).total;
@@ -682,9 +731,73 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
   }
   cudaError_t e;
   if (bf)
-    e = run_route_tma_d<uint16_t>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, append);
+    e = run_route_tma_d<uint16_t>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream,
+                                  append ? kPathAppend : kPathNone);
   else
-    e = run_route_tma_d<float>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, append);
+    e = run_route_tma_d<float>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream,
+                               append ? kPathAppend : kPathNone);
+  ++t->launches;
+  return e;
+}
+
+// Causal routing (and, with d_O, attention): query qg routes over the tree of tokens
+// 0 .. positions[qg % nq] (kPathPrefix).  Each query's shared memory holds the route's region
+// (grown for the attention's stages when attending, as planned by plan_decode) followed by
+// the path region of its prefix's right edge.
+cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
+                          const long long* d_positions, const void* d_K, const void* d_V, float scale,
+                          int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                          zha_dtype o_dtype, cudaStream_t stream, bool* unsupported) {
+  *unsupported = false;
+  RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, d_trace);
+  const int D = t->desc.head_dim;
+  const bool bf = t->desc.kv_dtype == ZHA_BF16;
+  const int row = D * (bf ? 2 : 4);
+  const bool attend = d_O != nullptr;
+  const DecodePlan dp = plan_decode(t, q_heads, nq, beam);
+  const bool wide = a.total_queries <= 2LL * t->sms;
+  // Route only: the route's rows.  Attending: the decode plan's row region; in narrow
+  // launches grown up to 64 KB, and any number of stages is accepted (the attention
+  // pipelines them), since a causal pass has no two-launch fallback.
+  size_t rows = std::max(route_rows_bytes(D, a.cmax), (size_t)4 * 16 * row);
+  int nbuf = 2, stage_tokens = (int)(rows / (4 * row)) / 16 * 16;
+  if (attend) {
+    rows = dp.rows_bytes;
+    nbuf = dp.nbuf;
+    stage_tokens = dp.stage_tokens;
+    if (!wide) {
+      const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
+      rows = std::max(rows, std::min((size_t)2 * row * (size_t)tokens, (size_t)64 * 1024));
+      stage_tokens = (int)(rows / (4 * row)) / 16 * 16;
+    }
+  }
+  a.rows_bytes = (int)rows;
+  a.K = static_cast<const char*>(d_K);
+  a.V = static_cast<const char*>(d_V);
+  a.kv_unit_stride = t->desc.capacity_tokens * D * (bf ? 2LL : 4LL);
+  a.lb = t->desc.leaf_block;
+  a.N = t->N;
+  a.qk_scale = scale * 1.4426950408889634f;
+  a.stage_tokens = stage_tokens;
+  a.attn_nbuf = nbuf;
+  a.O = d_O;
+  a.o_bf16 = o_dtype == ZHA_BF16;
+  a.positions = d_positions;
+  const int pw_warps = wide ? kRouteMaxWarps : narrow_wpq(a.cmax);
+  const size_t route_part = route_smem_layout(D, a.cmax, beam, (size_t)a.rows_bytes, pw_warps).total;
+  const size_t path_bytes = path_smem_layout(D, row, (int)a.lb, a.b, t->L).total;
+  a.path_smem_off = (long long)route_align(route_part, 128);
+  const size_t per_query = (size_t)a.path_smem_off + path_bytes;
+  if ((attend && stage_tokens < 16) || per_query > (wide ? kCtaSmemCap : kRouteSmemCap)) {
+    *unsupported = true;
+    return cudaSuccess;
+  }
+  a.query_smem_bytes = (int)per_query;
+  const StagedShape sh = staged_shape(t, a, per_query, attend ? dp.attn_warps : 0);
+  cudaError_t e = bf ? run_route_tma_d<uint16_t>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem,
+                                                 stream, kPathPrefix)
+                     : run_route_tma_d<float>(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem,
+                                              stream, kPathPrefix);
   ++t->launches;
   return e;
 }

@@ -49,9 +49,14 @@ struct RouteArgs {
   long long path_leaf;       // the leaf that received the new tokens
   int path_tokens;           // its tokens after the append
   long long path_smem_off;   // byte offset of the path region in a query's shared memory
+  // causal routing (kPathPrefix): query qg routes over tokens 0 .. positions[qg % nq]
+  const long long* positions;
 };
 
 struct NoKV {};  // route only: no attention epilogue
+
+// What the route kernel does besides routing the stored tree (decode_append.cuh).
+enum : int { kPathNone = 0, kPathAppend = 1, kPathPrefix = 2 };
 
 
 constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz

@@ -241,6 +241,46 @@ zha_status zha_decode_step(zha_tree* t, const void* d_K, const void* d_V, long l
                     d_trace, d_O, o_dtype, stream);
 }
 
+static zha_status causal_call(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                              const long long* d_positions, int beam, const void* d_K, const void* d_V,
+                              float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                              zha_dtype o_dtype, void* stream) {
+  if (!t || !dtype_ok(q_dtype) || !dtype_ok(o_dtype) || q_heads < 1 || nq < 0) return ZHA_ERR_INVALID_ARG;
+  if (q_heads % t->desc.kv_heads != 0) return ZHA_ERR_INVALID_ARG;
+  if (beam < 1 || beam > kMaxBeam) return ZHA_ERR_INVALID_ARG;
+  if ((long long)beam * t->desc.branching > kMaxCandidates) return ZHA_ERR_UNSUPPORTED;
+  if (t->N == 0) return ZHA_ERR_INVALID_ARG;
+  if (d_O && !(scale == scale)) return ZHA_ERR_INVALID_ARG;
+  if (nq == 0) return ZHA_OK;
+  if (!d_Q || !d_K || !d_positions || !d_leaf_idx || (d_O && !d_V)) return ZHA_ERR_INVALID_ARG;
+  if (!aligned(d_Q, 16) || !aligned(d_K, 16) || !aligned(d_positions, 8) || !aligned(d_leaf_idx, 4) ||
+      (d_O && (!aligned(d_O, 16) || !aligned(d_V, 16))) || (d_leaf_score && !aligned(d_leaf_score, 4)) ||
+      (d_trace && !aligned(d_trace, 4)))
+    return ZHA_ERR_INVALID_ARG;
+  bool unsupported = false;
+  const cudaError_t e = launch_causal(const_cast<zha_tree*>(t), d_Q, q_dtype, q_heads, nq, beam, d_positions,
+                                      d_K, d_V, scale, d_leaf_idx, d_leaf_score, d_trace, d_O, o_dtype,
+                                      static_cast<cudaStream_t>(stream), &unsupported);
+  if (unsupported) return ZHA_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+zha_status zha_route_causal(const zha_tree* t, const void* d_K, const void* d_Q, zha_dtype q_dtype,
+                            int q_heads, int nq, const long long* d_positions, int beam, int* d_leaf_idx,
+                            float* d_leaf_score, int* d_trace, void* stream) {
+  return causal_call(t, d_Q, q_dtype, q_heads, nq, d_positions, beam, d_K, nullptr, 1.0f, d_leaf_idx,
+                     d_leaf_score, d_trace, nullptr, ZHA_F32, stream);
+}
+
+zha_status zha_decode_causal(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                             const long long* d_positions, int beam, const void* d_K, const void* d_V,
+                             float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                             zha_dtype o_dtype, void* stream) {
+  if (!d_O) return ZHA_ERR_INVALID_ARG;
+  return causal_call(t, d_Q, q_dtype, q_heads, nq, d_positions, beam, d_K, d_V, scale, d_leaf_idx,
+                     d_leaf_score, d_trace, d_O, o_dtype, stream);
+}
+
 zha_status zha_tree_check(zha_tree* t, void* stream) {
   if (!t) return ZHA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -92,6 +92,14 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
                           void* d_O, zha_dtype o_dtype, cudaStream_t stream,
                           long long append_leaf = -1);
 
+// Causal routing (route.cu): query qg of every head routes over the tree of tokens
+// 0 .. positions[qg % nq], and attends over its leaves' tokens in that prefix when d_O is
+// given.  *unsupported: the shape does not fit the staged kernel (nothing launched).
+cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
+                          const long long* d_positions, const void* d_K, const void* d_V, float scale,
+                          int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
+                          zha_dtype o_dtype, cudaStream_t stream, bool* unsupported);
+
 // Attention (attend.cu).
 struct AttnPlan {
   int leaves_per_split;

@@ -27,7 +27,7 @@ EXPORTED = [
     "zha_tree_check", "zha_tree_seq_len", "zha_tree_levels", "zha_tree_level_nodes",
     "zha_tree_level_offset", "zha_tree_unit_rows", "zha_tree_summaries", "zha_tree_launch_count",
     "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
-    "zha_decode", "zha_decode_step",
+    "zha_decode", "zha_decode_step", "zha_route_causal", "zha_decode_causal",
 ]
 
 
@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
                                 _P]),
             "zha_decode_step": (_I, [_P, _P, _P, _LL, _P, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P,
                                      _P, _I, _P]),
+            "zha_route_causal": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
+            "zha_decode_causal": (_I, [_P, _P, _I, _I, _I, _P, _I, _P, _P, ctypes.c_float, _P, _P, _P,
+                                       _P, _I, _P]),
             "zha_tree_check": (_I, [_P, _P]),
             "zha_tree_seq_len": (_LL, [_P]),
             "zha_tree_levels": (_I, [_P]),
@@ -202,6 +205,27 @@ def zha_decode_step(handle, K: torch.Tensor, V: torch.Tensor, new_seq_len: int, 
     _check(lib().zha_decode_step(handle, _ptr(K), _ptr(V), new_seq_len, _ptr(Q), dtype_code(Q.dtype),
                                  Hq, nq, beam, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
                                  _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_step")
+
+
+def zha_route_causal(handle, K: torch.Tensor, Q: torch.Tensor, positions: torch.Tensor, beam: int,
+                     leaf_idx: torch.Tensor, leaf_score: torch.Tensor | None = None,
+                     trace: torch.Tensor | None = None, stream=None) -> None:
+    """Query i of every head routes over the tree of tokens 0 .. positions[i] (int64, device)."""
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_route_causal(handle, _ptr(K), _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions),
+                                  beam, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _stream(stream)),
+           "zha_route_causal")
+
+
+def zha_decode_causal(handle, Q: torch.Tensor, positions: torch.Tensor, beam: int, K: torch.Tensor,
+                      V: torch.Tensor, scale: float, leaf_idx: torch.Tensor, O: torch.Tensor,
+                      leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
+                      stream=None) -> None:
+    """Causal routing + attention over each query's prefix, one launch."""
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_decode_causal(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions), beam,
+                                   _ptr(K), _ptr(V), scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
+                                   _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_causal")
 
 
 def zha_noalloc_scratch_capacity() -> int:
@@ -360,6 +384,25 @@ class Tree:
             tr = torch.empty((B, Hq, nq, L, beam), dtype=torch.int32, device=Q.device)
         zha_decode_step(self.handle, K, V, new_seq_len, Q, beam, scale, idx, O, None, tr, stream)
         return (O, idx, tr) if trace else (O, idx)
+
+    def route_causal(self, K: torch.Tensor, Q: torch.Tensor, positions: torch.Tensor, beam: int,
+                     trace: bool = False, stream=None):
+        """Causal routing; returns (leaf_idx, trace or None)."""
+        B, Hq, nq, _ = Q.shape
+        idx = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=Q.device)
+        tr = (torch.empty((B, Hq, nq, max(self.levels, 1), beam), dtype=torch.int32, device=Q.device)
+              if trace else None)
+        zha_route_causal(self.handle, K, Q, positions, beam, idx, None, tr, stream)
+        return idx, tr
+
+    def decode_causal(self, Q: torch.Tensor, positions: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                      beam: int, scale: float, out_dtype: torch.dtype = torch.bfloat16, stream=None):
+        """Causal routing + attention; returns (O, leaf_idx)."""
+        B, Hq, nq, d = Q.shape
+        idx = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=Q.device)
+        O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
+        zha_decode_causal(self.handle, Q, positions, beam, K, V, scale, idx, O, None, None, stream)
+        return O, idx
 
     def check(self, stream=None) -> int:
         return zha_tree_check(self.handle, stream)
