@@ -69,6 +69,15 @@ def _load():
                                    ctypes.c_double, _P]
         lib.orc_dense.restype = None
         lib.orc_dense.argtypes = [_P, _P, _P, ctypes.c_int, _I64, _I64, ctypes.c_double, _P]
+        lib.orc_leaf_radii.restype = None
+        lib.orc_leaf_radii.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P, _I64, _P]
+        lib.orc_parent_radii.restype = None
+        lib.orc_parent_radii.argtypes = [_P, _P, _I64, _P, _I64, _I64, _I64, _P]
+        lib.orc_threshold_brute.restype = _I64
+        lib.orc_threshold_brute.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, ctypes.c_double, _P, _I64]
+        lib.orc_threshold_descent.restype = _I64
+        lib.orc_threshold_descent.argtypes = [_P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P,
+                                              ctypes.c_int, _P, ctypes.c_double, _P, _I64, _P]
         _lib = lib
     return _lib
 
@@ -184,6 +193,39 @@ class OracleTree:
         off = np.concatenate([[0], np.cumsum(cnt)[:-1]]).astype(np.int64)
         return np.ascontiguousarray(np.concatenate(self.levels, axis=0)), off, cnt
 
+    def radii(self, K: np.ndarray) -> list[np.ndarray]:
+        """Bounding-sphere radius of every node, per level (centers = the summaries): leaves
+        cover their tokens, a parent covers its children's spheres (orc_leaf_radii,
+        orc_parent_radii)."""
+        Kv, dt = _kv_view(K)
+        lib = _load()
+        out = [np.empty(self.levels[0].shape[0], np.float64)]
+        c0 = np.ascontiguousarray(self.levels[0])
+        lib.orc_leaf_radii(_ptr(Kv), dt, self.d, self.N, self.lb, _ptr(c0), c0.shape[0], _ptr(out[0]))
+        for lvl in range(1, self.L + 1):
+            cc = np.ascontiguousarray(self.levels[lvl - 1])
+            pc = np.ascontiguousarray(self.levels[lvl])
+            r = np.empty(pc.shape[0], np.float64)
+            lib.orc_parent_radii(_ptr(cc), _ptr(out[-1]), cc.shape[0], _ptr(pc), pc.shape[0], self.d, self.b,
+                                 _ptr(r))
+            out.append(r)
+        return out
+
+    def threshold(self, K: np.ndarray, q: np.ndarray, tau: float, radii=None, max_out: int | None = None):
+        """Threshold descent: (tokens t < N with q . k_t >= tau, ascending; sphere tests)."""
+        Kv, dt = _kv_view(K)
+        q = np.ascontiguousarray(q, dtype=np.float64).reshape(-1)
+        radii = radii if radii is not None else self.radii(K)
+        rows, off, cnt = self.flat()
+        rad = np.ascontiguousarray(np.concatenate(radii))
+        cap = self.N if max_out is None else max_out
+        out = np.empty(max(cap, 1), np.int64)
+        tested = np.zeros(1, np.int64)
+        n = _load().orc_threshold_descent(_ptr(rows), _ptr(rad), _ptr(off), _ptr(cnt), self.L, self.d, self.b,
+                                          self.lb, self.N, _ptr(Kv), dt, _ptr(q), float(tau), _ptr(out), cap,
+                                          _ptr(tested))
+        return out[:min(n, cap)].copy(), int(tested[0])
+
     def route(self, Q: np.ndarray, beam: int, flat=None):
         """Beam descent for queries Q ([nq, d], any float dtype, converted to fp64).
 
@@ -210,6 +252,15 @@ class OracleTree:
             raise RuntimeError("orc_route failed")
         return {"leaves": leaves, "leaf_scores": scores, "bounds": bounds,
                 "survivors": surv, "ncand": ncand}
+
+
+def threshold_brute(q: np.ndarray, K: np.ndarray, N: int, tau: float) -> np.ndarray:
+    """Every token t < N with q . k_t >= tau (fp64 scan of all keys), ascending."""
+    Kv, dt = _kv_view(K)
+    q = np.ascontiguousarray(q, dtype=np.float64).reshape(-1)
+    out = np.empty(max(N, 1), np.int64)
+    n = _load().orc_threshold_brute(_ptr(Kv), dt, q.shape[0], N, _ptr(q), float(tau), _ptr(out), N)
+    return out[:n].copy()
 
 
 def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int, leaf_block: int,

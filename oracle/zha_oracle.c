@@ -21,6 +21,10 @@
  *     node) is not scored, routing starts from its children;
  *   - final attention: exact softmax over the union of the tokens of the
  *     selected leaves, two passes (max, then exp/sum/weighted V).
+ *   - threshold descent ("Louver" explainer): bounding spheres centered on the
+ *     summaries (leaf radius: farthest token; node radius: farthest child sphere),
+ *     a child kept iff q . c + ||q|| r >= tau, exact check of the surviving
+ *     leaves' tokens; pinned against a scan of all keys.
  *
  * Every computation is a plain loop in fp64 over inputs converted exactly
  * (bf16 -> fp64 and fp32 -> fp64 are exact).  One library routine is used:
@@ -250,4 +254,122 @@ void orc_dense(const double *q, const void *K, const void *V, int dtype, int64_t
   if (N > 0)
     for (int64_t k = 0; k < d; ++k) out[k] /= den;
   free(s);
+}
+
+/*
+ * Bounding spheres and threshold descent ("Louver" explainer, index design: every cluster
+ * of keys is enclosed in a bounding sphere with a center and a radius; a query with
+ * threshold tau wants every key in the halfspace {p : q . p >= tau}; a cluster whose sphere
+ * misses the halfspace is pruned, the keys of the others are checked exactly, so no key
+ * with q . k >= tau is missed).  On this tree the center of a node is its summary and the
+ * radius covers every key of its subtree:
+ *   leaf i:  r = max over its tokens t < N of ||k_t - c_i||
+ *   node i:  r = max over its existing children j of (||c_j - c_i|| + r_j)
+ * (a child's sphere lies inside the ball of radius ||c_j - c_i|| + r_j around c_i, by the
+ * triangle inequality, so the node's sphere contains all of its subtree's keys).
+ */
+
+/* Radii of leaves [0, n0): centers [n0][d] (the leaf summaries). */
+void orc_leaf_radii(const void *K, int dtype, int64_t d, int64_t N, int64_t lb, const double *centers,
+                    int64_t n0, double *out) {
+  for (int64_t i = 0; i < n0; ++i) {
+    int64_t t0 = i * lb, t1 = t0 + lb < N ? t0 + lb : N;
+    double best = 0.0;
+    for (int64_t t = t0; t < t1; ++t) {
+      double s = 0.0;
+      for (int64_t k = 0; k < d; ++k) {
+        double e = in_elem(K, dtype, t * d + k) - centers[i * d + k];
+        s += e * e;
+      }
+      if (s > best) best = s;
+    }
+    out[i] = sqrt(best);
+  }
+}
+
+/* Radii of the parents [0, n_parent) of children [0, n_child) (centers and radii given). */
+void orc_parent_radii(const double *child_c, const double *child_r, int64_t n_child, const double *parent_c,
+                      int64_t n_parent, int64_t d, int64_t b, double *out) {
+  for (int64_t i = 0; i < n_parent; ++i) {
+    int64_t j0 = i * b, j1 = j0 + b < n_child ? j0 + b : n_child;
+    double best = 0.0;
+    for (int64_t j = j0; j < j1; ++j) {
+      double s = 0.0;
+      for (int64_t k = 0; k < d; ++k) {
+        double e = child_c[j * d + k] - parent_c[i * d + k];
+        s += e * e;
+      }
+      double r = sqrt(s) + child_r[j];
+      if (r > best) best = r;
+    }
+    out[i] = best;
+  }
+}
+
+/* Every token t < N with q . k_t >= tau, ascending (up to max_out written); returns the count. */
+int64_t orc_threshold_brute(const void *K, int dtype, int64_t d, int64_t N, const double *q, double tau,
+                            int64_t *out, int64_t max_out) {
+  int64_t n = 0;
+  for (int64_t t = 0; t < N; ++t) {
+    double s = 0.0;
+    for (int64_t k = 0; k < d; ++k) s += q[k] * in_elem(K, dtype, t * d + k);
+    if (s >= tau) {
+      if (n < max_out) out[n] = t;
+      n++;
+    }
+  }
+  return n;
+}
+
+/*
+ * Threshold descent over a tree (pyr: every level's summaries, level l at rows off[l] ..,
+ * cnt[l] nodes; radii in the same row order).  Survivors start as {root}; for l = L-1 .. 0
+ * the children of the survivors are kept iff q . c + ||q|| r >= tau.  The tokens of the
+ * surviving leaves are then checked exactly.  Writes the tokens found in ascending order (up
+ * to max_out), returns their count; *tested = number of sphere tests.
+ */
+int64_t orc_threshold_descent(const double *pyr, const double *radii, const int64_t *off, const int64_t *cnt,
+                              int L, int64_t d, int64_t b, int64_t lb, int64_t N, const void *K, int dtype,
+                              const double *q, double tau, int64_t *out, int64_t max_out, int64_t *tested) {
+  double qn = 0.0;
+  for (int64_t k = 0; k < d; ++k) qn += q[k] * q[k];
+  qn = sqrt(qn);
+  int64_t cap = cnt[0] + 1;
+  int64_t *cur = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
+  int64_t *nxt = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
+  int64_t m = 1, ntest = 0;
+  cur[0] = 0;
+  for (int l = L - 1; l >= 0; --l) {
+    int64_t mn = 0;
+    for (int64_t j = 0; j < m; ++j) {
+      int64_t c0 = cur[j] * b, c1 = c0 + b < cnt[l] ? c0 + b : cnt[l];
+      for (int64_t c = c0; c < c1; ++c) {
+        const double *row = pyr + (off[l] + c) * d;
+        double s = 0.0;
+        for (int64_t k = 0; k < d; ++k) s += q[k] * row[k];
+        ntest++;
+        if (s + qn * radii[off[l] + c] >= tau) nxt[mn++] = c;
+      }
+    }
+    int64_t *tmp = cur;
+    cur = nxt;
+    nxt = tmp;
+    m = mn;
+  }
+  int64_t n = 0;
+  for (int64_t j = 0; j < m; ++j) {
+    int64_t t0 = cur[j] * lb, t1 = t0 + lb < N ? t0 + lb : N;
+    for (int64_t t = t0; t < t1; ++t) {
+      double s = 0.0;
+      for (int64_t k = 0; k < d; ++k) s += q[k] * in_elem(K, dtype, t * d + k);
+      if (s >= tau) {
+        if (n < max_out) out[n] = t;
+        n++;
+      }
+    }
+  }
+  free(cur);
+  free(nxt);
+  if (tested) *tested = ntest;
+  return n;
 }

@@ -19,6 +19,7 @@ import pytest
 from scipy.special import softmax
 
 import oracle
+from tree_indexed_sparse_build_b200 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_tree.json")
 
@@ -318,3 +319,85 @@ def test_route_pads_when_fewer_leaves_than_beam():
     res = t.route(rng.standard_normal((2, d)), 5)
     assert (res["leaves"][:, :3] == np.arange(3)).all()
     assert (res["leaves"][:, 3:] == -1).all()
+
+
+# ---------------------------------------------------------------- threshold descent
+# Bounding spheres centered on the summaries ("Louver" explainer, index design): a leaf's
+# radius covers its tokens, a parent's covers its children's spheres; a node is expanded
+# iff q . c + ||q|| r >= tau, the surviving leaves' tokens are checked exactly.  Pinned
+# against direct numpy geometry and a scan of all keys.
+
+def _subtree_tokens(lvl, i, b, lb, N):
+    span = lb * b ** lvl
+    return i * span, min((i + 1) * span, N)
+
+
+@pytest.mark.parametrize("b,lb,N", [(2, 4, 37), (3, 5, 200), (8, 16, 1000)])
+def test_radii_bound_every_key_and_leaf_radius_is_farthest_token(b, lb, N):
+    rng = np.random.default_rng(b * 100 + lb)
+    d = 8
+    K = rng.standard_normal((N, d)).astype(np.float32)
+    t = oracle.OracleTree(d, lb, b).build(K, N)
+    radii = t.radii(K)
+    K64 = K.astype(np.float64)
+    for lvl, (cent, rad) in enumerate(zip(t.levels, radii)):
+        for i in range(cent.shape[0]):
+            t0, t1 = _subtree_tokens(lvl, i, b, lb, N)
+            far = np.linalg.norm(K64[t0:t1] - cent[i], axis=1).max()
+            assert far <= rad[i] * (1 + 1e-12) + 1e-15
+            if lvl == 0:
+                assert rad[i] == pytest.approx(far, rel=1e-12, abs=1e-15)
+
+
+def test_radii_hand_example():
+    # keys (0,0), (4,0), (0,3), (0,3) with leaf block 2, b = 2:
+    # leaf 0 = mean of (0,0), (4,0) = (2,0), radius 2; leaf 1 = (0,3), radius 0;
+    # root = mean of leaves = (1, 1.5); radius = max(||(2,0)-(1,1.5)|| + 2, ||(0,3)-(1,1.5)|| + 0)
+    #      = max(sqrt(3.25) + 2, sqrt(3.25)) = sqrt(3.25) + 2
+    K = np.array([[0, 0], [4, 0], [0, 3], [0, 3]], np.float32)
+    t = oracle.OracleTree(2, 2, 2).build(K, 4)
+    r = t.radii(K)
+    assert r[0].tolist() == [2.0, 0.0]
+    assert r[1][0] == pytest.approx(np.sqrt(3.25) + 2.0, rel=1e-15)
+    # tau = 2.5 with q = (1, 0): only (4,0) qualifies; leaf 1's sphere (x = 0) is pruned
+    toks, tested = t.threshold(K, np.array([1.0, 0.0]), 2.5)
+    assert toks.tolist() == [1]
+    assert tested == 2  # the two leaves are tested, the root is not scored
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("b,lb,N", [(2, 1, 50), (2, 16, 1024), (3, 7, 500), (8, 4, 3000)])
+def test_threshold_descent_equals_scan_of_all_keys(dt, b, lb, N):
+    rng = np.random.default_rng(N + b)
+    d = 16
+    K32 = rng.standard_normal((N, d)).astype(np.float32)
+    K = synth.round_to(K32.astype(np.float64), "bf16") if dt == "bf16" else K32
+    Kf = synth.to_f64(K)
+    t = oracle.OracleTree(d, lb, b).build(K, N)
+    radii = t.radii(K)
+    for trial in range(6):
+        q = rng.standard_normal(d)
+        s = np.sort(Kf @ q)
+        # thresholds between neighbouring scores (never on one): none, all, a few, many
+        taus = [s[-1] + 1.0, s[0] - 1.0] + [(s[-k] + s[-k - 1]) / 2 for k in (1, 5, N // 3)]
+        for tau in taus:
+            got, tested = t.threshold(K, q, tau, radii=radii)
+            np.testing.assert_array_equal(got, oracle.threshold_brute(q, K, N, tau))
+            assert tested <= sum(lv.shape[0] for lv in t.levels) - 1
+
+
+def test_threshold_descent_prunes_clustered_keys():
+    # 64 tight clusters of 16 keys (one per leaf) around spread-out centers: a query aimed
+    # at one cluster with a threshold only that cluster reaches tests far fewer spheres
+    # than the tree has nodes
+    rng = np.random.default_rng(7)
+    d, lb = 16, 16
+    centers = rng.standard_normal((64, d)) * 10
+    K = (np.repeat(centers, lb, axis=0) + 0.01 * rng.standard_normal((64 * lb, d))).astype(np.float32)
+    t = oracle.OracleTree(d, lb, 2).build(K, K.shape[0])
+    q = centers[17] / np.linalg.norm(centers[17])
+    tau = q @ centers[17] - 0.5
+    got, tested = t.threshold(K, q, tau)
+    np.testing.assert_array_equal(got, oracle.threshold_brute(q, K, K.shape[0], tau))
+    assert 17 * lb <= got.min() and got.max() < 18 * lb
+    assert tested < 0.5 * sum(lv.shape[0] for lv in t.levels)
