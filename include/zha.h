@@ -210,6 +210,33 @@ zha_status zha_decode_causal(const zha_tree* tree, const void* d_Q, zha_dtype q_
                              float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
                              zha_dtype o_dtype, void* stream);
 
+/* Bounding spheres for threshold descent ("Louver" explainer: every cluster of keys is
+ * enclosed in a sphere, a center and a radius).  The center of a node is its summary; the
+ * radius covers every key of its subtree (leaf: its farthest token; node: its farthest
+ * child sphere, ||c_child - c|| + r_child), stored as fp32 rounded up.  The radii live in a
+ * caller-owned device buffer of zha_tree_radii_bytes(tree) bytes ([units][unit_rows] fp32,
+ * rows as in zha_tree_summaries), 16-byte aligned.  zha_tree_attach_radii computes them for
+ * the current tree (d_K: the cache it was built over; may be NULL while the tree is empty);
+ * afterwards zha_tree_build, zha_tree_append and zha_decode_step keep them current (the
+ * latter then appends and decodes in two launches).  d_radii = NULL detaches. */
+size_t zha_tree_radii_bytes(const zha_tree* tree);
+zha_status zha_tree_attach_radii(zha_tree* tree, float* d_radii, size_t bytes, const void* d_K, void* stream);
+
+/* Threshold (halfspace) descent: for every query, all tokens t < seq_len with
+ * q . K[t] >= tau (unscaled dot product), found by descending the tree and pruning a node
+ * whose sphere cannot reach the threshold (q . c + ||q|| r < tau), then checking the tokens
+ * of the surviving leaves exactly (fp64).  No key with q . k >= tau is missed.
+ *   d_tau      [batch, q_heads, nq] fp32 thresholds, device
+ *   d_tokens   out [batch, q_heads, nq, max_tokens] int32: the tokens found, ascending, -1 after
+ *   d_count    out [batch, q_heads, nq] int32: how many were found (may exceed max_tokens; the
+ *              list then holds the first max_tokens); -1 when a level kept more than 8,192 nodes
+ *              (the descent stops; widen the threshold or route with zha_route)
+ *   d_stats    out, nullable: [batch, q_heads, nq, 2] int32: spheres tested, tokens checked
+ * Requires radii attached (zha_tree_attach_radii) and a non-empty tree. */
+zha_status zha_threshold_route(const zha_tree* tree, const void* d_K, const void* d_Q, zha_dtype q_dtype,
+                               int q_heads, int nq, const float* d_tau, int max_tokens, int* d_tokens,
+                               int* d_count, int* d_stats, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word:
  * ZHA_OK, ZHA_ERR_TIMEOUT or ZHA_ERR_DEVICE (or ZHA_ERR_CUDA if the stream failed). */
 zha_status zha_tree_check(zha_tree* tree, void* stream);

@@ -108,8 +108,10 @@ zha_status zha_tree_build(zha_tree* t, const void* d_K, long long seq_len, void*
   if (seq_len > 0 && (!d_K || !aligned(d_K, 16))) return ZHA_ERR_INVALID_ARG;
   set_shape(t, seq_len);
   if (seq_len == 0) return ZHA_OK;
-  return cuda_status(launch_pyramid(t, d_K, seq_len, 0, t->n[0] - 1,
-                                    static_cast<cudaStream_t>(stream), nullptr));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_pyramid(t, d_K, seq_len, 0, t->n[0] - 1, st, nullptr);
+  if (e == cudaSuccess) e = launch_radii(t, d_K, 0, t->n[0] - 1, st);
+  return cuda_status(e);
 }
 
 zha_status zha_tree_append(zha_tree* t, const void* d_K, long long new_seq_len, void* stream) {
@@ -121,8 +123,10 @@ zha_status zha_tree_append(zha_tree* t, const void* d_K, long long new_seq_len, 
   const long long lo = t->N / t->desc.leaf_block;
   const long long hi = (new_seq_len - 1) / t->desc.leaf_block;
   set_shape(t, new_seq_len);
-  return cuda_status(
-      launch_pyramid(t, d_K, new_seq_len, lo, hi, static_cast<cudaStream_t>(stream), nullptr));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_pyramid(t, d_K, new_seq_len, lo, hi, st, nullptr);
+  if (e == cudaSuccess) e = launch_radii(t, d_K, lo, hi, st);
+  return cuda_status(e);
 }
 
 zha_status zha_route(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
@@ -225,7 +229,8 @@ zha_status zha_decode_step(zha_tree* t, const void* d_K, const void* d_V, long l
     return ZHA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long lb = t->desc.leaf_block;
-  const bool one_leaf = t->N > 0 && new_seq_len > t->N && t->N / lb == (new_seq_len - 1) / lb;
+  // (a tree with radii attached takes the two launches: the fused append does not update them)
+  const bool one_leaf = t->N > 0 && new_seq_len > t->N && t->N / lb == (new_seq_len - 1) / lb && !t->radii;
   if (one_leaf && nq > 0) {
     zha_tree saved = *t;
     set_shape(t, new_seq_len);
@@ -279,6 +284,38 @@ zha_status zha_decode_causal(const zha_tree* t, const void* d_Q, zha_dtype q_dty
   if (!d_O) return ZHA_ERR_INVALID_ARG;
   return causal_call(t, d_Q, q_dtype, q_heads, nq, d_positions, beam, d_K, d_V, scale, d_leaf_idx,
                      d_leaf_score, d_trace, d_O, o_dtype, stream);
+}
+
+size_t zha_tree_radii_bytes(const zha_tree* t) {
+  return t ? (size_t)t->units * (size_t)t->unit_rows * sizeof(float) : 0;
+}
+
+zha_status zha_tree_attach_radii(zha_tree* t, float* d_radii, size_t bytes, const void* d_K, void* stream) {
+  if (!t) return ZHA_ERR_INVALID_ARG;
+  if (!d_radii) {
+    t->radii = nullptr;
+    return ZHA_OK;
+  }
+  if (!aligned(d_radii, 16) || bytes < zha_tree_radii_bytes(t)) return ZHA_ERR_INVALID_ARG;
+  if (t->N > 0 && (!d_K || !aligned(d_K, 16))) return ZHA_ERR_INVALID_ARG;
+  t->radii = d_radii;
+  if (t->N == 0) return ZHA_OK;
+  return cuda_status(launch_radii(t, d_K, 0, t->n[0] - 1, static_cast<cudaStream_t>(stream)));
+}
+
+zha_status zha_threshold_route(const zha_tree* t, const void* d_K, const void* d_Q, zha_dtype q_dtype,
+                               int q_heads, int nq, const float* d_tau, int max_tokens, int* d_tokens,
+                               int* d_count, int* d_stats, void* stream) {
+  if (!t || !dtype_ok(q_dtype) || q_heads < 1 || nq < 0 || max_tokens < 1) return ZHA_ERR_INVALID_ARG;
+  if (q_heads % t->desc.kv_heads != 0) return ZHA_ERR_INVALID_ARG;
+  if (t->N == 0 || !t->radii) return ZHA_ERR_INVALID_ARG;
+  if (nq == 0) return ZHA_OK;
+  if (!d_K || !d_Q || !d_tau || !d_tokens || !d_count) return ZHA_ERR_INVALID_ARG;
+  if (!aligned(d_K, 16) || !aligned(d_Q, 16) || !aligned(d_tau, 4) || !aligned(d_tokens, 4) ||
+      !aligned(d_count, 4) || (d_stats && !aligned(d_stats, 4)))
+    return ZHA_ERR_INVALID_ARG;
+  return cuda_status(launch_threshold(const_cast<zha_tree*>(t), d_K, d_Q, q_dtype, q_heads, nq, d_tau, max_tokens,
+                                      d_tokens, d_count, d_stats, static_cast<cudaStream_t>(stream)));
 }
 
 zha_status zha_tree_check(zha_tree* t, void* stream) {

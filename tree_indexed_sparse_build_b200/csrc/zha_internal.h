@@ -51,6 +51,7 @@ struct zha_tree {
   int L;                       // current levels (root at level L); 0 when empty
   long long n[zha::kMaxLevels];     // current nodes per level
   long long launches;          // kernels launched through this handle
+  float* radii;                // caller's bounding-sphere radii [units][unit_rows], or null
   int sms;                     // SMs of the device the tree was created on
   int device;
 };
@@ -99,6 +100,15 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
                           const long long* d_positions, const void* d_K, const void* d_V, float scale,
                           int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
                           zha_dtype o_dtype, cudaStream_t stream, bool* unsupported);
+
+// Bounding-sphere radii (radii.cu): recompute leaves [lo, hi] of every unit and all their
+// ancestors (no-op without radii attached).
+cudaError_t launch_radii(zha_tree* t, const void* d_K, long long lo, long long hi, cudaStream_t s);
+
+// Threshold descent (threshold.cu): every token t < N with q . k_t >= tau per query.
+cudaError_t launch_threshold(zha_tree* t, const void* d_K, const void* d_Q, zha_dtype q_dtype, int q_heads,
+                             int nq, const float* d_tau, int max_tokens, int* d_tokens, int* d_count,
+                             int* d_stats, cudaStream_t stream);
 
 // Attention (attend.cu).
 struct AttnPlan {

@@ -28,6 +28,7 @@ EXPORTED = [
     "zha_tree_level_offset", "zha_tree_unit_rows", "zha_tree_summaries", "zha_tree_launch_count",
     "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
     "zha_decode", "zha_decode_step", "zha_route_causal", "zha_decode_causal",
+    "zha_tree_radii_bytes", "zha_tree_attach_radii", "zha_threshold_route",
 ]
 
 
@@ -73,6 +74,9 @@ def lib() -> ctypes.CDLL:
             "zha_decode_step": (_I, [_P, _P, _P, _LL, _P, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P,
                                      _P, _I, _P]),
             "zha_route_causal": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
+            "zha_tree_radii_bytes": (_SZ, [_P]),
+            "zha_tree_attach_radii": (_I, [_P, _P, _SZ, _P, _P]),
+            "zha_threshold_route": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
             "zha_decode_causal": (_I, [_P, _P, _I, _I, _I, _P, _I, _P, _P, ctypes.c_float, _P, _P, _P,
                                        _P, _I, _P]),
             "zha_tree_check": (_I, [_P, _P]),
@@ -228,6 +232,25 @@ def zha_decode_causal(handle, Q: torch.Tensor, positions: torch.Tensor, beam: in
                                    _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_causal")
 
 
+def zha_tree_radii_bytes(handle) -> int:
+    return int(lib().zha_tree_radii_bytes(handle))
+
+
+def zha_tree_attach_radii(handle, radii: torch.Tensor | None, K: torch.Tensor | None, stream=None) -> None:
+    nbytes = 0 if radii is None else radii.numel() * radii.element_size()
+    _check(lib().zha_tree_attach_radii(handle, _ptr(radii), nbytes, _ptr(K), _stream(stream)),
+           "zha_tree_attach_radii")
+
+
+def zha_threshold_route(handle, K: torch.Tensor, Q: torch.Tensor, tau: torch.Tensor, max_tokens: int,
+                        tokens: torch.Tensor, count: torch.Tensor, stats: torch.Tensor | None = None,
+                        stream=None) -> None:
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_threshold_route(handle, _ptr(K), _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(tau),
+                                     max_tokens, _ptr(tokens), _ptr(count), _ptr(stats), _stream(stream)),
+           "zha_threshold_route")
+
+
 def zha_noalloc_scratch_capacity() -> int:
     return int(lib().zha_noalloc_scratch_capacity())
 
@@ -314,6 +337,10 @@ class Tree:
         units = self.desc.batch * self.desc.kv_heads
         d = self.desc.head_dim
         return self.workspace[256:256 + units * rows * d * 4].view(torch.float32).view(units, rows, d)
+
+    def level_offset(self, level: int) -> int:
+        """Row offset of a level inside each unit's summaries (and radii)."""
+        return zha_tree_level_offset(self.handle, level)
 
     def level(self, level: int) -> torch.Tensor:
         """[units, n_level, head_dim] view of one level's summaries."""
@@ -403,6 +430,23 @@ class Tree:
         O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
         zha_decode_causal(self.handle, Q, positions, beam, K, V, scale, idx, O, None, None, stream)
         return O, idx
+
+    def attach_radii(self, K: torch.Tensor | None, stream=None) -> torch.Tensor:
+        """Allocate and attach the bounding-sphere radii; returns them ([units, unit_rows])."""
+        n = zha_tree_radii_bytes(self.handle) // 4
+        self._radii = torch.zeros(n, dtype=torch.float32, device=self.workspace.device)
+        zha_tree_attach_radii(self.handle, self._radii, K, stream)
+        return self._radii.view(-1, zha_tree_unit_rows(self.handle))
+
+    def threshold(self, K: torch.Tensor, Q: torch.Tensor, tau: torch.Tensor, max_tokens: int,
+                  stats: bool = False, stream=None):
+        """Threshold descent; returns (tokens, count, stats or None)."""
+        B, Hq, nq, _ = Q.shape
+        toks = torch.empty((B, Hq, nq, max_tokens), dtype=torch.int32, device=Q.device)
+        cnt = torch.empty((B, Hq, nq), dtype=torch.int32, device=Q.device)
+        st = torch.empty((B, Hq, nq, 2), dtype=torch.int32, device=Q.device) if stats else None
+        zha_threshold_route(self.handle, K, Q, tau, max_tokens, toks, cnt, st, stream)
+        return toks, cnt, st
 
     def check(self, stream=None) -> int:
         return zha_tree_check(self.handle, stream)
