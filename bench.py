@@ -560,6 +560,52 @@ def run_causal(W, K, dev, flush):
     return out
 
 
+def run_threshold(W, K, dev, flush):
+    """Threshold (halfspace) descent, zha_threshold_route, on two 32K caches of the gqa_32k
+    geometry (8 x 8 KV heads, 32 query heads, b 8, 64-token leaves): its own keys (N(0, 1)
+    with planted needles) and clustered keys (each leaf block a random center plus 0.1 N(0, 1)
+    noise).  Per query tau lies halfway between its 16th and 17th largest key scores (dense
+    pass, untimed); every token at or above it is returned."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+
+    base = workloads.get("gqa_32k")
+    out = {}
+    for name in ("gqa_32k", "clustered_32k"):
+        w = base if name == "gqa_32k" else base.with_(needles=0)
+        Qn = synth.queries(w)
+        Kn = synth.keys(w, Q=Qn) if name == "gqa_32k" else synth.clustered_keys(w, 0.1)
+        Kd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Qn, dev)
+        del Kn
+        tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len, torch.bfloat16)
+        tree.build(Kd, w.seq_len)
+        tree.attach_radii(Kd)
+        kv = Kd.float().repeat_interleave(w.group, dim=1)  # [B, Hq, N, d]
+        top = torch.topk(torch.einsum("bhqd,bhnd->bhqn", Qd.float(), kv), 17, dim=-1).values
+        tau = ((top[..., 15] + top[..., 16]) / 2).contiguous()
+        del kv, top
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ms = []
+        for it in range(W + K):
+            flush.zero_()
+            e0.record()
+            toks, cnt, st = tree.threshold(Kd, Qd, tau, 64, stats=True)
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= W:
+                ms.append(e0.elapsed_time(e1))
+        assert tree.check() == zha.ZHA_OK
+        cnt, st = cnt.cpu().numpy(), st.cpu().numpy()
+        q = w.batch * w.q_heads * w.nq
+        nodes = sum(tree.level_nodes(lvl) for lvl in range(tree.levels))
+        out[name] = {"queries": q, "ms": float(np.mean(ms)), "qps": q / (np.mean(ms) * 1e-3),
+                     "found_per_query": float(cnt[cnt >= 0].mean()), "overflowed": int((cnt < 0).sum()),
+                     "spheres_tested_per_query": float(st[..., 0].mean()), "scored_nodes_per_tree": int(nodes),
+                     "tokens_checked_per_query": float(st[..., 1].mean()), "dense_keys_per_query": w.seq_len}
+        tree.close()
+    return out
+
+
 def run_profile_case(case: str, W: int, K: int):
     """A small case of a bench workload for ncu captures (eager launches, no graphs):
     deep_1m_2kv = the 1M-token tree with 2 KV heads and 16 query heads (group 8, 64 queries
@@ -841,6 +887,7 @@ def main():
     if not args.no_build and rank == 0:
         line["build_256k"] = run_build_256k(W, K, dev, flush)
         line["causal"] = run_causal(W, min(K, 10), dev, flush)
+        line["threshold"] = run_threshold(W, min(K, 10), dev, flush)
 
     if rank == 0 and world == 1:
         try:

@@ -154,3 +154,31 @@ def test_radii_follow_appends_and_decode_steps(dev):
     torch.cuda.synchronize()
     assert torch.equal(kept, tree._radii)
     _check_radii(w, tree, Kn, 1027)
+
+
+def test_threshold_prunes_clustered_keys_exactly(dev):
+    # keys clustered in leaf blocks: most spheres miss the halfspace, and the found set is
+    # still exactly the scan of all keys
+    from tree_indexed_sparse_build_b200 import zha
+    w = _wl("th_clustered", 1, 2, 8, 128, 8192, "bf16", 8, 64, 8, 4, 307)
+    Qn = synth.queries(w)
+    Kn = synth.clustered_keys(w, 0.1)
+    Q, K = torch_of(Qn, dev), torch_of(Kn, dev)
+    tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len, torch.bfloat16)
+    tree.build(K, w.seq_len)
+    tree.attach_radii(K)
+    tau = np.empty((1, w.q_heads, 4), np.float32)
+    for hq in range(w.q_heads):
+        s = np.sort(synth.to_f64(Kn[0, hq // w.group]) @ synth.to_f64(Qn[0, hq]).T, axis=0)
+        tau[0, hq] = ((s[-64] + s[-65]) / 2).astype(np.float32)
+    toks, cnt, st = tree.threshold(K, Q, torch.from_numpy(tau).to(dev), 128, stats=True)
+    torch.cuda.synchronize()
+    assert tree.check() == zha.ZHA_OK
+    toks, cnt, st = toks.cpu().numpy(), cnt.cpu().numpy(), st.cpu().numpy()
+    for hq in range(w.q_heads):
+        for i in range(4):
+            ref = oracle.threshold_brute(synth.to_f64(Qn[0, hq, i]), Kn[0, hq // w.group], w.seq_len,
+                                         float(tau[0, hq, i]))
+            assert cnt[0, hq, i] == len(ref) == 64
+            np.testing.assert_array_equal(toks[0, hq, i, :64], ref)
+    assert st[..., 1].mean() < 0.25 * w.seq_len  # most leaves pruned

@@ -98,3 +98,16 @@ def test_drift_keys_match_formula():
     t = np.arange(300.0)[:, None]
     x = x + 0.5 * (np.sin(2 * np.pi * t / P[None] + phi[None]) @ A.reshape(128, 8).T)
     np.testing.assert_array_equal(K[0, 0], synth.round_to(x, "bf16"))
+
+
+def test_clustered_keys_are_seeded_blocks_around_centers():
+    from tree_indexed_sparse_build_b200.workloads import Workload
+    w = Workload(name="c", batch=1, kv_heads=2, q_heads=2, head_dim=16, seq_len=100, kv_dtype="f32",
+                 branching=2, leaf_block=8, beam=2)
+    a = synth.clustered_keys(w, 0.1)
+    assert np.array_equal(a, synth.clustered_keys(w, 0.1))
+    x = a[0, 1].astype(np.float64)
+    blocks = [x[i:i + 8] for i in range(0, 100, 8)]
+    within = max(np.linalg.norm(blk - blk.mean(0), axis=1).max() for blk in blocks)
+    between = np.linalg.norm(blocks[0].mean(0) - blocks[1].mean(0))
+    assert within < 1.0 < between

@@ -41,6 +41,7 @@ _lib = None
 
 STREAM_K, STREAM_V, STREAM_Q, STREAM_NPOS, STREAM_NNOISE = 1, 2, 3, 4, 5
 STREAM_DRIFT_A, STREAM_DRIFT_PHI, STREAM_STEP_Q = 6, 7, 8
+STREAM_CLUSTER = 9  # cluster centers of clustered_keys
 
 _U64, _I64, _P, _D = ctypes.c_uint64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_double
 
@@ -214,6 +215,23 @@ def keys(w: Workload, capacity: int | None = None, Q: np.ndarray | None = None,
                 z = normal(w.seed, STREAM_NNOISE, (u << 20) + i * d, d, "f64")
                 flat[u, p * d:(p + 1) * d] = round_to(w.needle_amp * qhat + w.needle_sigma * z,
                                                       w.kv_dtype)
+    return out
+
+
+def clustered_keys(w: Workload, spread: float, capacity: int | None = None) -> np.ndarray:
+    """K cache [B, H_kv, capacity, d] whose tokens cluster in blocks of w.leaf_block
+    consecutive tokens: K[t] = C[t // leaf_block] + spread * e_t, C and e ~ N(0, I) (streams
+    STREAM_CLUSTER and STREAM_K), rounded once to the storage type."""
+    cap = w.capacity if capacity is None else capacity
+    d, lb = w.head_dim, w.leaf_block
+    dt = np.uint16 if w.kv_dtype == "bf16" else np.float32
+    out = np.zeros((w.batch, w.kv_heads, cap, d), dt)
+    flat = out.reshape(w.units, cap, d)
+    nblk = -(-cap // lb)
+    for u in range(w.units):
+        C = normal(w.seed, STREAM_CLUSTER, u << 40, nblk * d).reshape(nblk, d)
+        e = normal(w.seed, STREAM_K, u << 40, cap * d).reshape(cap, d)
+        flat[u] = round_to(np.repeat(C, lb, axis=0)[:cap] + spread * e, w.kv_dtype)
     return out
 
 
