@@ -58,6 +58,16 @@ struct NoKV {};  // route only: no attention epilogue
 // What the route kernel does besides routing the stored tree (decode_append.cuh).
 enum : int { kPathNone = 0, kPathAppend = 1, kPathPrefix = 2 };
 
+struct RouteArgs;
+// Launch route_tma_kernel for one KV type (route_tma_*.cu): route only (nokv), or route and
+// attention / path with bf16 or fp32 K rows.  narrow / grouped pick the launch shape.
+cudaError_t route_tma_launch_nokv(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                                  int threads, size_t smem, cudaStream_t s, int path);
+cudaError_t route_tma_launch_bf16(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                                  int threads, size_t smem, cudaStream_t s, int path);
+cudaError_t route_tma_launch_f32(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                                 int threads, size_t smem, cudaStream_t s, int path);
+
 
 constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 

@@ -1,0 +1,378 @@
+// The staged route kernel (route_tma_kernel) and its launch helpers.  Its instantiations
+// are spread over route_tma_nokv.cu, route_tma_bf16.cu and route_tma_f32.cu (one per KV
+// type), which compile in parallel; route.cu plans the launches and calls them through
+// route_tma_launch_* (route_common.cuh).
+#pragma once
+
+#include <algorithm>
+#include <type_traits>
+
+#include "attn_core.cuh"
+#include "decode_append.cuh"
+#include "decode_attn.cuh"
+#include "device_common.cuh"
+#include "route_common.cuh"
+#include "zha_internal.h"
+
+namespace zha {
+
+// Staged routing.  qpc queries per CTA, wpq warps per query (blockDim.x = 32 qpc wpq).
+// GROUPED (wpq > 1): the warps of query qi synchronise on named barrier 1 + qi; otherwise
+// each query is one warp, synchronised only within the warp.
+//
+// With TKV = the KV storage type (not NoKV) the kernel is the fused decode: once the
+// last level is selected, the query's warps attend over the tokens of its leaves.  The
+// candidate-row region, free after the leaf-level scoring, becomes two K/V stage buffers
+// filled by one bulk copy per leaf piece (K and V) on the two mbarriers; the warps run
+// the online softmax of attn_core.cuh over each stage, merge their states through shared
+// memory and write O.  No leaf list goes through global memory and nothing is launched
+// between the route and the attention.
+// NARROW instantiations are built for CTAs of at most 8 warps, three per SM (register cap).
+// PATH (decode_append.cuh; needs TKV, the type of the K rows the path reads):
+//  kPathAppend (fused decode, one query per CTA) -- the kernel first extends the tree by
+//    the tokens appended to one leaf, and stores the path (one CTA per unit);
+//  kPathPrefix (causal routing) -- query qg routes over the tree of tokens 0 .. p, p =
+//    positions[qg % nq]: its own depth and node counts, and its prefix's right edge
+//    recomputed into shared memory (never stored).
+// With a KV type, the query then attends over its leaves unless O is null.
+template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH = kPathNone>
+__global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3 : 1)
+    route_tma_kernel(const RouteArgs a) {
+  constexpr bool ATTEND = !std::is_same<TKV, NoKV>::value;
+  constexpr bool APPEND = PATH == kPathAppend;
+  constexpr bool PREFIX = PATH == kPathPrefix;
+  constexpr bool HASPATH = PATH != kPathNone;
+  static_assert(!HASPATH || ATTEND, "the path reads K rows of type TKV");
+  constexpr int CPL = D / 16;  // 16-byte chunks of a row per lane (4 lanes per row)
+  constexpr int R = 8;         // candidate keys held per lane in the selecting warp
+  extern __shared__ __align__(128) unsigned char rsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = GROUPED ? a.wpq : 1;  // warps of this query
+  const int qi = warp / nw;
+  const int wq = warp - qi * nw;
+  const int bar_id = 1 + qi, bar_n = 32 * nw;
+  const long long qg = (long long)blockIdx.x * a.qpc + qi;
+  const bool valid = qg < a.total_queries;
+  const RouteSmem Ls =
+      route_smem_layout(D, a.cmax, a.beam, (size_t)a.rows_bytes, ATTEND ? nw : 0);
+  unsigned char* base = rsm + (size_t)qi * a.query_smem_bytes;
+  const float* rows = reinterpret_cast<const float*>(base + Ls.rows);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + Ls.keys);
+  int* cand = reinterpret_cast<int*>(base + Ls.cand);
+  int* surv_a = reinterpret_cast<int*>(base + Ls.surv_a);
+  int* surv_b = reinterpret_cast<int*>(base + Ls.surv_b);
+  float* leaf_sc = reinterpret_cast<float*>(base + Ls.leaf_sc);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + Ls.bar);
+  unsigned* red = reinterpret_cast<unsigned*>(base + Ls.red);
+
+  auto qsync = [&]() {  // all warps of this query
+    if (GROUPED) group_sync(bar_id, bar_n); else __syncwarp();
+  };
+  pdl_wait();
+  pdl_release();
+
+  long long unit = 0;
+  if (valid) {
+    const long long hq_flat = qg / a.nq;
+    const int h = (int)(hq_flat % a.q_heads);
+    unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
+  }
+  const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
+  // the path region (fused append or causal prefix)
+  unsigned char* pb = base + a.path_smem_off;
+  PathSmem Ps{};
+  if (HASPATH) Ps = path_smem_layout(D, D * (int)sizeof(TKV), (int)a.lb, a.b, a.L);
+  uint64_t* pbar = reinterpret_cast<uint64_t*>(pb + Ps.bar);
+  // this query's tree: the whole tree, or (PREFIX) the tree of its prefix
+  long long Nq = a.N;
+  bool live = valid;  // a query with a position outside the tree routes nowhere
+  if constexpr (PREFIX) {
+    const long long pos = valid ? a.positions[qg % a.nq] : 0;
+    if (valid && (pos < 0 || pos >= a.N)) {
+      if (wq == 0 && lane == 0) atomicOr(a.err, kDevErrBadLeaf);
+      live = false;
+    }
+    Nq = live ? pos + 1 : 1;
+    if (wq == 0 && lane == 0) {
+      long long* qn = reinterpret_cast<long long*>(pb + Ps.qn);
+      qn[0] = (Nq + a.lb - 1) / a.lb;
+      int L = 0;
+      do {  // L = smallest L >= 1 with b^L >= n0
+        qn[L + 1] = (qn[L] + a.b - 1) / a.b;
+        ++L;
+      } while (qn[L] > 1);
+      qn[kMaxLevels - 1] = L;
+    }
+    qsync();
+  }
+  const long long* nl = PREFIX ? reinterpret_cast<const long long*>(pb + Ps.qn) : a.n;
+  const int Lq = PREFIX ? (int)nl[kMaxLevels - 1] : a.L;
+  if (wq == 0 && lane == 0) {
+    mbar_init(&bar[0], 1);
+    if (ATTEND)
+      for (int i = 0; i < a.attn_nbuf; ++i) {
+        if (i > 0) mbar_init(&bar[i], 1);  // "full" (bar[0] serves the route first)
+        mbar_init(&bar[3 + i], nw);        // "empty": one arrival per warp
+      }
+    if (HASPATH) mbar_init(pbar, 1);
+    fence_mbar_init();
+    surv_a[0] = 0;  // the root
+    if constexpr (HASPATH) {
+      if (live) {
+        fence_proxy_async_smem();
+        const long long leaf = APPEND ? a.path_leaf : (Nq - 1) / a.lb;
+        const int ntok = APPEND ? a.path_tokens : (int)(Nq - leaf * a.lb);
+        path_issue<TKV, D>(Ps, pb, a.K + unit * a.kv_unit_stride, pyr_u, a.off, nl, a.b, Lq, leaf,
+                           ntok, a.lb, pbar);
+      }
+    }
+  }
+  qsync();
+
+  // Four lanes per row: lane (rg = lane / 4, sub = lane % 4) reads chunks 4 (j ^ par) + sub,
+  // par = rg & 1, so the two rows of a shared-memory phase use opposite bank halves.
+  const int sub = lane & 3, rg = lane >> 2, par = rg & 1;
+  float4 qv[CPL];
+  int* cur = surv_a;
+  int* nxt = surv_b;
+  int m = live ? 1 : 0;
+  uint32_t parity = 0;
+  for (int l = Lq - 1; l >= 0; --l) {
+    int C = 0;
+    if (m > 0) {
+      const long long last = cur[m - 1];
+      C = (m - 1) * a.b + (int)min((long long)a.b, nl[l] - (long long)a.b * last);
+    }
+    const float* S = pyr_u + a.off[l] * D;
+    if (wq == 0 && C > 0) {
+      // one bulk copy per survivor (its children are consecutive rows) + candidate ids
+      if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)C * D * 4);
+      __syncwarp();
+      fence_proxy_async_smem();
+      for (int j = lane; j < m; j += 32) {
+        const long long node0 = (long long)a.b * cur[j];
+        const int nc = (int)min((long long)a.b, nl[l] - node0);
+        bulk_copy_g2s((void*)(rows + (size_t)j * a.b * D), S + node0 * D, (uint32_t)nc * D * 4, bar);
+      }
+      for (int j = lane; j < m; j += 32) {  // survivor j's children are candidates j b ..
+        const int node0 = a.b * cur[j];
+        const int nc = min(a.b, C - j * a.b);
+        for (int i = 0; i < nc; ++i) cand[j * a.b + i] = node0 + i;
+      }
+    }
+    if (HASPATH && wq == 0) {
+      // candidate slot of the path node at this level: its parent is a survivor j, and the
+      // parent's children are candidates j b .. j b + b - 1
+      const long long* node = reinterpret_cast<const long long*>(pb + Ps.node);
+      int* kpos = reinterpret_cast<int*>(pb + Ps.kpos);
+      int found = -1;
+      for (int j0 = 0; j0 < m; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned hit = __ballot_sync(0xffffffffu, j < m && live && cur[j] == node[l + 1]);
+        if (hit && found < 0) found = j0 + __ffs(hit) - 1;
+      }
+      if (lane == 0) kpos[0] = found < 0 ? -1 : (int)(found * a.b + (node[l] - a.b * node[l + 1]));
+    }
+    if (l == Lq - 1 && valid) {  // load q while the first level is in flight
+      const long long qo = qg * D;
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int c = 4 * (j ^ par) + sub;
+        float f[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          f[e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[qo + 4 * c + e])
+                          : static_cast<const float*>(a.Q)[qo + 4 * c + e];
+        qv[j] = make_float4(f[0], f[1], f[2], f[3]);
+      }
+    }
+    if (HASPATH && l == Lq - 1) {
+      // the path rows, while the first level's copies are in flight
+      const bool pok = !live || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+      const bool pfail = GROUPED ? group_any(bar_id, bar_n, !pok) : __any_sync(0xffffffffu, !pok);
+      if (pfail) {
+        if (wq == 0 && lane == 0) {  // let all copies land before the CTA exits
+          if (live) mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+          if (C > 0) mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+        }
+        return;
+      }
+      if constexpr (HASPATH) {
+        if (live) {
+          // fused append: the first query of each unit stores the path
+          const bool writer = APPEND && (qg % a.nq) == 0 && ((qg / a.nq) % a.q_heads) % a.group == 0;
+          const int ntok = APPEND ? a.path_tokens : (int)(Nq - ((Nq - 1) / a.lb) * a.lb);
+          path_compute<TKV, D>(Ps, pb, const_cast<float*>(pyr_u), a.off, nl, a.b, Lq, ntok, writer,
+                               32 * wq + lane, bar_n, qsync);
+        }
+      }
+    }
+    const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+    const bool failed = GROUPED ? group_any(bar_id, bar_n, !ok) : __any_sync(0xffffffffu, !ok);
+    if (failed) {
+      if (wq == 0 && lane == 0 && C > 0)  // let the copies land before the CTA exits
+        mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+      return;  // the whole group leaves together
+    }
+    if (!GROUPED) __syncwarp();  // candidate ids written by other lanes
+    if (C > 0) parity ^= 1u;
+    if (HASPATH) {
+      // the staged row of the path node may predate the append, or (prefix) cover tokens
+      // past the query's prefix: use the recomputed one
+      const int k = *reinterpret_cast<const int*>(pb + Ps.kpos);
+      if (k >= 0) {
+        const float* pf = reinterpret_cast<const float*>(pb + Ps.pf) + (size_t)l * D;
+        float* dst = const_cast<float*>(rows) + (size_t)k * D;
+        for (int e = 32 * wq + lane; e < D; e += bar_n) dst[e] = pf[e];
+        qsync();
+      }
+    }
+
+    // score: rows r = 8 (wq + nw t) + rg, two rows per lane in flight
+    for (int r0 = 8 * wq; r0 < C; r0 += 16 * nw) {
+      // four running sums per row (dims 4c + e for e = 0..3), updated pairwise by packed FMAs
+      float2 acc[2][2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int r = r0 + 8 * nw * u + rg;
+        acc[u][0] = make_float2(0.f, 0.f);
+        acc[u][1] = make_float2(0.f, 0.f);
+        if (r < C) {
+          const float4* row = reinterpret_cast<const float4*>(rows + (size_t)r * D);
+#pragma unroll
+          for (int j = 0; j < CPL; ++j) {
+            const float4 v = row[4 * (j ^ par) + sub];
+            acc[u][0] = __ffma2_rn(make_float2(qv[j].x, qv[j].y), make_float2(v.x, v.y), acc[u][0]);
+            acc[u][1] = __ffma2_rn(make_float2(qv[j].z, qv[j].w), make_float2(v.z, v.w), acc[u][1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float s = (acc[u][0].x + acc[u][0].y) + (acc[u][1].x + acc[u][1].y);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        const int r = r0 + 8 * nw * u + rg;
+        if (sub == 0 && r < C) keys[r] = route_key(s, cand[r]);
+      }
+    }
+    qsync();
+    if (C > 0 && C <= 128 && C <= 64 * nw) {  // C is the same for the whole group
+      const int kept =
+          select_rank_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red, wq, lane, nw, bar_id);
+      qsync();
+      if (wq == 0 && a.trace && valid) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
+      }
+    } else if (GROUPED && C <= 32 * nw) {  // radix selection over the group
+      const int kept = select_radix_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red,
+                                          reinterpret_cast<unsigned*>(base + Ls.hist), wq, lane, nw, bar_id);
+      group_sync(bar_id, bar_n);
+      if (wq == 0 && a.trace && valid) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
+      }
+    } else if (wq == 0 && C > 0) {
+      const int kept = C <= 64    ? select_compact<2>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
+                       : C <= 128 ? select_compact<4>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
+                                  : select_compact<R>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0);
+      __syncwarp();
+      if (a.trace && valid) {
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
+      }
+    }
+    m = min(C, a.beam);
+    qsync();
+    int* tmp = cur;
+    cur = nxt;
+    nxt = tmp;
+  }
+  if (PREFIX && valid && wq == 0 && a.trace)  // levels above this query's tree
+    for (int l = Lq; l < a.L; ++l) {
+      int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+      for (int k = lane; k < a.beam; k += 32) tr[k] = -1;
+    }
+  if (valid && wq == 0 && a.leaf_idx) {
+    int* out = a.leaf_idx + qg * a.beam;
+    for (int k = lane; k < a.beam; k += 32) out[k] = k < m ? cur[k] : -1;
+  }
+  if (valid && wq == 0 && a.leaf_score) {
+    float* os = a.leaf_score + qg * a.beam;
+    for (int k = lane; k < a.beam; k += 32) os[k] = k < m ? leaf_sc[k] : __int_as_float(0x7fc00000);
+  }
+  if constexpr (ATTEND) {
+    if (a.O == nullptr) return;  // route only (the path needed the K type)
+    using S = AttnShape<TKV, D>;
+    StagedAttn sa;
+    sa.leaves = cur;
+    sa.lb = (int)a.lb;
+    sa.total = leaf_tokens(cur, m, a.lb, Nq);
+    sa.TS = a.stage_tokens;
+    sa.nbuf = a.attn_nbuf;
+    sa.sb = base + Ls.rows;  // the candidate rows (and the append path) are no longer needed
+    sa.bars = bar;
+    sa.empty = bar + 3;
+    sa.ph0 = parity;  // bar[0] carries on from the route's level copies
+    sa.Ku = a.K + unit * a.kv_unit_stride;
+    sa.Vu = a.V + unit * a.kv_unit_stride;
+    sa.qk_scale = a.qk_scale;
+    sa.O = a.O;
+    sa.o_bf16 = a.o_bf16;
+    sa.err = a.err;
+    sa.wait_cycles = kRouteWaitCycles;
+    const int nst = (sa.total + sa.TS - 1) / sa.TS;
+    if (wq == 0)
+      for (int st = 0; st < min(nst, sa.nbuf); ++st)
+        attn_issue_stage<S::ROWB>(cur, sa.lb, sa.total, sa.TS, st, sa.nbuf, sa.sb, sa.Ku, sa.Vu, bar, lane);
+    float qa[S::CPL][S::VEC];
+    if (valid) attn_load_q<TKV, D>(a.Q, a.q_bf16 != 0, qg, lane, qa);
+    float* pw = reinterpret_cast<float*>(base + Ls.pw) + wq * 16;
+    attend_staged<TKV, D>(sa, qg, valid, qa, pw, reinterpret_cast<float*>(red), wq, nw, lane, bar_id);
+  }
+}
+
+template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH = kPathNone>
+cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
+                          cudaStream_t s) {
+  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW, PATH>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <typename TKV, int PATH>
+cudaError_t run_shape(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks, int threads,
+                      size_t smem, cudaStream_t s) {
+  if constexpr (PATH != kPathAppend) {  // the fused append runs in wide launches only
+    if (narrow) {
+      if (grouped)
+        return D == 128 ? run_route_tma<128, true, TKV, true, PATH>(a, blocks, threads, smem, s)
+                        : run_route_tma<64, true, TKV, true, PATH>(a, blocks, threads, smem, s);
+      return D == 128 ? run_route_tma<128, false, TKV, true, PATH>(a, blocks, threads, smem, s)
+                      : run_route_tma<64, false, TKV, true, PATH>(a, blocks, threads, smem, s);
+    }
+  } else if (narrow) {
+    return cudaErrorNotSupported;
+  }
+  if (grouped)
+    return D == 128 ? run_route_tma<128, true, TKV, false, PATH>(a, blocks, threads, smem, s)
+                    : run_route_tma<64, true, TKV, false, PATH>(a, blocks, threads, smem, s);
+  return D == 128 ? run_route_tma<128, false, TKV, false, PATH>(a, blocks, threads, smem, s)
+                  : run_route_tma<64, false, TKV, false, PATH>(a, blocks, threads, smem, s);
+}
+
+template <typename TKV>
+cudaError_t run_route_tma_d_impl(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                            int threads, size_t smem, cudaStream_t s, int path = kPathNone) {
+  if constexpr (!std::is_same<TKV, NoKV>::value) {
+    if (path == kPathAppend) return run_shape<TKV, kPathAppend>(D, grouped, narrow, a, blocks, threads, smem, s);
+    if (path == kPathPrefix) return run_shape<TKV, kPathPrefix>(D, grouped, narrow, a, blocks, threads, smem, s);
+  }
+  return run_shape<TKV, kPathNone>(D, grouped, narrow, a, blocks, threads, smem, s);
+}
+
+}  // namespace zha
