@@ -75,6 +75,8 @@ def _load():
         lib.orc_parent_radii.argtypes = [_P, _P, _I64, _P, _I64, _I64, _I64, _P]
         lib.orc_threshold_brute.restype = _I64
         lib.orc_threshold_brute.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, ctypes.c_double, _P, _I64]
+        lib.orc_round_bf16.restype = None
+        lib.orc_round_bf16.argtypes = [_P, _I64]
         lib.orc_threshold_descent.restype = _I64
         lib.orc_threshold_descent.argtypes = [_P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P,
                                               ctypes.c_int, _P, ctypes.c_double, _P, _I64, _P]
@@ -104,19 +106,38 @@ def num_levels(n0: int, b: int) -> int:
     return int(_load().orc_num_levels(n0, b))
 
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """The stored value of each element under bf16 summary storage: nearest fp32 (ties to
+    even), then nearest bf16 (ties to even), as fp64 (orc_round_bf16)."""
+    out = np.array(x, dtype=np.float64, copy=True, order="C")
+    if out.size:
+        _load().orc_round_bf16(_ptr(out), out.size)
+    return out
+
+
 class OracleTree:
     """Tree of mean key summaries over one (batch, KV-head) slice, in fp64.
 
     ``levels[l]`` is an ``[n_l, d]`` fp64 array; ``levels[0]`` are the leaves
     and ``levels[L]`` the single root.
+
+    ``summary="f64"`` keeps every summary exact (the reference for fp32-stored trees);
+    ``summary="bf16"`` mirrors bf16 storage: every node computed is replaced by its stored
+    value (``round_bf16``) before its parent averages it.
     """
 
-    def __init__(self, d: int, leaf_block: int, branching: int):
+    def __init__(self, d: int, leaf_block: int, branching: int, summary: str = "f64"):
         if leaf_block < 1 or branching < 2:
             raise ValueError("leaf_block >= 1 and branching >= 2 required")
+        if summary not in ("f64", "bf16"):
+            raise ValueError("summary must be 'f64' or 'bf16'")
         self.d, self.lb, self.b = d, leaf_block, branching
+        self.summary = summary
         self.N = 0
         self.levels: list[np.ndarray] = []
+
+    def _store(self, x):
+        return round_bf16(x) if self.summary == "bf16" else x
 
     @property
     def L(self) -> int:
@@ -127,14 +148,14 @@ class OracleTree:
         out = np.empty((max(i1 - i0, 0), self.d), np.float64)
         if i1 > i0:
             _load().orc_leaf_means(_ptr(K), dt, self.d, N, self.lb, i0, i1, _ptr(out))
-        return out
+        return self._store(out)
 
     def _parent_means(self, child, i0, i1):
         child = np.ascontiguousarray(child, dtype=np.float64)
         out = np.empty((max(i1 - i0, 0), self.d), np.float64)
         if i1 > i0:
             _load().orc_parent_means(_ptr(child), child.shape[0], self.d, self.b, i0, i1, _ptr(out))
-        return out
+        return self._store(out)
 
     def build(self, K: np.ndarray, N: int) -> "OracleTree":
         """Summaries of tokens [0, N) of K ([>=N, d])."""

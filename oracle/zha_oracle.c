@@ -25,6 +25,8 @@
  *     summaries (leaf radius: farthest token; node radius: farthest child sphere),
  *     a child kept iff q . c + ||q|| r >= tau, exact check of the surviving
  *     leaves' tokens; pinned against a scan of all keys.
+ *   - bf16-stored summaries (optional): each stored node is the bf16 rounding of
+ *     its fp32-rounded fp64 mean, and parents average the stored children.
  *
  * Every computation is a plain loop in fp64 over inputs converted exactly
  * (bf16 -> fp64 and fp32 -> fp64 are exact).  One library routine is used:
@@ -372,4 +374,30 @@ int64_t orc_threshold_descent(const double *pyr, const double *radii, const int6
   free(nxt);
   if (tested) *tested = ntest;
   return n;
+}
+
+/*
+ * Summaries stored in bf16 (an option of the tree, halving the bytes a route reads).  The
+ * pages fix no storage precision; the reading taken here: the stored value of a node is its
+ * fp64 mean rounded to the nearest fp32 (ties to even) and that fp32 value rounded to the
+ * nearest bf16 (ties to even) -- the bf16 rounding of what an fp32 tree would store -- and
+ * every parent averages the STORED values of its children.  This replaces each x[i] by the
+ * fp64 value of its stored bf16.  Rounding to bf16 by hand: keep the top 16 bits of the
+ * fp32 pattern after adding half a bf16 unit (0x7FFF) plus the lowest kept bit (ties to
+ * even); NaN stays NaN.
+ */
+void orc_round_bf16(double *x, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) {
+    float f = (float)x[i];
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) {
+      u |= 0x00400000u;
+    } else {
+      u += 0x7FFFu + ((u >> 16) & 1u);
+    }
+    u &= 0xFFFF0000u;
+    memcpy(&f, &u, 4);
+    x[i] = (double)f;
+  }
 }
