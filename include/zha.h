@@ -71,13 +71,19 @@ typedef struct {
   int leaf_block;            /* tokens per leaf >= 1                               */
   long long capacity_tokens; /* rows allocated per unit in K and V, >= 1          */
   zha_dtype kv_dtype;        /* storage type of K, V                               */
+  /* Storage type of the summaries.  ZHA_F32 (0, the default of a zeroed desc): each node
+   * holds its fp64 mean rounded to fp32.  ZHA_BF16: each node holds that fp32 value rounded
+   * to the nearest bf16 (ties to even), and a parent averages its children's stored bf16
+   * values; a route then reads half the bytes.  Scores are formed in fp32 either way. */
+  zha_dtype summary_dtype;
 } zha_tree_desc;
 
 typedef struct zha_tree zha_tree; /* opaque host handle */
 
 /* Device bytes the caller must provide to zha_tree_init: a 256-byte header
- * (device error word) followed by the fp32 summaries of every unit, laid out
- * unit-major, level-contiguous with capacity-sized levels.  0 on a bad desc. */
+ * (device error word) followed by the summaries of every unit (fp32 or bf16, the desc's
+ * summary_dtype), laid out unit-major, level-contiguous with capacity-sized levels.
+ * 0 on a bad desc. */
 size_t zha_tree_workspace_bytes(const zha_tree_desc* desc);
 
 /* Creates a host handle over caller-owned workspace (>= zha_tree_workspace_bytes,
@@ -247,7 +253,8 @@ int zha_tree_levels(const zha_tree* tree);                        /* L; 0 when e
 long long zha_tree_level_nodes(const zha_tree* tree, int level);  /* n_level now       */
 long long zha_tree_level_offset(const zha_tree* tree, int level); /* row offset in unit */
 long long zha_tree_unit_rows(const zha_tree* tree);               /* rows per unit      */
-const float* zha_tree_summaries(const zha_tree* tree); /* device: [units, unit_rows, head_dim] */
+/* device: [units, unit_rows, head_dim] of the desc's summary_dtype (fp32, or bf16 bits) */
+const void* zha_tree_summaries(const zha_tree* tree);
 /* Kernel launches issued through this handle since zha_tree_init (all calls). */
 long long zha_tree_launch_count(const zha_tree* tree);
 

@@ -20,9 +20,10 @@ def make_inputs(w: Workload, capacity: int | None = None, nq: int | None = None)
     return Q, K, V
 
 
-def oracle_tree(w: Workload, K: np.ndarray, unit: int, N: int) -> oracle.OracleTree:
+def oracle_tree(w: Workload, K: np.ndarray, unit: int, N: int, summary: str = "f64") -> oracle.OracleTree:
+    """The oracle's tree of one unit; summary "bf16" mirrors bf16-stored summaries."""
     b, h = divmod(unit, w.kv_heads)
-    return oracle.OracleTree(w.head_dim, w.leaf_block, w.branching).build(K[b, h], N)
+    return oracle.OracleTree(w.head_dim, w.leaf_block, w.branching, summary=summary).build(K[b, h], N)
 
 
 def summary_rel_err(got: np.ndarray, ref: np.ndarray) -> float:

@@ -54,11 +54,14 @@ def test_workspace_bytes_matches_capacity_layout():
     assert zha.zha_tree_workspace_bytes(
         _desc(batch=1, kv_heads=1, head_dim=64, branching=2, leaf_block=16,
               capacity_tokens=1024, kv_dtype=zha.ZHA_F32)) == 256 + 127 * 64 * 4
+    # bf16-stored summaries: two bytes an element
+    assert zha.zha_tree_workspace_bytes(_desc(summary_dtype=zha.ZHA_BF16)) == 256 + 8 * rows * 128 * 2
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(branching=1), dict(leaf_block=0),
                                  dict(capacity_tokens=0), dict(batch=0), dict(kv_heads=0),
-                                 dict(batch=300, kv_heads=300), dict(kv_dtype=7)])
+                                 dict(batch=300, kv_heads=300), dict(kv_dtype=7),
+                                 dict(summary_dtype=2)])
 def test_workspace_bytes_rejects_bad_desc(bad):
     assert zha.zha_tree_workspace_bytes(_desc(**bad)) == 0
 

@@ -40,17 +40,18 @@ def _positions(w, nq, seed):
     return pos
 
 
-def _setup(w, dev, nq):
+def _setup(w, dev, nq, summary_dtype=None):
     from tree_indexed_sparse_build_b200 import zha
     Qn, Kn, Vn = make_inputs(w, nq=nq)
     Q, K, V = torch_of(Qn, dev), torch_of(Kn, dev), torch_of(Vn, dev)
     tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len,
-                    torch.float32 if w.kv_dtype == "f32" else torch.bfloat16)
+                    torch.float32 if w.kv_dtype == "f32" else torch.bfloat16,
+                    summary_dtype=summary_dtype or torch.float32)
     tree.build(K, w.seq_len)
     return tree, (Qn, Kn, Vn), (Q, K, V)
 
 
-def _check(w, tree, Qn, Kn, Vn, pos, idx, tr, O=None):
+def _check(w, tree, Qn, Kn, Vn, pos, idx, tr, O=None, summary="f64"):
     idx, tr = idx.cpu().numpy(), tr.cpu().numpy()
     got_o = out_to_f64(O) if O is not None else None
     L = tree.levels
@@ -62,7 +63,7 @@ def _check(w, tree, Qn, Kn, Vn, pos, idx, tr, O=None):
             q64 = synth.to_f64(Qn[b, hq])
             for i, p in enumerate(pos):
                 n = int(p) + 1
-                ot = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching).build(Kn[b, h], n)
+                ot = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching, summary=summary).build(Kn[b, h], n)
                 res = ot.route(q64[i:i + 1], w.beam)
                 if oracle.well_conditioned(res["bounds"])[0]:
                     np.testing.assert_array_equal(idx[b, hq, i], res["leaves"][0])

@@ -65,12 +65,13 @@ def _tdt(w):
     return torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
 
 
-def _setup(w, dev, capacity=None, nq=None):
+def _setup(w, dev, capacity=None, nq=None, summary_dtype=None):
     from tree_indexed_sparse_build_b200 import zha
     cap = capacity or w.seq_len
     Qn, Kn, Vn = make_inputs(w, capacity=cap, nq=nq)
     Q, K, V = torch_of(Qn, dev), torch_of(Kn, dev), torch_of(Vn, dev)
-    tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, cap, _tdt(w))
+    tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, cap, _tdt(w),
+                    summary_dtype=summary_dtype or torch.float32)
     return tree, (Qn, Kn, Vn), (Q, K, V)
 
 
@@ -124,15 +125,16 @@ def test_append_grows_depth(dev):
     _check_levels(tree, w, Kn, 1064)
 
 
-def _route_compare(tree, w, Qn, Kn, idx, trace, N, units=None):
-    """Exact match on well-conditioned queries; returns (n_checked, n_ill, n_ill_mismatch)."""
+def _route_compare(tree, w, Qn, Kn, idx, trace, N, units=None, summary="f64"):
+    """Exact match on well-conditioned queries; returns (n_checked, n_ill, n_ill_mismatch).
+    summary: the oracle's summary storage ("bf16" for trees with bf16 summaries)."""
     idx = idx.cpu().numpy()
     trace = trace.cpu().numpy() if trace is not None else None
     g = w.group
     checked = ill = ill_bad = 0
     for u in (range(w.units) if units is None else units):
         b, h = divmod(u, w.kv_heads)
-        ot = oracle_tree(w, Kn, u, N)
+        ot = oracle_tree(w, Kn, u, N, summary=summary)
         flat = ot.flat()
         for hq in range(h * g, h * g + g):
             q64 = synth.to_f64(Qn[b, hq])

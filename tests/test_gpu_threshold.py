@@ -31,13 +31,14 @@ def dev():
     return torch.device("cuda:0")
 
 
-def _setup(w, dev, nq, capacity=None):
+def _setup(w, dev, nq, capacity=None, summary_dtype=None):
     from tree_indexed_sparse_build_b200 import zha
     cap = capacity or w.seq_len
     Qn, Kn, Vn = make_inputs(w, capacity=cap, nq=nq)
     Q, K, V = torch_of(Qn, dev), torch_of(Kn, dev), torch_of(Vn, dev)
     tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, cap,
-                    torch.float32 if w.kv_dtype == "f32" else torch.bfloat16)
+                    torch.float32 if w.kv_dtype == "f32" else torch.bfloat16,
+                    summary_dtype=summary_dtype or torch.float32)
     return tree, (Qn, Kn, Vn), (Q, K, V)
 
 
@@ -47,7 +48,7 @@ def _check_radii(w, tree, Kn, N, units=None):
         b, h = divmod(u, w.kv_heads)
         K64 = synth.to_f64(Kn[b, h, :N])
         for lvl in range(tree.levels + 1):
-            cent = tree.level(lvl)[u].cpu().numpy().astype(np.float64)
+            cent = tree.level(lvl)[u].float().cpu().numpy().astype(np.float64)
             off = tree.level_offset(lvl)
             rad = radii[u, off:off + cent.shape[0]]
             span = w.leaf_block * w.branching ** lvl

@@ -6,8 +6,9 @@
 // Every CTA that routes a query of the unit recomputes that path itself, with the same
 // arithmetic and summation order as the stand-alone append kernel (leaf = fp64 sum of its
 // tokens in order / count; a parent = fp64 sum of its existing children in index order /
-// count, the touched child taken from its fp64 value, the others from their stored fp32
-// rows), so the rows are bit-identical to what the append kernel writes.  One CTA per unit
+// count, the touched child taken from its kept fp64 value, the others from their stored
+// rows; SumT rounds and keeps as the append kernel does for fp32 and bf16 summaries), so the
+// rows are bit-identical to what the append kernel writes.  One CTA per unit
 // writes them back; every CTA patches them into its own staged candidate rows, so no CTA
 // waits for another.  The path's copies (the leaf's tokens, each level's children of the
 // path node) are in flight together with the route's first level.
@@ -18,23 +19,24 @@
 
 namespace zha {
 
-// Shared memory of the path, for head_dim D, token rows of row_bytes, leaf block lb,
-// branching b and (at most) L levels below the root.
+// Shared memory of the path, for head_dim D, token rows of row_bytes, summary elements of
+// sum_bytes, leaf block lb, branching b and (at most) L levels below the root.
 struct PathSmem {
   size_t tok, sib, pv, pf, node, kpos, qn, bar, total;
 };
 __host__ __device__ inline size_t path_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
-__host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int lb, int b, int L) {
+__host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int sum_bytes, int lb, int b,
+                                                     int L) {
   PathSmem s;
   size_t o = 0;
   s.tok = o;   // the leaf's tokens [lb][row_bytes]
   o = path_align(o + (size_t)lb * row_bytes, 16);
-  s.sib = o;   // for l = 1..L: the children of path node l, fp32 [b][D]
-  o += (size_t)L * b * D * 4;
+  s.sib = o;   // for l = 1..L: the children of path node l, stored rows [b][D]
+  o += (size_t)L * b * D * sum_bytes;
   s.pv = o;    // fp64 values of the path node at two consecutive levels [2][D]
   o += (size_t)2 * D * 8;
-  s.pf = o;    // the stored (fp32) path rows, levels 0..L [L + 1][D]
-  o += (size_t)(L + 1) * D * 4;
+  s.pf = o;    // the stored path rows, levels 0..L [L + 1][D]
+  o = path_align(o + (size_t)(L + 1) * D * sum_bytes, 8);
   s.node = o;  // path node index per level [L + 1]
   o += (size_t)(L + 1) * 8;
   s.kpos = o;  // candidate slot of the path node at the current route level
@@ -50,8 +52,8 @@ __host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int l
 // One thread: path nodes, then the bulk copies of the leaf's tokens and of every level's
 // children of the path node, all completing on pbar.  Ku: the unit's K rows; pyr_u: the
 // unit's summaries; off / n: level offsets and node counts after the append.
-template <typename TIn, int D>
-__device__ void path_issue(const PathSmem& P, unsigned char* pb, const char* Ku, const float* pyr_u,
+template <typename TIn, typename TS, int D>
+__device__ void path_issue(const PathSmem& P, unsigned char* pb, const char* Ku, const TS* pyr_u,
                            const long long* off, const long long* n, int b, int L, long long leaf,
                            int ntok, long long lb, uint64_t* pbar) {
   long long* node = reinterpret_cast<long long*>(pb + P.node);
@@ -60,27 +62,27 @@ __device__ void path_issue(const PathSmem& P, unsigned char* pb, const char* Ku,
   uint32_t bytes = (uint32_t)ntok * D * sizeof(TIn);
   for (int l = 1; l <= L; ++l) {
     const long long c0 = node[l] * b, c1 = min(c0 + (long long)b, n[l - 1]);
-    bytes += (uint32_t)(c1 - c0) * D * 4;
+    bytes += (uint32_t)(c1 - c0) * D * (uint32_t)sizeof(TS);
   }
   mbar_arrive_expect_tx(pbar, bytes);
   bulk_copy_g2s(pb + P.tok, Ku + leaf * lb * D * (long long)sizeof(TIn), (uint32_t)ntok * D * sizeof(TIn),
                 pbar);
   for (int l = 1; l <= L; ++l) {
     const long long c0 = node[l] * b, c1 = min(c0 + (long long)b, n[l - 1]);
-    bulk_copy_g2s(pb + P.sib + (size_t)(l - 1) * b * D * 4, pyr_u + (off[l - 1] + c0) * D,
-                  (uint32_t)(c1 - c0) * D * 4, pbar);
+    bulk_copy_g2s(pb + P.sib + (size_t)(l - 1) * b * D * sizeof(TS), pyr_u + (off[l - 1] + c0) * D,
+                  (uint32_t)(c1 - c0) * D * (uint32_t)sizeof(TS), pbar);
   }
 }
 
 // Threads tid < D of the group (nt threads in all): the path rows, after pbar completed.
 // sync() synchronises the group.  writer: also store the rows into the unit's summaries.
-template <typename TIn, int D, typename Sync>
-__device__ void path_compute(const PathSmem& P, unsigned char* pb, float* pyr_u, const long long* off,
+template <typename TIn, typename TS, int D, typename Sync>
+__device__ void path_compute(const PathSmem& P, unsigned char* pb, TS* pyr_u, const long long* off,
                              const long long* n, int b, int L, int ntok, bool writer, int tid, int nt,
                              Sync sync) {
   const TIn* tok = reinterpret_cast<const TIn*>(pb + P.tok);
   double* pv = reinterpret_cast<double*>(pb + P.pv);
-  float* pf = reinterpret_cast<float*>(pb + P.pf);
+  TS* pf = reinterpret_cast<TS*>(pb + P.pf);
   const long long* node = reinterpret_cast<const long long*>(pb + P.node);
   for (int e = tid; e < D; e += nt) {
     double s = 0.0;
@@ -91,24 +93,24 @@ __device__ void path_compute(const PathSmem& P, unsigned char* pb, float* pyr_u,
         s += (double)tok[(size_t)r * D + e];
     }
     const double v = s / (double)ntok;
-    pv[e] = v;
-    pf[e] = (float)v;
-    if (writer) pyr_u[(off[0] + node[0]) * D + e] = (float)v;
+    pv[e] = SumT<TS>::kept(v);
+    pf[e] = SumT<TS>::store(v);
+    if (writer) pyr_u[(off[0] + node[0]) * D + e] = pf[e];
   }
   sync();
   for (int l = 1; l <= L; ++l) {
     const double* cur = pv + (size_t)((l - 1) & 1) * D;
     double* nxt = pv + (size_t)(l & 1) * D;
-    const float* sib = reinterpret_cast<const float*>(pb + P.sib + (size_t)(l - 1) * b * D * 4);
+    const TS* sib = reinterpret_cast<const TS*>(pb + P.sib + (size_t)(l - 1) * b * D * sizeof(TS));
     const long long c0 = node[l] * b, c1 = min(c0 + (long long)b, n[l - 1]);
     for (int e = tid; e < D; e += nt) {
       double s = 0.0;
       for (long long c = c0; c < c1; ++c)
-        s += c == node[l - 1] ? cur[e] : (double)sib[(c - c0) * D + e];
+        s += c == node[l - 1] ? cur[e] : (double)SumT<TS>::load(sib[(c - c0) * D + e]);
       const double v = s / (double)(c1 - c0);
-      nxt[e] = v;
-      pf[(size_t)l * D + e] = (float)v;
-      if (writer) pyr_u[(off[l] + node[l]) * D + e] = (float)v;
+      nxt[e] = SumT<TS>::kept(v);
+      pf[(size_t)l * D + e] = SumT<TS>::store(v);
+      if (writer) pyr_u[(off[l] + node[l]) * D + e] = pf[(size_t)l * D + e];
     }
     sync();
   }

@@ -36,6 +36,23 @@ template <> struct Vec16<float> {
   }
 };
 
+// Summary storage (fp32, or bf16 bits in uint16_t).  store(): the stored element of a node
+// whose fp64 mean is v (nearest fp32; for bf16 that fp32 rounded once more to the nearest
+// bf16, ties to even).  kept(): the fp64 value the node's parent averages -- for bf16 the
+// stored value itself; fp32 trees keep the unrounded fp64 mean between the levels that one
+// kernel computes.  load(): a stored element as fp32.
+template <typename TS> struct SumT;
+template <> struct SumT<float> {
+  __device__ __forceinline__ static float store(double v) { return __double2float_rn(v); }
+  __device__ __forceinline__ static double kept(double v) { return v; }
+  __device__ __forceinline__ static float load(float x) { return x; }
+};
+template <> struct SumT<uint16_t> {
+  __device__ __forceinline__ static uint16_t store(double v) { return f32_to_bf16_bits(__double2float_rn(v)); }
+  __device__ __forceinline__ static double kept(double v) { return (double)bf16_bits_to_f32(store(v)); }
+  __device__ __forceinline__ static float load(uint16_t x) { return bf16_bits_to_f32(x); }
+};
+
 __device__ __forceinline__ uint4 ldg16(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }

@@ -1,7 +1,7 @@
 // Bounding-sphere radii of the tree's nodes ("Louver" explainer, index design: every cluster
 // of keys is enclosed in a bounding sphere, a center and a radius, so a query can prune the
 // clusters whose sphere misses its halfspace {p : q . p >= tau}).  The center of a node is
-// its stored (fp32) summary; the radius covers every key of its subtree:
+// its stored summary (fp32 or bf16); the radius covers every key of its subtree:
 //   leaf i:  r = max over its tokens t < N of ||k_t - c_i||
 //   node i:  r = max over its existing children j of (||c_j - c_i|| + r_j)
 // (a child's sphere lies inside the ball of radius ||c_j - c_i|| + r_j around c_i).
@@ -27,9 +27,9 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 
 __device__ __forceinline__ float radius_up(double r) { return __double2float_ru(r * (1.0 + 1e-12)); }
 
-template <typename TK, int D>
+template <typename TK, typename TS, int D>
 __global__ void __launch_bounds__(kRadThreads) radius_leaf_kernel(const char* K, long long k_unit_stride,
-                                                                  const float* pyr, long long pyr_unit_stride,
+                                                                  const void* pyr, long long pyr_unit_stride,
                                                                   float* radii, long long off0, long long lo,
                                                                   long long count, long long units,
                                                                   long long N, long long lb) {
@@ -40,11 +40,11 @@ __global__ void __launch_bounds__(kRadThreads) radius_leaf_kernel(const char* K,
   pdl_release();
   if (w >= units * count) return;
   const long long unit = w / count, i = lo + (w - unit * count);
-  const float* c = pyr + unit * pyr_unit_stride + (off0 + i) * D;
+  const TS* c = static_cast<const TS*>(pyr) + unit * pyr_unit_stride + (off0 + i) * D;
   const TK* Ku = reinterpret_cast<const TK*>(K + unit * k_unit_stride);
   double cv[DPL];
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) cv[e] = (double)c[lane * DPL + e];
+  for (int e = 0; e < DPL; ++e) cv[e] = (double)SumT<TS>::load(c[lane * DPL + e]);
   const long long t0 = i * lb, t1 = min(t0 + lb, N);
   double best = 0.0;
   for (long long t = t0; t < t1; ++t) {
@@ -65,8 +65,8 @@ __global__ void __launch_bounds__(kRadThreads) radius_leaf_kernel(const char* K,
   if (lane == 0) radii[unit * pyr_unit_stride / D + off0 + i] = radius_up(sqrt(best));
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRadThreads) radius_level_kernel(const float* pyr, long long pyr_unit_stride,
+template <typename TS, int D>
+__global__ void __launch_bounds__(kRadThreads) radius_level_kernel(const void* pyr, long long pyr_unit_stride,
                                                                    float* radii, long long off_l,
                                                                    long long off_c, long long lo,
                                                                    long long count, long long units,
@@ -78,18 +78,18 @@ __global__ void __launch_bounds__(kRadThreads) radius_level_kernel(const float* 
   pdl_release();
   if (w >= units * count) return;
   const long long unit = w / count, i = lo + (w - unit * count);
-  const float* pu = pyr + unit * pyr_unit_stride;
+  const TS* pu = static_cast<const TS*>(pyr) + unit * pyr_unit_stride;
   const float* ru = radii + unit * (pyr_unit_stride / D);
   double cv[DPL];
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) cv[e] = (double)pu[(off_l + i) * D + lane * DPL + e];
+  for (int e = 0; e < DPL; ++e) cv[e] = (double)SumT<TS>::load(pu[(off_l + i) * D + lane * DPL + e]);
   const long long j0 = i * b, j1 = min(j0 + (long long)b, n_child);
   double best = 0.0;
   for (long long j = j0; j < j1; ++j) {
     double s = 0.0;
 #pragma unroll
     for (int e = 0; e < DPL; ++e) {
-      const double x = (double)pu[(off_c + j) * D + lane * DPL + e] - cv[e];
+      const double x = (double)SumT<TS>::load(pu[(off_c + j) * D + lane * DPL + e]) - cv[e];
       s = fma(x, x, s);
     }
     s = warp_sum_d(s);
@@ -100,32 +100,15 @@ __global__ void __launch_bounds__(kRadThreads) radius_level_kernel(const float* 
 
 unsigned grid_for(long long warps) { return (unsigned)((warps * 32 + kRadThreads - 1) / kRadThreads); }
 
-}  // namespace
-
-cudaError_t launch_radii(zha_tree* t, const void* d_K, long long lo, long long hi, cudaStream_t s) {
-  if (!t->radii || t->N == 0 || hi < lo) return cudaSuccess;
-  const int D = t->desc.head_dim;
-  const bool bf = t->desc.kv_dtype == ZHA_BF16;
-  const char* K = static_cast<const char*>(d_K);
-  const long long k_stride = t->desc.capacity_tokens * D * (bf ? 2LL : 4LL);
+template <typename TK, typename TS, int D>
+cudaError_t radii_levels(zha_tree* t, const char* K, long long lo, long long hi, cudaStream_t s) {
+  const long long k_stride = t->desc.capacity_tokens * D * (long long)sizeof(TK);
   const long long stride = t->unit_rows * D;
   const long long units = t->units;
-  cudaError_t e;
   long long cnt = hi - lo + 1;
-  if (bf)
-    e = D == 128 ? launch_pdl(radius_leaf_kernel<uint16_t, 128>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0,
-                              s, K, k_stride, (const float*)t->pyr, stride, t->radii, t->off[0], lo, cnt, units,
-                              t->N, (long long)t->desc.leaf_block)
-                 : launch_pdl(radius_leaf_kernel<uint16_t, 64>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0,
-                              s, K, k_stride, (const float*)t->pyr, stride, t->radii, t->off[0], lo, cnt, units,
-                              t->N, (long long)t->desc.leaf_block);
-  else
-    e = D == 128 ? launch_pdl(radius_leaf_kernel<float, 128>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0, s,
-                              K, k_stride, (const float*)t->pyr, stride, t->radii, t->off[0], lo, cnt, units, t->N,
-                              (long long)t->desc.leaf_block)
-                 : launch_pdl(radius_leaf_kernel<float, 64>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0, s,
-                              K, k_stride, (const float*)t->pyr, stride, t->radii, t->off[0], lo, cnt, units, t->N,
-                              (long long)t->desc.leaf_block);
+  cudaError_t e = launch_pdl(radius_leaf_kernel<TK, TS, D>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0, s,
+                             K, k_stride, (const void*)t->pyr, stride, t->radii, t->off[0], lo, cnt, units, t->N,
+                             (long long)t->desc.leaf_block);
   ++t->launches;
   if (e != cudaSuccess) return e;
   const int b = t->desc.branching;
@@ -133,16 +116,29 @@ cudaError_t launch_radii(zha_tree* t, const void* d_K, long long lo, long long h
     lo /= b;
     hi /= b;
     cnt = hi - lo + 1;
-    e = D == 128 ? launch_pdl(radius_level_kernel<128>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0, s,
-                              (const float*)t->pyr, stride, t->radii, t->off[l], t->off[l - 1], lo, cnt, units,
-                              t->n[l - 1], b)
-                 : launch_pdl(radius_level_kernel<64>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0, s,
-                              (const float*)t->pyr, stride, t->radii, t->off[l], t->off[l - 1], lo, cnt, units,
-                              t->n[l - 1], b);
+    e = launch_pdl(radius_level_kernel<TS, D>, dim3(grid_for(units * cnt)), dim3(kRadThreads), 0, s,
+                   (const void*)t->pyr, stride, t->radii, t->off[l], t->off[l - 1], lo, cnt, units, t->n[l - 1], b);
     ++t->launches;
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
+}
+
+template <typename TK, typename TS>
+cudaError_t radii_d(zha_tree* t, const char* K, long long lo, long long hi, cudaStream_t s) {
+  return t->desc.head_dim == 128 ? radii_levels<TK, TS, 128>(t, K, lo, hi, s)
+                                 : radii_levels<TK, TS, 64>(t, K, lo, hi, s);
+}
+
+}  // namespace
+
+cudaError_t launch_radii(zha_tree* t, const void* d_K, long long lo, long long hi, cudaStream_t s) {
+  if (!t->radii || t->N == 0 || hi < lo) return cudaSuccess;
+  const char* K = static_cast<const char*>(d_K);
+  const bool bf = t->desc.kv_dtype == ZHA_BF16;
+  if (sum_bf16(t))
+    return bf ? radii_d<uint16_t, uint16_t>(t, K, lo, hi, s) : radii_d<float, uint16_t>(t, K, lo, hi, s);
+  return bf ? radii_d<uint16_t, float>(t, K, lo, hi, s) : radii_d<float, float>(t, K, lo, hi, s);
 }
 
 }  // namespace zha

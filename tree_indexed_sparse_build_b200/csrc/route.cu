@@ -29,8 +29,11 @@
 // Fallback kernel (route_reg_kernel) for levels too wide to stage in shared memory:
 // the same selection, with candidate rows loaded into registers in batches.
 //
+// Summaries are stored in fp32 or bf16 (the tree's summary type, TS in the kernels); rows
+// are read as stored and widened to fp32 for scoring.
+//
 // Files: route_tma_kernel and its launch helpers are in route_kernel.cuh, instantiated per
-// KV type in route_tma_nokv.cu / route_tma_bf16.cu / route_tma_f32.cu; this file holds the
+// KV type and summary type in route_tma_{nokv,bf16,f32}{,_s16}.cu; this file holds the
 // register kernel and the host-side plans (launch_route, plan_decode, launch_decode,
 // launch_causal).
 #include <algorithm>
@@ -45,9 +48,10 @@
 
 namespace zha {
 
-template <int D, int U>
+template <int D, int U, typename TS>
 __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const RouteArgs a) {
-  constexpr int NJ = D / 32;  // 16-byte chunks per lane per row
+  constexpr int EPC = 16 / (int)sizeof(TS);  // summary elements per 16-byte chunk
+  constexpr int NJ = D / (8 * EPC);          // 16-byte chunks per lane per row (8 lanes a row)
   extern __shared__ unsigned long long route_smem[];
   __shared__ int s_m[kRouteMaxWarps];  // survivors per query of the CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -63,21 +67,21 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
   float* leaf_sc = reinterpret_cast<float*>(surv_b + a.beam);
 
   long long unit = 0;
-  float q[NJ * 4];
+  float q[NJ * EPC];
   const int l8 = lane & 7, grp = lane >> 3;
   if (valid) {
     const long long hq_flat = qg / a.nq;  // b * q_heads + h
     const int h = (int)(hq_flat % a.q_heads);
     unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
-    // This lane's slice of q: chunks c = l8 + 8j, dims 4c .. 4c+3.
+    // This lane's slice of q: chunks c = l8 + 8j, dims EPC c .. EPC c + EPC - 1.
     const long long qo = qg * D;
 #pragma unroll
     for (int j = 0; j < NJ; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const long long dim = qo + (l8 + 8 * j) * 4 + e;
-        q[j * 4 + e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[dim])
-                                : static_cast<const float*>(a.Q)[dim];
+      for (int e = 0; e < EPC; ++e) {
+        const long long dim = qo + (l8 + 8 * j) * EPC + e;
+        q[j * EPC + e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[dim])
+                                  : static_cast<const float*>(a.Q)[dim];
       }
   }
   if (wq == 0 && lane == 0) {
@@ -86,7 +90,7 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
   }
   __syncthreads();
 
-  const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
+  const TS* pyr_u = static_cast<const TS*>(a.pyr) + unit * a.pyr_unit_stride;
   int* cur = surv_a;
   int* nxt = surv_b;
   for (int l = a.L - 1; l >= 0; --l) {
@@ -96,10 +100,10 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
       const long long last = cur[m - 1];
       C = (m - 1) * a.b + (int)min((long long)a.b, a.n[l] - (long long)a.b * last);
     }
-    const float* S = pyr_u + a.off[l] * D;
+    const TS* S = pyr_u + a.off[l] * D;
 #pragma unroll 1
     for (int k0 = wq * 4 * U; k0 < C; k0 += a.wpq * 4 * U) {
-      float4 v[U][NJ];
+      uint4 v[U][NJ];
       int node[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
         node[u] = -1;
         if (k < C) {
           node[u] = a.b * cur[k / a.b] + k % a.b;
-          const float4* row = reinterpret_cast<const float4*>(S + (long long)node[u] * D);
+          const uint4* row = reinterpret_cast<const uint4*>(S + (long long)node[u] * D);
 #pragma unroll
           for (int j = 0; j < NJ; ++j) v[u][j] = __ldg(row + l8 + 8 * j);
         }
@@ -118,10 +122,10 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
         if (node[u] >= 0) {
 #pragma unroll
           for (int j = 0; j < NJ; ++j) {
-            s = fmaf(q[4 * j + 0], v[u][j].x, s);
-            s = fmaf(q[4 * j + 1], v[u][j].y, s);
-            s = fmaf(q[4 * j + 2], v[u][j].z, s);
-            s = fmaf(q[4 * j + 3], v[u][j].w, s);
+            float f[EPC];
+            Vec16<TS>::to_f32(v[u][j], f);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) s = fmaf(q[EPC * j + e], f[e], s);
           }
         }
         s += __shfl_xor_sync(0xffffffffu, s, 1);
@@ -173,10 +177,10 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
 }
 
 namespace {
-template <int D, int U>
+template <int D, int U, typename TS>
 cudaError_t run_route(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
                       cudaStream_t s) {
-  auto kern = route_reg_kernel<D, U>;
+  auto kern = route_reg_kernel<D, U, TS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
@@ -186,6 +190,16 @@ cudaError_t run_route(const RouteArgs& a, unsigned blocks, int threads, size_t s
 
 constexpr size_t kRouteSmemCap = 200 * 1024;  // staged kernel: shared memory per query
 constexpr size_t kCtaSmemCap = 227 * 1024;    // dynamic shared memory of one CTA
+
+// The staged kernel's instantiation set for this tree: route only (kv false) or with the
+// cache's K/V type, over its summary type.
+using RouteLaunch = cudaError_t (*)(int, bool, bool, const RouteArgs&, unsigned, int, size_t, cudaStream_t, int);
+RouteLaunch staged_launch(const zha_tree* t, bool kv) {
+  const bool s16 = sum_bf16(t);
+  if (!kv) return s16 ? route_tma_launch_nokv_s16 : route_tma_launch_nokv;
+  if (t->desc.kv_dtype == ZHA_BF16) return s16 ? route_tma_launch_bf16_s16 : route_tma_launch_bf16;
+  return s16 ? route_tma_launch_f32_s16 : route_tma_launch_f32;
+}
 
 // Arguments common to the route and the fused decode.
 RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
@@ -268,14 +282,14 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   const long long cmax = a.cmax;
   cudaError_t e;
 
-  a.rows_bytes = (int)route_rows_bytes(D, a.cmax);
+  a.rows_bytes = (int)route_rows_bytes(D, a.cmax, sum_bytes(t));
   // Staged kernel when a query's widest level fits in shared memory.
   const size_t per_query = route_smem_layout(D, a.cmax, beam, a.rows_bytes, 0).total;
   if (per_query <= kRouteSmemCap) {
     a.query_smem_bytes = (int)per_query;
     // 8 rows per warp step, two steps in flight
     const StagedShape sh = staged_shape(t, a, per_query, 0);
-    e = route_tma_launch_nokv(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, kPathNone);
+    e = staged_launch(t, false)(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, kPathNone);
     ++t->launches;
     return e;
   }
@@ -297,8 +311,12 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   const size_t smem = (size_t)words * 8 * a.qpc;
   const int threads = a.qpc * a.wpq * 32;
   const unsigned blocks = (unsigned)((a.total_queries + a.qpc - 1) / a.qpc);
-  e = D == 128 ? run_route<128, kU128>(a, blocks, threads, smem, stream)
-               : run_route<64, kU64>(a, blocks, threads, smem, stream);
+  if (sum_bf16(t))
+    e = D == 128 ? run_route<128, kU128, uint16_t>(a, blocks, threads, smem, stream)
+                 : run_route<64, kU64, uint16_t>(a, blocks, threads, smem, stream);
+  else
+    e = D == 128 ? run_route<128, kU128, float>(a, blocks, threads, smem, stream)
+                 : run_route<64, kU64, float>(a, blocks, threads, smem, stream);
   ++t->launches;
   return e;
 }
@@ -322,7 +340,7 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
   for (int l = 0; l < t->L; ++l)
     cmax = std::max(cmax, std::min(std::min((long long)beam, t->n[l + 1]) * t->desc.branching, t->n[l]));
   const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
-  const size_t route_rows = route_rows_bytes(D, (int)cmax);
+  const size_t route_rows = route_rows_bytes(D, (int)cmax, sum_bytes(t));
   if (!wide) {
     p.nbuf = 2;
     p.rows_bytes = std::max(route_rows, (size_t)4 * 16 * row);  // two stages of 16 tokens at least
@@ -336,7 +354,7 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
   const size_t cap = own_sm ? 192 * 1024 : 96 * 1024;
   size_t rows = std::min((size_t)2 * row * (size_t)tokens, cap);  // all the tokens, if they fit
   rows = std::max(std::max(rows, route_rows), (size_t)4 * 16 * row);
-  p.path_bytes = path_smem_layout(D, row, (int)t->desc.leaf_block, t->desc.branching, t->L).total;
+  p.path_bytes = path_smem_layout(D, row, sum_bytes(t), (int)t->desc.leaf_block, t->desc.branching, t->L).total;
   p.path_off = route_align(route_rows, 128);
   if (own_sm) rows = std::max(rows, p.path_off + p.path_bytes);
   p.nbuf = rows >= (size_t)3 * 2 * 16 * row ? 3 : 2;
@@ -375,13 +393,8 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
     a.path_tokens = (int)(std::min(append_leaf * a.lb + a.lb, t->N) - append_leaf * a.lb);
     a.path_smem_off = (long long)p.path_off;  // inside the row region, after the route's rows
   }
-  cudaError_t e;
-  if (bf)
-    e = route_tma_launch_bf16(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream,
-                                  append ? kPathAppend : kPathNone);
-  else
-    e = route_tma_launch_f32(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream,
-                               append ? kPathAppend : kPathNone);
+  const cudaError_t e = staged_launch(t, true)(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream,
+                                               append ? kPathAppend : kPathNone);
   ++t->launches;
   return e;
 }
@@ -405,7 +418,7 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
   // Route only: the route's rows.  Attending: the decode plan's row region; in narrow
   // launches grown up to 64 KB, and any number of stages is accepted (the attention
   // pipelines them), since a causal pass has no two-launch fallback.
-  size_t rows = std::max(route_rows_bytes(D, a.cmax), (size_t)4 * 16 * row);
+  size_t rows = std::max(route_rows_bytes(D, a.cmax, sum_bytes(t)), (size_t)4 * 16 * row);
   int nbuf = 2, stage_tokens = (int)(rows / (4 * row)) / 16 * 16;
   if (attend) {
     rows = dp.rows_bytes;
@@ -431,7 +444,7 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
   a.positions = d_positions;
   const int pw_warps = wide ? kRouteMaxWarps : narrow_wpq(a.cmax);
   const size_t route_part = route_smem_layout(D, a.cmax, beam, (size_t)a.rows_bytes, pw_warps).total;
-  const size_t path_bytes = path_smem_layout(D, row, (int)a.lb, a.b, t->L).total;
+  const size_t path_bytes = path_smem_layout(D, row, sum_bytes(t), (int)a.lb, a.b, t->L).total;
   a.path_smem_off = (long long)route_align(route_part, 128);
   const size_t per_query = (size_t)a.path_smem_off + path_bytes;
   if ((attend && stage_tokens < 16) || per_query > (wide ? kCtaSmemCap : kRouteSmemCap)) {
@@ -440,10 +453,8 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
   }
   a.query_smem_bytes = (int)per_query;
   const StagedShape sh = staged_shape(t, a, per_query, attend ? dp.attn_warps : 0);
-  cudaError_t e = bf ? route_tma_launch_bf16(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem,
-                                                 stream, kPathPrefix)
-                     : route_tma_launch_f32(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem,
-                                              stream, kPathPrefix);
+  const cudaError_t e =
+      staged_launch(t, true)(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream, kPathPrefix);
   ++t->launches;
   return e;
 }

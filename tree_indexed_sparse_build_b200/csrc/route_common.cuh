@@ -21,8 +21,8 @@ struct RouteArgs {
   int q_bf16;
   int q_heads, nq, group, kv_heads;
   int head_dim;
-  const float* pyr;
-  long long pyr_unit_stride;  // floats
+  const void* pyr;            // summaries (the kernel's summary type)
+  long long pyr_unit_stride;  // elements
   long long off[kMaxLevels];
   long long n[kMaxLevels];
   int L, b, beam, cmax;
@@ -59,14 +59,19 @@ struct NoKV {};  // route only: no attention epilogue
 enum : int { kPathNone = 0, kPathAppend = 1, kPathPrefix = 2 };
 
 struct RouteArgs;
-// Launch route_tma_kernel for one KV type (route_tma_*.cu): route only (nokv), or route and
-// attention / path with bf16 or fp32 K rows.  narrow / grouped pick the launch shape.
-cudaError_t route_tma_launch_nokv(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
-                                  int threads, size_t smem, cudaStream_t s, int path);
-cudaError_t route_tma_launch_bf16(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
-                                  int threads, size_t smem, cudaStream_t s, int path);
-cudaError_t route_tma_launch_f32(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
-                                 int threads, size_t smem, cudaStream_t s, int path);
+// Launch route_tma_kernel for one KV type and summary type (route_tma_*.cu): route only
+// (nokv), or route and attention / path with bf16 or fp32 K rows; fp32 summaries, or bf16
+// summaries (the _s16 forms).  narrow / grouped pick the launch shape.
+#define ZHA_ROUTE_LAUNCH_DECL(name)                                                                    \
+  cudaError_t name(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks, int threads, \
+                   size_t smem, cudaStream_t s, int path)
+ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_nokv);
+ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_bf16);
+ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_f32);
+ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_nokv_s16);
+ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_bf16_s16);
+ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_f32_s16);
+#undef ZHA_ROUTE_LAUNCH_DECL
 
 
 constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
@@ -76,14 +81,16 @@ struct RouteSmem {
   size_t rows, keys, cand, surv_a, surv_b, leaf_sc, red, hist, pw, bar, total;
 };
 __host__ __device__ inline size_t route_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
-__host__ __device__ inline size_t route_rows_bytes(int D, int cmax) { return (size_t)cmax * D * 4; }
-// rows_bytes >= route_rows_bytes(D, cmax); a fused decode may ask for more room to stage
+__host__ __device__ inline size_t route_rows_bytes(int D, int cmax, int sum_bytes) {
+  return (size_t)cmax * D * sum_bytes;
+}
+// rows_bytes >= route_rows_bytes(D, cmax, sum_bytes); a fused decode may ask for more room to stage
 // K/V, and for 16 floats of softmax weights per attending warp (pw_warps).
 __host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam, size_t rows_bytes,
                                                        int pw_warps) {
   RouteSmem s;
   size_t o = 0;
-  s.rows = o;   // candidate summary rows, fp32 [cmax][D]; K/V stage buffers after the route
+  s.rows = o;   // candidate summary rows [cmax][D]; K/V stage buffers after the route
   o += rows_bytes;
   s.keys = o;   // candidate keys [cmax]
   o += (size_t)cmax * 8;

@@ -1,6 +1,6 @@
 // The staged route kernel (route_tma_kernel) and its launch helpers.  Its instantiations
-// are spread over route_tma_nokv.cu, route_tma_bf16.cu and route_tma_f32.cu (one per KV
-// type), which compile in parallel; route.cu plans the launches and calls them through
+// are spread over route_tma_{nokv,bf16,f32}{,_s16}.cu (one per KV type and summary type),
+// which compile in parallel; route.cu plans the launches and calls them through
 // route_tma_launch_* (route_common.cuh).
 #pragma once
 
@@ -35,7 +35,9 @@ namespace zha {
 //    positions[qg % nq]: its own depth and node counts, and its prefix's right edge
 //    recomputed into shared memory (never stored).
 // With a KV type, the query then attends over its leaves unless O is null.
-template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH = kPathNone>
+// TS: the summaries' storage (float, or bf16 bits in uint16_t); rows are staged as stored
+// and widened to fp32 as they are scored.
+template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH, typename TS>
 __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3 : 1)
     route_tma_kernel(const RouteArgs a) {
   constexpr bool ATTEND = !std::is_same<TKV, NoKV>::value;
@@ -43,7 +45,9 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   constexpr bool PREFIX = PATH == kPathPrefix;
   constexpr bool HASPATH = PATH != kPathNone;
   static_assert(!HASPATH || ATTEND, "the path reads K rows of type TKV");
-  constexpr int CPL = D / 16;  // 16-byte chunks of a row per lane (4 lanes per row)
+  constexpr int EPC = 16 / (int)sizeof(TS);      // summary elements per 16-byte chunk
+  constexpr int CPL = D * (int)sizeof(TS) / 64;  // 16-byte chunks of a row per lane (4 lanes per row)
+  constexpr uint32_t SROW = D * (uint32_t)sizeof(TS);  // bytes of a summary row
   constexpr int R = 8;         // candidate keys held per lane in the selecting warp
   extern __shared__ __align__(128) unsigned char rsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -56,7 +60,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   const RouteSmem Ls =
       route_smem_layout(D, a.cmax, a.beam, (size_t)a.rows_bytes, ATTEND ? nw : 0);
   unsigned char* base = rsm + (size_t)qi * a.query_smem_bytes;
-  const float* rows = reinterpret_cast<const float*>(base + Ls.rows);
+  const TS* rows = reinterpret_cast<const TS*>(base + Ls.rows);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + Ls.keys);
   int* cand = reinterpret_cast<int*>(base + Ls.cand);
   int* surv_a = reinterpret_cast<int*>(base + Ls.surv_a);
@@ -77,11 +81,11 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     const int h = (int)(hq_flat % a.q_heads);
     unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
   }
-  const float* pyr_u = a.pyr + unit * a.pyr_unit_stride;
+  const TS* pyr_u = static_cast<const TS*>(a.pyr) + unit * a.pyr_unit_stride;
   // the path region (fused append or causal prefix)
   unsigned char* pb = base + a.path_smem_off;
   PathSmem Ps{};
-  if (HASPATH) Ps = path_smem_layout(D, D * (int)sizeof(TKV), (int)a.lb, a.b, a.L);
+  if (HASPATH) Ps = path_smem_layout(D, D * (int)sizeof(TKV), (int)sizeof(TS), (int)a.lb, a.b, a.L);
   uint64_t* pbar = reinterpret_cast<uint64_t*>(pb + Ps.bar);
   // this query's tree: the whole tree, or (PREFIX) the tree of its prefix
   long long Nq = a.N;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         fence_proxy_async_smem();
         const long long leaf = APPEND ? a.path_leaf : (Nq - 1) / a.lb;
         const int ntok = APPEND ? a.path_tokens : (int)(Nq - leaf * a.lb);
-        path_issue<TKV, D>(Ps, pb, a.K + unit * a.kv_unit_stride, pyr_u, a.off, nl, a.b, Lq, leaf,
+        path_issue<TKV, TS, D>(Ps, pb, a.K + unit * a.kv_unit_stride, pyr_u, a.off, nl, a.b, Lq, leaf,
                            ntok, a.lb, pbar);
       }
     }
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   // Four lanes per row: lane (rg = lane / 4, sub = lane % 4) reads chunks 4 (j ^ par) + sub,
   // par = rg & 1, so the two rows of a shared-memory phase use opposite bank halves.
   const int sub = lane & 3, rg = lane >> 2, par = rg & 1;
-  float4 qv[CPL];
+  float qv[CPL][EPC];
   int* cur = surv_a;
   int* nxt = surv_b;
   int m = live ? 1 : 0;
@@ -143,16 +147,16 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       const long long last = cur[m - 1];
       C = (m - 1) * a.b + (int)min((long long)a.b, nl[l] - (long long)a.b * last);
     }
-    const float* S = pyr_u + a.off[l] * D;
+    const TS* S = pyr_u + a.off[l] * D;
     if (wq == 0 && C > 0) {
       // one bulk copy per survivor (its children are consecutive rows) + candidate ids
-      if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)C * D * 4);
+      if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)C * SROW);
       __syncwarp();
       fence_proxy_async_smem();
       for (int j = lane; j < m; j += 32) {
         const long long node0 = (long long)a.b * cur[j];
         const int nc = (int)min((long long)a.b, nl[l] - node0);
-        bulk_copy_g2s((void*)(rows + (size_t)j * a.b * D), S + node0 * D, (uint32_t)nc * D * 4, bar);
+        bulk_copy_g2s((void*)(rows + (size_t)j * a.b * D), S + node0 * D, (uint32_t)nc * SROW, bar);
       }
       for (int j = lane; j < m; j += 32) {  // survivor j's children are candidates j b ..
         const int node0 = a.b * cur[j];
@@ -178,12 +182,10 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
         const int c = 4 * (j ^ par) + sub;
-        float f[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          f[e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[qo + 4 * c + e])
-                          : static_cast<const float*>(a.Q)[qo + 4 * c + e];
-        qv[j] = make_float4(f[0], f[1], f[2], f[3]);
+        for (int e = 0; e < EPC; ++e)
+          qv[j][e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[qo + EPC * c + e])
+                              : static_cast<const float*>(a.Q)[qo + EPC * c + e];
       }
     }
     if (HASPATH && l == Lq - 1) {
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
           // fused append: the first query of each unit stores the path
           const bool writer = APPEND && (qg % a.nq) == 0 && ((qg / a.nq) % a.q_heads) % a.group == 0;
           const int ntok = APPEND ? a.path_tokens : (int)(Nq - ((Nq - 1) / a.lb) * a.lb);
-          path_compute<TKV, D>(Ps, pb, const_cast<float*>(pyr_u), a.off, nl, a.b, Lq, ntok, writer,
+          path_compute<TKV, TS, D>(Ps, pb, const_cast<TS*>(pyr_u), a.off, nl, a.b, Lq, ntok, writer,
                                32 * wq + lane, bar_n, qsync);
         }
       }
@@ -221,8 +223,8 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       // past the query's prefix: use the recomputed one
       const int k = *reinterpret_cast<const int*>(pb + Ps.kpos);
       if (k >= 0) {
-        const float* pf = reinterpret_cast<const float*>(pb + Ps.pf) + (size_t)l * D;
-        float* dst = const_cast<float*>(rows) + (size_t)k * D;
+        const TS* pf = reinterpret_cast<const TS*>(pb + Ps.pf) + (size_t)l * D;
+        TS* dst = const_cast<TS*>(rows) + (size_t)k * D;
         for (int e = 32 * wq + lane; e < D; e += bar_n) dst[e] = pf[e];
         qsync();
       }
@@ -238,12 +240,17 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         acc[u][0] = make_float2(0.f, 0.f);
         acc[u][1] = make_float2(0.f, 0.f);
         if (r < C) {
-          const float4* row = reinterpret_cast<const float4*>(rows + (size_t)r * D);
+          const uint4* row = reinterpret_cast<const uint4*>(rows + (size_t)r * D);
 #pragma unroll
           for (int j = 0; j < CPL; ++j) {
-            const float4 v = row[4 * (j ^ par) + sub];
-            acc[u][0] = __ffma2_rn(make_float2(qv[j].x, qv[j].y), make_float2(v.x, v.y), acc[u][0]);
-            acc[u][1] = __ffma2_rn(make_float2(qv[j].z, qv[j].w), make_float2(v.z, v.w), acc[u][1]);
+            float v[EPC];
+            Vec16<TS>::to_f32(row[4 * (j ^ par) + sub], v);
+#pragma unroll
+            for (int e = 0; e < EPC; e += 4) {
+              acc[u][0] = __ffma2_rn(make_float2(qv[j][e], qv[j][e + 1]), make_float2(v[e], v[e + 1]), acc[u][0]);
+              acc[u][1] =
+                  __ffma2_rn(make_float2(qv[j][e + 2], qv[j][e + 3]), make_float2(v[e + 2], v[e + 3]), acc[u][1]);
+            }
           }
         }
       }
@@ -333,10 +340,10 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   }
 }
 
-template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH = kPathNone>
+template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH, typename TS>
 cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size_t smem,
                           cudaStream_t s) {
-  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW, PATH>;
+  auto kern = route_tma_kernel<D, GROUPED, TKV, NARROW, PATH, TS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, a);
@@ -344,35 +351,37 @@ cudaError_t run_route_tma(const RouteArgs& a, unsigned blocks, int threads, size
   return cudaGetLastError();
 }
 
-template <typename TKV, int PATH>
+template <typename TKV, int PATH, typename TS>
 cudaError_t run_shape(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks, int threads,
                       size_t smem, cudaStream_t s) {
   if constexpr (PATH != kPathAppend) {  // the fused append runs in wide launches only
     if (narrow) {
       if (grouped)
-        return D == 128 ? run_route_tma<128, true, TKV, true, PATH>(a, blocks, threads, smem, s)
-                        : run_route_tma<64, true, TKV, true, PATH>(a, blocks, threads, smem, s);
-      return D == 128 ? run_route_tma<128, false, TKV, true, PATH>(a, blocks, threads, smem, s)
-                      : run_route_tma<64, false, TKV, true, PATH>(a, blocks, threads, smem, s);
+        return D == 128 ? run_route_tma<128, true, TKV, true, PATH, TS>(a, blocks, threads, smem, s)
+                        : run_route_tma<64, true, TKV, true, PATH, TS>(a, blocks, threads, smem, s);
+      return D == 128 ? run_route_tma<128, false, TKV, true, PATH, TS>(a, blocks, threads, smem, s)
+                      : run_route_tma<64, false, TKV, true, PATH, TS>(a, blocks, threads, smem, s);
     }
   } else if (narrow) {
     return cudaErrorNotSupported;
   }
   if (grouped)
-    return D == 128 ? run_route_tma<128, true, TKV, false, PATH>(a, blocks, threads, smem, s)
-                    : run_route_tma<64, true, TKV, false, PATH>(a, blocks, threads, smem, s);
-  return D == 128 ? run_route_tma<128, false, TKV, false, PATH>(a, blocks, threads, smem, s)
-                  : run_route_tma<64, false, TKV, false, PATH>(a, blocks, threads, smem, s);
+    return D == 128 ? run_route_tma<128, true, TKV, false, PATH, TS>(a, blocks, threads, smem, s)
+                    : run_route_tma<64, true, TKV, false, PATH, TS>(a, blocks, threads, smem, s);
+  return D == 128 ? run_route_tma<128, false, TKV, false, PATH, TS>(a, blocks, threads, smem, s)
+                  : run_route_tma<64, false, TKV, false, PATH, TS>(a, blocks, threads, smem, s);
 }
 
-template <typename TKV>
+template <typename TKV, typename TS>
 cudaError_t run_route_tma_d_impl(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
-                            int threads, size_t smem, cudaStream_t s, int path = kPathNone) {
+                                 int threads, size_t smem, cudaStream_t s, int path = kPathNone) {
   if constexpr (!std::is_same<TKV, NoKV>::value) {
-    if (path == kPathAppend) return run_shape<TKV, kPathAppend>(D, grouped, narrow, a, blocks, threads, smem, s);
-    if (path == kPathPrefix) return run_shape<TKV, kPathPrefix>(D, grouped, narrow, a, blocks, threads, smem, s);
+    if (path == kPathAppend)
+      return run_shape<TKV, kPathAppend, TS>(D, grouped, narrow, a, blocks, threads, smem, s);
+    if (path == kPathPrefix)
+      return run_shape<TKV, kPathPrefix, TS>(D, grouped, narrow, a, blocks, threads, smem, s);
   }
-  return run_shape<TKV, kPathNone>(D, grouped, narrow, a, blocks, threads, smem, s);
+  return run_shape<TKV, kPathNone, TS>(D, grouped, narrow, a, blocks, threads, smem, s);
 }
 
 }  // namespace zha

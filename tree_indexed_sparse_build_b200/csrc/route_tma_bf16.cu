@@ -1,11 +1,11 @@
-// Instantiations of route_tma_kernel with KV type uint16_t (see route_kernel.cuh).
+// Instantiations of route_tma_kernel for bf16 K/V rows and fp32 summaries (see route_kernel.cuh).
 #include "route_kernel.cuh"
 
 namespace zha {
 
 cudaError_t route_tma_launch_bf16(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
                                  int threads, size_t smem, cudaStream_t s, int path) {
-  return run_route_tma_d_impl<uint16_t>(D, grouped, narrow, a, blocks, threads, smem, s, path);
+  return run_route_tma_d_impl<uint16_t, float>(D, grouped, narrow, a, blocks, threads, smem, s, path);
 }
 
 }  // namespace zha

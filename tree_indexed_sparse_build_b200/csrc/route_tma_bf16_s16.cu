@@ -1,0 +1,11 @@
+// Instantiations of route_tma_kernel for bf16 K/V rows and bf16 summaries (see route_kernel.cuh).
+#include "route_kernel.cuh"
+
+namespace zha {
+
+cudaError_t route_tma_launch_bf16_s16(int D, bool grouped, bool narrow, const RouteArgs& a, unsigned blocks,
+                                 int threads, size_t smem, cudaStream_t s, int path) {
+  return run_route_tma_d_impl<uint16_t, uint16_t>(D, grouped, narrow, a, blocks, threads, smem, s, path);
+}
+
+}  // namespace zha

@@ -31,8 +31,8 @@ struct ThreshArgs {
   const void* Q;
   int q_bf16;
   int q_heads, nq, group, kv_heads;
-  const float* pyr;
-  long long pyr_unit_stride;  // floats
+  const void* pyr;            // summaries (fp32 or bf16, the kernel's TS)
+  long long pyr_unit_stride;  // elements
   const float* radii;
   long long off[kMaxLevels];
   long long n[kMaxLevels];
@@ -85,7 +85,7 @@ __device__ int chunk_compact(const unsigned char* flags, int n, int* pos, int* w
   return total;
 }
 
-template <typename TK, int D>
+template <typename TK, typename TS, int D>
 __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs a) {
   constexpr int DPL = D / 32;
   extern __shared__ __align__(16) unsigned char tsm[];
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
   const long long hq_flat = qg / a.nq;
   const int h = (int)(hq_flat % a.q_heads);
   const long long unit = (hq_flat / a.q_heads) * a.kv_heads + h / a.group;
-  const float* pu = a.pyr + unit * a.pyr_unit_stride;
+  const TS* pu = static_cast<const TS*>(a.pyr) + unit * a.pyr_unit_stride;
   const float* ru = a.radii + unit * (a.pyr_unit_stride / D);
   const TK* Ku = reinterpret_cast<const TK*>(a.K + unit * a.k_unit_stride);
   const double tau = (double)a.tau[qg];
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
   __syncthreads();
   for (int l = a.L - 1; l >= 0 && !overflow; --l) {
     const long long total = (long long)m * a.b;  // child slots of the survivors
-    const float* S = pu + a.off[l] * D;
+    const TS* S = pu + a.off[l] * D;
     const float* R = ru + a.off[l];
     int mn = 0;
     for (long long c0 = 0; c0 < total; c0 += kChunk) {
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
           double dot = 0.0, mag = 0.0;
 #pragma unroll
           for (int e = 0; e < DPL; ++e) {
-            const double c = (double)S[node * D + lane * DPL + e];
+            const double c = (double)SumT<TS>::load(S[node * D + lane * DPL + e]);
             dot = fma(qv[e], c, dot);
             mag += fabs(qv[e] * c);
           }
@@ -225,9 +225,9 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
   }
 }
 
-template <typename TK, int D>
+template <typename TK, typename TS, int D>
 cudaError_t run_threshold(const ThreshArgs& a, size_t smem, cudaStream_t s) {
-  auto kern = threshold_kernel<TK, D>;
+  auto kern = threshold_kernel<TK, TS, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3((unsigned)a.total_queries), dim3(kThThreads), smem, s, a);
@@ -242,6 +242,7 @@ cudaError_t launch_threshold(zha_tree* t, const void* d_K, const void* d_Q, zha_
   ThreshArgs a{};
   const int D = t->desc.head_dim;
   const bool bf = t->desc.kv_dtype == ZHA_BF16;
+  const bool sbf = sum_bf16(t);
   a.Q = d_Q;
   a.q_bf16 = q_dtype == ZHA_BF16;
   a.q_heads = q_heads;
@@ -269,10 +270,16 @@ cudaError_t launch_threshold(zha_tree* t, const void* d_K, const void* d_Q, zha_
   a.total_queries = (long long)t->desc.batch * q_heads * nq;
   const size_t smem = (size_t)2 * kFrontierCap * 4 + kChunk * 4 + kChunk + kThWarps * 4;
   cudaError_t e;
-  if (bf)
-    e = D == 128 ? run_threshold<uint16_t, 128>(a, smem, stream) : run_threshold<uint16_t, 64>(a, smem, stream);
+  if (sbf)
+    e = bf ? (D == 128 ? run_threshold<uint16_t, uint16_t, 128>(a, smem, stream)
+                       : run_threshold<uint16_t, uint16_t, 64>(a, smem, stream))
+           : (D == 128 ? run_threshold<float, uint16_t, 128>(a, smem, stream)
+                       : run_threshold<float, uint16_t, 64>(a, smem, stream));
   else
-    e = D == 128 ? run_threshold<float, 128>(a, smem, stream) : run_threshold<float, 64>(a, smem, stream);
+    e = bf ? (D == 128 ? run_threshold<uint16_t, float, 128>(a, smem, stream)
+                       : run_threshold<uint16_t, float, 64>(a, smem, stream))
+           : (D == 128 ? run_threshold<float, float, 128>(a, smem, stream)
+                       : run_threshold<float, float, 64>(a, smem, stream));
   ++t->launches;
   return e;
 }

@@ -4,11 +4,13 @@
 // over the KV cache; the tree deepens as the cache grows).
 //
 // One launch ("pass") computes a first level from its source rows (K tokens for the
-// leaves, or the stored fp32 level below) and up to k further levels above it inside
-// the CTA.  A CTA owns `chunk` consecutive first-level nodes, a multiple of b^k, so the
-// k upper levels of its subtree need no other CTA.  Sums are formed in fp64 and kept in
-// shared memory in fp64 between the levels of a pass; each level is rounded once to
-// fp32 when stored.  Only nodes inside the touched range [lo, hi] of each level are
+// leaves, or the stored level below) and up to k further levels above it inside the CTA.
+// A CTA owns `chunk` consecutive first-level nodes, a multiple of b^k, so the k upper
+// levels of its subtree need no other CTA.  Sums are formed in fp64 and kept in shared
+// memory in fp64 between the levels of a pass; each level is rounded once when stored
+// (fp32 storage), or to fp32 and then bf16 (bf16 storage, where the kept fp64 value is the
+// stored one, so a parent always averages its children's stored values; SumT in
+// device_common.cuh).  Only nodes inside the touched range [lo, hi] of each level are
 // recomputed; the others are read back from the pyramid (append).
 //
 // Memory: the first pass streams K once with 16-byte coalesced loads (a row of
@@ -34,8 +36,8 @@ struct PassArgs {
   int b;
   int k;                              // levels above the first, inside the CTA
   int chunk;                          // first-level nodes per CTA (multiple of b^k)
-  float* pyr;                         // unit 0 of the pyramid
-  long long pyr_unit_stride;          // floats between units
+  void* pyr;                          // unit 0 of the pyramid (summary storage type)
+  long long pyr_unit_stride;          // elements between units
   long long lvl_off[kMaxPassLevels];  // row offset of the pass's level m inside a unit
   long long lvl_n[kMaxPassLevels];    // nodes at level m
   long long lo[kMaxPassLevels];       // touched range at level m (inclusive)
@@ -43,7 +45,21 @@ struct PassArgs {
   long long chunk0;                   // chunk index of blockIdx.x == 0
 };
 
-template <typename TIn, int D>
+// VEC consecutive stored elements from registers (16- or 8-byte stores).
+template <typename TS, int VEC>
+__device__ __forceinline__ void store_piece(TS* dst, const TS* v) {
+  constexpr int BYTES = VEC * (int)sizeof(TS);
+  if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+    for (int c = 0; c < BYTES / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(v)[c];
+  } else {
+    static_assert(BYTES == 8, "4 bf16 values");
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(v);
+  }
+}
+
+// TIn: the source rows' type (K's, or the summaries' for the upper passes); TS: summaries.
+template <typename TIn, typename TS, int D>
 __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassArgs a) {
   constexpr int VEC = Vec16<TIn>::N;  // elements per 16-byte load
   constexpr int LPR = D / VEC;        // lanes covering one row
@@ -64,14 +80,14 @@ __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassAr
   const int slot = warp * SPW + lane / LPR;
   const int col = (lane % LPR) * VEC;
   const char* src = a.src + (long long)unit * a.src_unit_stride + (long long)col * sizeof(TIn);
-  float* pyr_u = a.pyr + (long long)unit * a.pyr_unit_stride;
+  TS* pyr_u = static_cast<TS*>(a.pyr) + (long long)unit * a.pyr_unit_stride;
 
   // ---- first level of the pass: one node per lane group
   const long long base0 = chunk * a.chunk;
   for (int j = slot; j < a.chunk; j += SLOTS) {
     const long long i = base0 + j;
     if (i >= a.lvl_n[0]) break;  // nodes ascend with j
-    float* dst = pyr_u + (a.lvl_off[0] + i) * D + col;
+    TS* dst = pyr_u + (a.lvl_off[0] + i) * D + col;
     double* sm = bufA + (size_t)j * D + col;
     if (i >= a.lo[0] && i <= a.hi[0]) {
       const long long r0 = i * a.blk0;
@@ -101,25 +117,17 @@ __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassAr
         for (int e = 0; e < VEC; ++e) acc[e] += (double)f[e];
       }
       const double cnt = (double)nrows;
-      float out[VEC];
+      alignas(16) TS out[VEC];
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
-        acc[e] = acc[e] / cnt;
-        out[e] = (float)acc[e];
-        sm[e] = acc[e];
+        const double v = acc[e] / cnt;
+        out[e] = SumT<TS>::store(v);
+        sm[e] = SumT<TS>::kept(v);
       }
-#pragma unroll
-      for (int e = 0; e < VEC; e += 4)
-        *reinterpret_cast<float4*>(dst + e) = make_float4(out[e], out[e + 1], out[e + 2], out[e + 3]);
+      store_piece<TS, VEC>(dst, out);
     } else {
 #pragma unroll
-      for (int e = 0; e < VEC; e += 4) {
-        const float4 s = *reinterpret_cast<const float4*>(dst + e);
-        sm[e] = s.x;
-        sm[e + 1] = s.y;
-        sm[e + 2] = s.z;
-        sm[e + 3] = s.w;
-      }
+      for (int e = 0; e < VEC; ++e) sm[e] = (double)SumT<TS>::load(dst[e]);
     }
   }
   __syncthreads();
@@ -137,16 +145,17 @@ __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassAr
       const long long i = basem + j;
       if (i >= a.lvl_n[m]) continue;
       double v;
-      float* dst = pyr_u + (a.lvl_off[m] + i) * D + e;
+      TS* dst = pyr_u + (a.lvl_off[m] + i) * D + e;
       if (i >= a.lo[m] && i <= a.hi[m]) {
         const long long c0 = i * a.b;
         const long long c1 = min(c0 + (long long)a.b, a.lvl_n[m - 1]);
         double s = 0.0;
         for (long long c = c0; c < c1; ++c) s += cur[(size_t)(c - basec) * D + e];
-        v = s / (double)(c1 - c0);
-        *dst = (float)v;
+        const double mean = s / (double)(c1 - c0);
+        *dst = SumT<TS>::store(mean);
+        v = SumT<TS>::kept(mean);
       } else {
-        v = (double)*dst;
+        v = (double)SumT<TS>::load(*dst);
       }
       nxt[(size_t)j * D + e] = v;
     }
@@ -176,8 +185,8 @@ struct AppendPathArgs {
   long long k_unit_stride;     // bytes between units
   long long N, lb;
   int b, L;
-  float* pyr;
-  long long pyr_unit_stride;   // floats
+  void* pyr;
+  long long pyr_unit_stride;   // elements
   long long off[kMaxLevels];
   long long n[kMaxLevels];
   long long lo, hi;            // touched leaves
@@ -190,12 +199,12 @@ struct AppendPathArgs {
   unsigned* err;
 };
 
-template <typename TIn, int D>
+template <typename TIn, typename TS, int D>
 __global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendPathArgs a) {
   extern __shared__ __align__(128) unsigned char psm[];
   const int unit = blockIdx.x;
   const char* Ku = a.K + (long long)unit * a.k_unit_stride;
-  float* pyr_u = a.pyr + (long long)unit * a.pyr_unit_stride;
+  TS* pyr_u = static_cast<TS*>(a.pyr) + (long long)unit * a.pyr_unit_stride;
   const TIn* tok = reinterpret_cast<const TIn*>(psm);
   double* cur = reinterpret_cast<double*>(psm + a.fp64_off);
   double* nxt = cur + kPathMaxLeaves * D;
@@ -207,14 +216,14 @@ __global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendP
     mbar_init(bar, 1);
     fence_mbar_init();
     uint32_t bytes = (uint32_t)a.tok_rows * D * sizeof(TIn);
-    for (int l = 1; l <= a.L; ++l) bytes += (uint32_t)a.sib_rows[l] * D * 4;
+    for (int l = 1; l <= a.L; ++l) bytes += (uint32_t)a.sib_rows[l] * D * (uint32_t)sizeof(TS);
     mbar_arrive_expect_tx(bar, bytes);
     const long long r0 = a.lo * a.lb;
     bulk_copy_g2s(psm, Ku + r0 * D * (long long)sizeof(TIn), (uint32_t)a.tok_rows * D * sizeof(TIn), bar);
     for (int l = 1; l <= a.L; ++l)
       if (a.sib_rows[l] > 0)
         bulk_copy_g2s(psm + a.sib_off[l], pyr_u + (a.off[l - 1] + a.sib0[l]) * D,
-                      (uint32_t)a.sib_rows[l] * D * 4, bar);
+                      (uint32_t)a.sib_rows[l] * D * (uint32_t)sizeof(TS), bar);
   }
   __syncthreads();
   const bool ok = mbar_wait_bounded(bar, 0, a.err, kDevErrTimeout, kPathWaitCycles);
@@ -238,8 +247,8 @@ __global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendP
         s += (double)tok[(base + r) * D + e];
     }
     const double v = s / (double)(r1 - r0);
-    cur[j * D + e] = v;
-    pyr_u[(a.off[0] + i) * D + e] = (float)v;
+    cur[j * D + e] = SumT<TS>::kept(v);
+    pyr_u[(a.off[0] + i) * D + e] = SumT<TS>::store(v);
   }
   __syncthreads();
 
@@ -247,17 +256,17 @@ __global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendP
   for (int l = 1; l <= a.L; ++l) {
     const long long plo = lo / a.b, phi = hi / a.b;
     const int np = (int)(phi - plo + 1);
-    const float* sib = reinterpret_cast<const float*>(psm + a.sib_off[l]);
+    const TS* sib = reinterpret_cast<const TS*>(psm + a.sib_off[l]);
     for (int idx = threadIdx.x; idx < np * D; idx += kPathThreads) {
       const int j = idx / D, e = idx - (idx / D) * D;
       const long long i = plo + j;
       const long long c0 = i * a.b, c1 = min(c0 + (long long)a.b, a.n[l - 1]);
       double s = 0.0;
       for (long long c = c0; c < c1; ++c)
-        s += (c >= lo && c <= hi) ? cur[(c - lo) * D + e] : (double)sib[(c - a.sib0[l]) * D + e];
+        s += (c >= lo && c <= hi) ? cur[(c - lo) * D + e] : (double)SumT<TS>::load(sib[(c - a.sib0[l]) * D + e]);
       const double v = s / (double)(c1 - c0);
-      nxt[j * D + e] = v;
-      pyr_u[(a.off[l] + i) * D + e] = (float)v;
+      nxt[j * D + e] = SumT<TS>::kept(v);
+      pyr_u[(a.off[l] + i) * D + e] = SumT<TS>::store(v);
     }
     __syncthreads();
     double* tmp = cur;
@@ -281,9 +290,9 @@ int levels_for(long long n0, long long b) {
 
 namespace {
 
-template <typename TIn, int D>
+template <typename TIn, typename TS, int D>
 cudaError_t launch_pass(const PassArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-  auto kern = pyramid_pass_kernel<TIn, D>;
+  auto kern = pyramid_pass_kernel<TIn, TS, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, grid, dim3(kPassThreads), smem, s, a);
@@ -291,9 +300,9 @@ cudaError_t launch_pass(const PassArgs& a, dim3 grid, size_t smem, cudaStream_t 
   return cudaGetLastError();
 }
 
-template <typename TIn, int D>
+template <typename TIn, typename TS, int D>
 cudaError_t launch_path(const AppendPathArgs& a, unsigned grid, size_t smem, cudaStream_t s) {
-  auto kern = append_path_kernel<TIn, D>;
+  auto kern = append_path_kernel<TIn, TS, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(grid), dim3(kPathThreads), smem, s, a);
@@ -312,6 +321,8 @@ long long ipow(long long b, int k) {
 cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long lo,
                            long long hi, cudaStream_t stream, int* launches) {
   const int D = t->desc.head_dim;
+  const bool sbf = sum_bf16(t);
+  const int ssz = sum_bytes(t);
   if (hi - lo + 1 <= kPathMaxLeaves) {
     // a few touched leaves (small appends, tiny trees): one launch walks the path to the root
     AppendPathArgs a{};
@@ -342,7 +353,7 @@ cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long 
       a.sib0[l] = r0;
       a.sib_rows[l] = (int)(r1 - r0);
       a.sib_off[l] = (int)o;
-      o += (size_t)(r1 - r0) * D * 4;
+      o += (size_t)(r1 - r0) * D * ssz;
       clo = plo;
       chi = phi;
     }
@@ -354,12 +365,16 @@ cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long 
     if (o <= kPathSmemCap) {
       const unsigned grid = (unsigned)t->units;
       cudaError_t e;
-      if (bf)
-        e = D == 128 ? launch_path<uint16_t, 128>(a, grid, o, stream)
-                     : launch_path<uint16_t, 64>(a, grid, o, stream);
+      if (sbf)
+        e = bf ? (D == 128 ? launch_path<uint16_t, uint16_t, 128>(a, grid, o, stream)
+                           : launch_path<uint16_t, uint16_t, 64>(a, grid, o, stream))
+               : (D == 128 ? launch_path<float, uint16_t, 128>(a, grid, o, stream)
+                           : launch_path<float, uint16_t, 64>(a, grid, o, stream));
       else
-        e = D == 128 ? launch_path<float, 128>(a, grid, o, stream)
-                     : launch_path<float, 64>(a, grid, o, stream);
+        e = bf ? (D == 128 ? launch_path<uint16_t, float, 128>(a, grid, o, stream)
+                           : launch_path<uint16_t, float, 64>(a, grid, o, stream))
+               : (D == 128 ? launch_path<float, float, 128>(a, grid, o, stream)
+                           : launch_path<float, float, 64>(a, grid, o, stream));
       ++t->launches;
       if (launches) *launches = 1;
       return e;
@@ -391,15 +406,16 @@ cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long 
       a.hi[m] = std::min(hi_l / sm, t->n[level + m] - 1);
     }
     const bool from_tokens = level == 0;
-    const size_t esz = (from_tokens && t->desc.kv_dtype == ZHA_BF16) ? 2 : 4;
+    // source rows: K tokens (the cache's type) or the stored level below (the summaries')
+    const bool src_bf = from_tokens ? t->desc.kv_dtype == ZHA_BF16 : sbf;
     if (from_tokens) {
       a.src = static_cast<const char*>(d_K);
-      a.src_unit_stride = t->desc.capacity_tokens * D * (long long)esz;
+      a.src_unit_stride = t->desc.capacity_tokens * D * (long long)(src_bf ? 2 : 4);
       a.n_src = N;
       a.blk0 = t->desc.leaf_block;
     } else {
-      a.src = reinterpret_cast<const char*>(t->pyr + t->off[level - 1] * D);
-      a.src_unit_stride = t->unit_rows * D * 4;
+      a.src = static_cast<const char*>(t->pyr) + t->off[level - 1] * D * (long long)ssz;
+      a.src_unit_stride = t->unit_rows * D * (long long)ssz;
       a.n_src = t->n[level - 1];
       a.blk0 = b;
     }
@@ -408,12 +424,16 @@ cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long 
     dim3 grid((unsigned)(c1 - c0 + 1), (unsigned)t->units);
     const size_t smem = (size_t)(chunk + (k > 0 ? chunk / b : 0)) * D * sizeof(double);
     cudaError_t e;
-    if (from_tokens && t->desc.kv_dtype == ZHA_BF16)
-      e = D == 128 ? launch_pass<uint16_t, 128>(a, grid, smem, stream)
-                   : launch_pass<uint16_t, 64>(a, grid, smem, stream);
+    if (sbf)
+      e = src_bf ? (D == 128 ? launch_pass<uint16_t, uint16_t, 128>(a, grid, smem, stream)
+                             : launch_pass<uint16_t, uint16_t, 64>(a, grid, smem, stream))
+                 : (D == 128 ? launch_pass<float, uint16_t, 128>(a, grid, smem, stream)
+                             : launch_pass<float, uint16_t, 64>(a, grid, smem, stream));
     else
-      e = D == 128 ? launch_pass<float, 128>(a, grid, smem, stream)
-                   : launch_pass<float, 64>(a, grid, smem, stream);
+      e = src_bf ? (D == 128 ? launch_pass<uint16_t, float, 128>(a, grid, smem, stream)
+                             : launch_pass<uint16_t, float, 64>(a, grid, smem, stream))
+                 : (D == 128 ? launch_pass<float, float, 128>(a, grid, smem, stream)
+                             : launch_pass<float, float, 64>(a, grid, smem, stream));
     if (e != cudaSuccess) return e;
     ++count;
     ++t->launches;

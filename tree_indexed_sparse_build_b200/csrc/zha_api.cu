@@ -17,6 +17,7 @@ bool desc_ok(const zha_tree_desc* d) {
   if (d->batch < 1 || d->kv_heads < 1 || (long long)d->batch * d->kv_heads > 65535) return false;
   if (d->branching < 2 || d->leaf_block < 1 || d->capacity_tokens < 1) return false;
   if (d->kv_dtype != ZHA_F32 && d->kv_dtype != ZHA_BF16) return false;
+  if (d->summary_dtype != ZHA_F32 && d->summary_dtype != ZHA_BF16) return false;
   return true;
 }
 
@@ -63,7 +64,8 @@ size_t zha_tree_workspace_bytes(const zha_tree_desc* desc) {
   long long ncap[kMaxLevels], off[kMaxLevels], rows;
   int L;
   if (!layout(desc, ncap, off, &L, &rows)) return 0;
-  return kHeaderBytes + (size_t)desc->batch * desc->kv_heads * (size_t)rows * desc->head_dim * 4;
+  const size_t esz = desc->summary_dtype == ZHA_BF16 ? 2 : 4;
+  return kHeaderBytes + (size_t)desc->batch * desc->kv_heads * (size_t)rows * desc->head_dim * esz;
 }
 
 zha_status zha_tree_init(const zha_tree_desc* desc, void* d_workspace, size_t workspace_bytes,
@@ -82,7 +84,7 @@ zha_status zha_tree_init(const zha_tree_desc* desc, void* d_workspace, size_t wo
   t->ws = static_cast<char*>(d_workspace);
   t->ws_bytes = workspace_bytes;
   t->d_err = reinterpret_cast<unsigned*>(t->ws);
-  t->pyr = reinterpret_cast<float*>(t->ws + kHeaderBytes);
+  t->pyr = t->ws + kHeaderBytes;
   t->units = (long long)desc->batch * desc->kv_heads;
   layout(desc, t->ncap, t->off, &t->Lcap, &t->unit_rows);
   set_shape(t, 0);
@@ -345,7 +347,7 @@ long long zha_tree_level_offset(const zha_tree* t, int level) {
   return t->off[level];
 }
 long long zha_tree_unit_rows(const zha_tree* t) { return t ? t->unit_rows : 0; }
-const float* zha_tree_summaries(const zha_tree* t) { return t ? t->pyr : nullptr; }
+const void* zha_tree_summaries(const zha_tree* t) { return t ? t->pyr : nullptr; }
 long long zha_tree_launch_count(const zha_tree* t) { return t ? t->launches : -1; }
 
 const char* zha_status_string(zha_status s) {

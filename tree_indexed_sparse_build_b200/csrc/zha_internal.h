@@ -41,7 +41,7 @@ struct zha_tree {
   char* ws;                    // caller's workspace
   size_t ws_bytes;
   unsigned* d_err;             // device error word (workspace header)
-  float* pyr;                  // summaries: [units][unit_rows][head_dim] fp32
+  void* pyr;                   // summaries: [units][unit_rows][head_dim], fp32 or bf16 bits
   long long units;
   long long unit_rows;         // rows per unit, all capacity-sized levels
   int Lcap;                    // levels for a full cache
@@ -57,6 +57,10 @@ struct zha_tree {
 };
 
 namespace zha {
+
+// Bytes of one stored summary element (desc.summary_dtype).
+inline int sum_bytes(const zha_tree* t) { return t->desc.summary_dtype == ZHA_BF16 ? 2 : 4; }
+inline bool sum_bf16(const zha_tree* t) { return t->desc.summary_dtype == ZHA_BF16; }
 
 // Levels above the leaves for n0 leaves: smallest L >= 1 with b^L >= n0 (0 if n0 == 0).
 int levels_for(long long n0, long long b);

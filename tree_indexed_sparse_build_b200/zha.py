@@ -35,7 +35,8 @@ EXPORTED = [
 class zha_tree_desc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("branching", ctypes.c_int), ("leaf_block", ctypes.c_int),
-                ("capacity_tokens", ctypes.c_longlong), ("kv_dtype", ctypes.c_int)]
+                ("capacity_tokens", ctypes.c_longlong), ("kv_dtype", ctypes.c_int),
+                ("summary_dtype", ctypes.c_int)]
 
 
 class ZhaError(RuntimeError):
@@ -289,9 +290,11 @@ class Tree:
     """A tree set over a [batch, kv_heads, capacity, head_dim] cache, with its workspace."""
 
     def __init__(self, batch: int, kv_heads: int, head_dim: int, branching: int,
-                 leaf_block: int, capacity: int, kv_dtype: torch.dtype, device="cuda"):
+                 leaf_block: int, capacity: int, kv_dtype: torch.dtype, device="cuda",
+                 summary_dtype: torch.dtype = torch.float32):
         self.desc = zha_tree_desc(batch, kv_heads, head_dim, branching, leaf_block, capacity,
-                                  dtype_code(kv_dtype))
+                                  dtype_code(kv_dtype), dtype_code(summary_dtype))
+        self.summary_dtype = summary_dtype
         nbytes = zha_tree_workspace_bytes(self.desc)
         if nbytes == 0:
             raise ZhaError(ZHA_ERR_UNSUPPORTED, "zha_tree_workspace_bytes")
@@ -332,11 +335,12 @@ class Tree:
         zha_tree_append(self.handle, K, new_seq_len, stream)
 
     def summaries(self) -> torch.Tensor:
-        """[units, unit_rows, head_dim] fp32 view of the workspace's summaries."""
+        """[units, unit_rows, head_dim] view of the workspace's summaries (summary_dtype)."""
         rows = zha_tree_unit_rows(self.handle)
         units = self.desc.batch * self.desc.kv_heads
         d = self.desc.head_dim
-        return self.workspace[256:256 + units * rows * d * 4].view(torch.float32).view(units, rows, d)
+        esz = 2 if self.summary_dtype == torch.bfloat16 else 4
+        return self.workspace[256:256 + units * rows * d * esz].view(self.summary_dtype).view(units, rows, d)
 
     def level_offset(self, level: int) -> int:
         """Row offset of a level inside each unit's summaries (and radii)."""
