@@ -59,10 +59,10 @@ def level_counts(N: int, lb: int, b: int) -> list[int]:
     return out
 
 
-def append_bytes(N_new: int, lb: int, b: int, d: int, kv_bytes: int, units: int) -> int:
+def append_bytes(N_new: int, lb: int, b: int, d: int, kv_bytes: int, units: int, sum_bytes: int = 4) -> int:
     """Algorithmic bytes of a one-leaf append that ends at N_new tokens: per unit, the
     touched leaf's tokens and, at every level above, the stored children of the path node
-    are read; the L + 1 path rows (fp32) are written."""
+    are read; the L + 1 path rows (sum_bytes an element) are written."""
     counts = level_counts(N_new, lb, b)
     L = len(counts) - 1
     leaf = (N_new - 1) // lb
@@ -70,8 +70,8 @@ def append_bytes(N_new: int, lb: int, b: int, d: int, kv_bytes: int, units: int)
     node = leaf
     for lvl in range(1, L + 1):
         node //= b
-        per_unit += (min(node * b + b, counts[lvl - 1]) - node * b) * d * 4
-    per_unit += (L + 1) * d * 4
+        per_unit += (min(node * b + b, counts[lvl - 1]) - node * b) * d * sum_bytes
+    per_unit += (L + 1) * d * sum_bytes
     return per_unit * units
 
 
@@ -84,11 +84,12 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def path_bytes(idx, trace, counts, N, lb, b, d, kv_bytes, g, out_bytes):
+def path_bytes(idx, trace, counts, N, lb, b, d, kv_bytes, g, out_bytes, sum_bytes=4):
     """Algorithmic bytes of one route call and one attend call, plus per-query counts.
 
-    Bytes are the union per (batch, KV head) of distinct summary rows scored (fp32) and
-    of distinct leaf-token K/V rows attended, plus Q in, indices and O out.
+    Bytes are the union per (batch, KV head) of distinct summary rows scored (sum_bytes an
+    element: 4 for fp32 summaries, 2 for bf16) and of distinct leaf-token K/V rows attended,
+    plus Q in, indices and O out.
     """
     B, Hq, nq, beam = idx.shape
     L = trace.shape[3]
@@ -119,7 +120,7 @@ def path_bytes(idx, trace, counts, N, lb, b, d, kv_bytes, g, out_bytes):
             u = np.unique(lv[valid])
             attend_tokens += int((np.minimum((u + 1) * lb, N) - u * lb).sum())
     q = B * Hq * nq
-    route_b = route_rows * d * 4 + q * d * kv_bytes + q * beam * 4
+    route_b = route_rows * d * sum_bytes + q * d * kv_bytes + q * beam * 4
     attend_b = attend_tokens * 2 * d * kv_bytes + q * d * kv_bytes + q * beam * 4 + q * d * out_bytes
     return {"route_bytes": int(route_b), "attend_bytes": int(attend_b),
             "summaries_per_query": float(np.concatenate(scored).mean()),
@@ -217,7 +218,8 @@ def _graph_events(n):
     return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
 
-def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="step"):
+def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="step", summary_dtype=None,
+               e2e=True):
     """128K decode steps: append 1 token + route + attend, one CUDA graph per step.
 
     mode "step": one zha_decode_step launch per step (append, route and attention fused);
@@ -231,6 +233,8 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     import torch
     from tree_indexed_sparse_build_b200 import ranks, synth, zha
 
+    summary_dtype = summary_dtype or torch.float32
+    sum_bytes = 2 if summary_dtype == torch.bfloat16 else 4
     N, cap = w.seq_len, w.seq_len + W + 2 * K
     w = w.with_(seed=ranks.rank_seed(w.seed, rank))
     Qs = np.stack([synth.queries(w, step=s) for s in range(W + 2 * K)])
@@ -238,7 +242,8 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     Vn = synth.values(w, capacity=cap)
     Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qs, dev)
     B, Hq, nq, d, beam = w.batch, w.q_heads, 1, w.head_dim, w.beam
-    tree = zha.Tree(B, w.kv_heads, d, w.branching, w.leaf_block, cap, torch.bfloat16)
+    tree = zha.Tree(B, w.kv_heads, d, w.branching, w.leaf_block, cap, torch.bfloat16,
+                    summary_dtype=summary_dtype)
     tree.build(Kd, N)
     scratch = tree.scratch_for(Hq, nq, beam, dev)
     idx = torch.empty((2 * K, B, Hq, nq, beam), dtype=torch.int32, device=dev)
@@ -341,15 +346,18 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
            "append_bytes": 0}
     for s in range(K, 2 * K):  # the kernel pass's calls, whose times the roofline uses
         Nst = N + W + s + 1
-        acc["append_bytes"] += append_bytes(Nst, w.leaf_block, w.branching, d, 2, w.units) / K
+        acc["append_bytes"] += append_bytes(Nst, w.leaf_block, w.branching, d, 2, w.units, sum_bytes) / K
         pb = path_bytes(idx_n[s], tr_n[s], level_counts(Nst, w.leaf_block, w.branching), Nst,
-                        w.leaf_block, w.branching, d, 2, w.group, 2)
+                        w.leaf_block, w.branching, d, 2, w.group, 2, sum_bytes=sum_bytes)
         for k in pb:
             acc[k] += pb[k] / K
     del graphs, graphs2
     res = {"step_ms": t_step, "append_ms": t_app, "decode_ms": t_dec,
            "queries_per_step": B * Hq * nq, "launches_per_step": launches, "clocks": smp.summary(),
            **acc}
+    if not e2e:
+        tree.close()
+        return res
 
     # End to end through the public API: per step, H2D of the new K/V rows and the query
     # from pinned memory, append + route + attend, D2H of the output, synchronize.
@@ -389,9 +397,10 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     return res
 
 
-def run_1m(W, K, rank, dev, flush, eager=False):
+def run_1m(W, K, rank, dev, flush, eager=False, summary_dtype=None):
     """1M-token cache, 8 KV heads: route + attend with 64 queries per head (throughput)
-    and with 1 query per head (single step)."""
+    and with 1 query per head (single step).  summary_dtype: the tree's summary storage
+    (fp32 by default; torch.bfloat16 halves the rows a route reads)."""
     import torch
     from tree_indexed_sparse_build_b200 import ranks, synth, workloads, zha
 
@@ -404,7 +413,10 @@ def run_1m(W, K, rank, dev, flush, eager=False):
     Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
     del Kn, Vn
     d, beam, N = w.head_dim, w.beam, w.seq_len
-    tree = zha.Tree(w.batch, w.kv_heads, d, w.branching, w.leaf_block, N, torch.bfloat16)
+    summary_dtype = summary_dtype or torch.float32
+    sum_bytes = 2 if summary_dtype == torch.bfloat16 else 4
+    tree = zha.Tree(w.batch, w.kv_heads, d, w.branching, w.leaf_block, N, torch.bfloat16,
+                    summary_dtype=summary_dtype)
     tree.build(Kd, N)
     torch.cuda.synchronize()
     counts = level_counts(N, w.leaf_block, w.branching)
@@ -458,7 +470,7 @@ def run_1m(W, K, rank, dev, flush, eager=False):
         tr_ms, at_ms = times[3][:, 0], times[3][:, 1]
         step_ms = times[2][:, 0]
         pb = path_bytes(idx.cpu().numpy(), tr.cpu().numpy(), counts, N, w.leaf_block,
-                        w.branching, d, 2, w.group, 2)
+                        w.branching, d, 2, w.group, 2, sum_bytes=sum_bytes)
         out[mode] = {"route_ms": tr_ms, "attend_ms": at_ms, "step_ms": step_ms,
                      "queries_per_step": w.batch * w.q_heads * nq, "launches_per_step": launches, **pb}
         del runs
@@ -862,8 +874,7 @@ def main():
         "clocks": r["clocks"],
     }
 
-    if not args.no_1m:
-        m = run_1m(W, K, rank, dev, flush, eager=args.eager)
+    def ctx_1m(m):
         one = {}
         for mode in ("throughput", "single"):
             x = m[mode]
@@ -882,7 +893,26 @@ def main():
         one["workload"] = ("deep_1m: 1 x 8 KV heads x 64 query heads, d 128, 1,048,576 bf16 tokens, "
                            "b 8, leaf block 4, beam 8; throughput = 64 queries per head per step")
         one["launches_per_step"] = {k: m[k]["launches_per_step"] for k in ("throughput", "single")}
-        line["ctx_1m"] = one
+        return one
+
+    # the same 128K decode steps over bf16-stored summaries (device-timed pass only)
+    rb = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager, mode=args.mode,
+                    summary_dtype=torch.bfloat16, e2e=False)
+    ms_b = max_over_ranks(float(rb["step_ms"].mean()))
+    dec_b = rb["route_bytes"] + rb["attend_bytes"] + (rb["append_bytes"] if fused_append else 0)
+    line["decode_128k_bf16_summaries"] = {
+        "qps": ranks.weak_scaling_rate(rb["queries_per_step"], world, ms_b), "ms_per_step": ms_b,
+        "decode_kernel_ms": float(rb["decode_ms"].mean()),
+        "decode_kernel_gbs": dec_b / (float(rb["decode_ms"].mean()) * 1e-3) / 1e9,
+        "decode_kernel_bytes": int(dec_b), "route_bytes": int(rb["route_bytes"]),
+        "summaries_per_query": rb["summaries_per_query"], "clocks": rb["clocks"]}
+
+    if not args.no_1m:
+        line["ctx_1m"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager))
+        # the same step over bf16-stored summaries (half the route's bytes; routing then
+        # follows the bf16 tree, so the leaf sets may differ from the fp32 tree's)
+        line["ctx_1m_bf16_summaries"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager,
+                                                      summary_dtype=torch.bfloat16))
 
     if not args.no_build and rank == 0:
         line["build_256k"] = run_build_256k(W, K, dev, flush)

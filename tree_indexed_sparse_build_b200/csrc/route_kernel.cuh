@@ -111,6 +111,13 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   }
   const long long* nl = PREFIX ? reinterpret_cast<const long long*>(pb + Ps.qn) : a.n;
   const int Lq = PREFIX ? (int)nl[kMaxLevels - 1] : a.L;
+  // A level with at most `beam` nodes is kept whole once every node above it is: starting
+  // from the root, such levels need no scoring, and routing begins at the highest level
+  // l_first >= 1 with more than `beam` nodes (else at the leaves), from every node of the
+  // level above it.  The leaves are always scored (their scores are an output).
+  int l_first = Lq - 1;
+  while (l_first >= 1 && nl[l_first] <= a.beam) --l_first;
+  const int m_first = (int)nl[l_first + 1];
   if (wq == 0 && lane == 0) {
     mbar_init(&bar[0], 1);
     if (ATTEND)
@@ -120,7 +127,6 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
     if (HASPATH) mbar_init(pbar, 1);
     fence_mbar_init();
-    surv_a[0] = 0;  // the root
     if constexpr (HASPATH) {
       if (live) {
         fence_proxy_async_smem();
@@ -131,6 +137,14 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
     }
   }
+  if (wq == 0) {
+    for (int k = lane; k < m_first; k += 32) surv_a[k] = k;  // every node of level l_first + 1
+    if (a.trace && valid)
+      for (int l = l_first + 1; l < Lq; ++l) {  // the levels kept whole: all their nodes
+        int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
+        for (int k = lane; k < a.beam; k += 32) tr[k] = (live && k < nl[l]) ? k : -1;
+      }
+  }
   qsync();
 
   // Four lanes per row: lane (rg = lane / 4, sub = lane % 4) reads chunks 4 (j ^ par) + sub,
@@ -139,9 +153,9 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   float qv[CPL][EPC];
   int* cur = surv_a;
   int* nxt = surv_b;
-  int m = live ? 1 : 0;
+  int m = live ? m_first : 0;
   uint32_t parity = 0;
-  for (int l = Lq - 1; l >= 0; --l) {
+  for (int l = l_first; l >= 0; --l) {
     int C = 0;
     if (m > 0) {
       const long long last = cur[m - 1];
@@ -177,7 +191,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
       if (lane == 0) kpos[0] = found < 0 ? -1 : (int)(found * a.b + (node[l] - a.b * node[l + 1]));
     }
-    if (l == Lq - 1 && valid) {  // load q while the first level is in flight
+    if (l == l_first && valid) {  // load q while the first level is in flight
       const long long qo = qg * D;
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
@@ -188,7 +202,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
                               : static_cast<const float*>(a.Q)[qo + EPC * c + e];
       }
     }
-    if (HASPATH && l == Lq - 1) {
+    if (HASPATH && l == l_first) {
       // the path rows, while the first level's copies are in flight
       const bool pok = !live || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
       const bool pfail = GROUPED ? group_any(bar_id, bar_n, !pok) : __any_sync(0xffffffffu, !pok);
