@@ -216,6 +216,27 @@ zha_status zha_decode_causal(const zha_tree* tree, const void* d_Q, zha_dtype q_
                              float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
                              zha_dtype o_dtype, void* stream);
 
+/* Decode with an append buffer ("Louver" explainer, dynamic updates: keys produced during
+ * decoding wait in a small buffer that every query reads directly, and a full buffer is
+ * merged into the index in the background, concurrently with the attention).  Each query
+ * routes over the tree of the first n_routed tokens (the prefix of zha_route_causal at
+ * position n_routed - 1) and attends, exactly, over the tokens of its leaves together with
+ * every buffered token n_routed .. n_tokens - 1 of the cache; O as in zha_decode.
+ *   n_routed   a multiple of the leaf block, 1 <= n_routed <= zha_tree_seq_len: the tree
+ *              must summarise the first n_routed tokens, through calls ordered before this
+ *              one on `stream`
+ *   n_tokens   n_routed <= n_tokens <= capacity; tokens n_routed .. n_tokens - 1 of d_K and
+ *              d_V written by the caller before the call
+ * The call reads no summary that an append of tokens at or after n_routed writes, so the
+ * caller may commit the buffer (zha_tree_append to n_tokens) on another stream while it
+ * keeps decoding with the old n_routed, and switch n_routed once that append has completed.
+ * d_leaf_idx / d_leaf_score / d_trace describe the routed leaves only (as in
+ * zha_route_causal).  ZHA_ERR_UNSUPPORTED when the shape does not fit the fused kernel. */
+zha_status zha_decode_buffered(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                               int beam, const void* d_K, const void* d_V, long long n_routed,
+                               long long n_tokens, float scale, int* d_leaf_idx, float* d_leaf_score,
+                               int* d_trace, void* d_O, zha_dtype o_dtype, void* stream);
+
 /* Bounding spheres for threshold descent ("Louver" explainer: every cluster of keys is
  * enclosed in a sphere, a center and a radius).  The center of a node is its summary; the
  * radius covers every key of its subtree (leaf: its farthest token; node: its farthest

@@ -298,6 +298,22 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int, leaf_block: int,
     return out, int(ntok)
 
 
+def buffer_leaves(n_routed: int, n_tokens: int, lb: int) -> np.ndarray:
+    """Leaves holding the buffered tokens n_routed .. n_tokens - 1 (n_routed a multiple of lb)."""
+    return np.arange(n_routed // lb, -(-n_tokens // lb), dtype=np.int64)
+
+
+def attend_buffered(q: np.ndarray, K: np.ndarray, V: np.ndarray, leaves: np.ndarray, n_routed: int,
+                    n_tokens: int, lb: int, scale: float) -> tuple[np.ndarray, int]:
+    """Decode with an append buffer ("Louver" explainer, dynamic updates: keys that arrive during
+    decoding wait in a buffer the queries read directly): exact softmax attention over the
+    tokens of the routed leaves (a route over the tree of the first n_routed tokens, so all of
+    them lie before n_routed) together with every buffered token n_routed .. n_tokens - 1."""
+    lv = np.asarray(leaves, dtype=np.int64).ravel()
+    lv = lv[lv >= 0]
+    return attend(q, K, V, n_tokens, lb, np.concatenate([lv, buffer_leaves(n_routed, n_tokens, lb)]), scale)
+
+
 def dense(q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int, scale: float) -> np.ndarray:
     """Exact softmax attention of one query over all tokens t < N."""
     q = np.ascontiguousarray(q, dtype=np.float64).ravel()

@@ -81,6 +81,8 @@ def test_calls_reject_null_tree_on_host():
         zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_decode_causal(None, None, 1, 8, 1, None, 4, None, None, ctypes.c_float(0.1), None,
                                  None, None, None, 1, None) == zha.ZHA_ERR_INVALID_ARG
+    assert lib.zha_decode_buffered(None, None, 1, 8, 1, 4, None, None, 16, 16, ctypes.c_float(0.1), None,
+                                   None, None, None, 1, None) == zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_tree_attach_radii(None, None, 0, None, None) == zha.ZHA_ERR_INVALID_ARG
     assert lib.zha_tree_radii_bytes(None) == 0
     assert lib.zha_threshold_route(None, None, None, 1, 8, 1, None, 16, None, None, None, None) == \

@@ -296,6 +296,43 @@ def test_single_token_attention_is_its_value():
     np.testing.assert_array_equal(o, V[leaves[0]].astype(np.float64))
 
 
+# ---------------------------------------------------------------- append buffer
+
+def test_buffered_attention_over_one_routed_leaf_and_the_rest_is_dense():
+    # routed prefix = the first leaf (one leaf, kept whatever the query), buffer = every
+    # later token: the union is the whole cache, so the result is a library softmax over all
+    rng = np.random.default_rng(21)
+    d, lb, N = 8, 4, 203
+    K = _f32(rng.standard_normal((N, d)))
+    V = _f32(rng.standard_normal((N, d)))
+    q = rng.standard_normal(d)
+    t = oracle.OracleTree(d, lb, 2).build(K, lb)
+    leaves = t.route(q[None], 1)["leaves"][0]
+    np.testing.assert_array_equal(leaves, [0])
+    o, ntok = oracle.attend_buffered(q, K, V, leaves, lb, N, lb, 0.3)
+    assert ntok == N
+    w = softmax(0.3 * (K.astype(np.float64) @ q))
+    np.testing.assert_allclose(o, w @ V.astype(np.float64), rtol=1e-12, atol=1e-14)
+
+
+def test_buffered_attention_is_the_union_of_leaf_and_buffer_tokens():
+    rng = np.random.default_rng(22)
+    d, lb, b, n_routed, n_tokens = 6, 5, 3, 400, 437
+    K = _f32(rng.standard_normal((n_tokens, d)))
+    V = _f32(rng.standard_normal((n_tokens, d)))
+    q = rng.standard_normal(d)
+    t = oracle.OracleTree(d, lb, b).build(K, n_routed)
+    leaves = t.route(q[None], 4)["leaves"][0]
+    o, ntok = oracle.attend_buffered(q, K, V, leaves, n_routed, n_tokens, lb, 0.5)
+    tok = np.concatenate([np.arange(l * lb, l * lb + lb) for l in leaves] + [np.arange(n_routed, n_tokens)])
+    assert ntok == len(tok) == 4 * lb + 37
+    w = softmax(0.5 * (K[tok].astype(np.float64) @ q))
+    np.testing.assert_allclose(o, w @ V[tok].astype(np.float64), rtol=1e-12, atol=1e-14)
+    # an empty buffer is the plain attention over the routed leaves
+    o0, _ = oracle.attend_buffered(q, K, V, leaves, n_routed, n_routed, lb, 0.5)
+    np.testing.assert_array_equal(o0, oracle.attend(q, K, V, n_routed, lb, leaves, 0.5)[0])
+
+
 @pytest.mark.parametrize("lb,b,N", [(16, 2, 1024), (4, 8, 40000), (64, 8, 32768)])
 def test_needle_on_quiet_background_is_retrieved(lb, b, N):
     rng = np.random.default_rng(8)

@@ -25,11 +25,13 @@ __device__ __forceinline__ int leaf_tokens(const int* leaves, int m, long long l
 
 // Stage st covers tokens [st TS, min(st TS + TS, total)) and goes to buffer st % nbuf of
 // sb, completing on bars[st % nbuf].  Called by all lanes of one warp; each lane copies the
-// K and V pieces of some of the stage's leaves.
+// K and V pieces of some of the stage's leaves.  Token slot j lb .. j lb + lb - 1 belongs to
+// leaf leaves[j] for j < m and to leaf buf_leaf0 + (j - m) after them (an append buffer:
+// consecutive leaves after the routed ones, the last one possibly partial).
 template <int ROWB>
-__device__ __forceinline__ void attn_issue_stage(const int* leaves, int lb, int total, int TS, int st,
-                                                 int nbuf, unsigned char* sb, const char* Ku,
-                                                 const char* Vu, uint64_t* bars, int lane) {
+__device__ __forceinline__ void attn_issue_stage(const int* leaves, int m, long long buf_leaf0, int lb,
+                                                 int total, int TS, int st, int nbuf, unsigned char* sb,
+                                                 const char* Ku, const char* Vu, uint64_t* bars, int lane) {
   const size_t stage_bytes = (size_t)TS * ROWB;
   const int b = st % nbuf;
   unsigned char* kb = sb + (size_t)b * 2 * stage_bytes;
@@ -40,7 +42,8 @@ __device__ __forceinline__ void attn_issue_stage(const int* leaves, int lb, int 
   for (int j = w0 / lb + lane; j <= (w1 - 1) / lb; j += 32) {
     const int p0 = j * lb;
     const int a0 = max(p0, w0), a1 = min(p0 + lb, w1);
-    const long long row = (long long)leaves[j] * lb + (a0 - p0);
+    const long long leaf = j < m ? (long long)leaves[j] : buf_leaf0 + (j - m);
+    const long long row = leaf * lb + (a0 - p0);
     const uint32_t bytes = (uint32_t)((a1 - a0) * ROWB);
     bulk_copy_g2s(kb + (size_t)(a0 - w0) * ROWB, Ku + row * ROWB, bytes, &bars[b]);
     bulk_copy_g2s(kb + stage_bytes + (size_t)(a0 - w0) * ROWB, Vu + row * ROWB, bytes, &bars[b]);
@@ -50,8 +53,10 @@ __device__ __forceinline__ void attn_issue_stage(const int* leaves, int lb, int 
 // Where the attention of one query runs and what it reads.
 struct StagedAttn {
   const int* leaves;     // shared memory, ascending
+  int m;                 // routed leaves
+  long long buf_leaf0;   // first leaf of the append buffer's tokens (slots m, m + 1, ..)
   int lb;                // tokens per leaf
-  int total;             // tokens (leaf_tokens)
+  int total;             // tokens (leaf_tokens, plus the buffer's)
   int TS;                // tokens per stage buffer, a multiple of 16
   int nbuf;              // stage buffers, 2 or 3
   unsigned char* sb;     // the stage buffers; >= nw * D * 4 bytes (warp merge reuses them)
@@ -118,7 +123,7 @@ __device__ bool attend_staged(const StagedAttn& s, long long qg, bool valid,
                              s.wait_cycles);
       __syncwarp();
       if (ok) {
-        attn_issue_stage<ROWB>(s.leaves, s.lb, s.total, s.TS, st + s.nbuf, s.nbuf, s.sb, s.Ku, s.Vu,
+        attn_issue_stage<ROWB>(s.leaves, s.m, s.buf_leaf0, s.lb, s.total, s.TS, st + s.nbuf, s.nbuf, s.sb, s.Ku, s.Vu,
                                s.bars, lane);
         issued = st + s.nbuf + 1;
       }

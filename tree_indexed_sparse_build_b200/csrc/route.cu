@@ -234,19 +234,54 @@ RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int 
   return a;
 }
 
-// Warps per query in narrow launches: enough that each warp scores about 16 rows of the
-// widest level (at most 4).
+// Narrow launches: CTAs of at most 8 warps, three resident per SM (the NARROW kernels'
+// register cap), in the 228 KB of shared memory an SM holds (1 KB of it reserved per CTA).
+// Each level of a route is one memory round trip, so throughput follows the number of
+// queries resident per SM: the launch takes the warps per query (4, 2 or 1; at most enough
+// that each warp scores about 16 rows of the widest level) and queries per CTA that keep
+// the most queries resident, preferring more warps per query, then fewer queries per CTA.
+constexpr int kNarrowMaxWpq = 4;
+constexpr int kNarrowCtasPerSm = 3;
+constexpr size_t kSmSmem = 228 * 1024, kCtaReserved = 1024;
 #ifndef ZHA_NARROW_WPQ
-#define ZHA_NARROW_WPQ 0  // 0: by the widest level; else a fixed count (1, 2 or 4)
+#define ZHA_NARROW_WPQ 0  // 0: by the rule above; else a fixed count (1, 2 or 4)
 #endif
-int narrow_wpq(long long cmax) {
+int narrow_qpc(int wpq, size_t per_query, long long* resident = nullptr) {
+  int best = 1;
+  long long best_r = -1;
+  for (int q = 1; q <= 8 / wpq; ++q) {
+    const size_t cta = (size_t)q * per_query;
+    if (cta > kCtaSmemCap) break;
+    const long long r = (long long)q * std::min<long long>(kNarrowCtasPerSm, kSmSmem / (cta + kCtaReserved));
+    if (r > best_r) {
+      best_r = r;
+      best = q;
+    }
+  }
+  if (resident) *resident = best_r;
+  return best;
+}
+int narrow_wpq(long long cmax, size_t per_query) {
   if (ZHA_NARROW_WPQ > 0) return ZHA_NARROW_WPQ;
-  return (int)std::min<long long>(4, std::max<long long>(1, (cmax + 15) / 16));
+  const int want = (int)std::min<long long>(kNarrowMaxWpq, std::max<long long>(1, (cmax + 15) / 16));
+  int best = want;
+  long long best_r;
+  narrow_qpc(want, per_query, &best_r);
+  for (int w = want / 2; w >= 1; w /= 2) {
+    long long r;
+    narrow_qpc(w, per_query, &r);
+    if (r > best_r) {
+      best_r = r;
+      best = w;
+    }
+  }
+  return best;
 }
 
 // Launch shape of the staged kernel.  Wide (at most two queries per SM): one query per
 // CTA, enough warps for the widest level (and, fused, for the attention tokens).
-// Narrow: up to 8 warps per CTA, narrow_wpq warps per query.
+// Narrow: up to 8 warps per CTA, narrow_wpq warps per query, narrow_qpc queries per CTA
+// (per_query sized with the per-warp weight area of kNarrowMaxWpq warps).
 struct StagedShape {
   bool wide, grouped;
   unsigned blocks;
@@ -263,8 +298,8 @@ StagedShape staged_shape(const zha_tree* t, RouteArgs& a, size_t per_query, int 
     sh.blocks = (unsigned)a.total_queries;
     sh.smem = per_query;
   } else {
-    a.wpq = narrow_wpq(a.cmax);
-    a.qpc = (int)std::max<size_t>(1, std::min<size_t>(8 / a.wpq, (96 * 1024) / per_query));
+    a.wpq = narrow_wpq(a.cmax, per_query);
+    a.qpc = narrow_qpc(a.wpq, per_query);
     sh.blocks = (unsigned)((a.total_queries + a.qpc - 1) / a.qpc);
     sh.smem = per_query * a.qpc;
   }
@@ -346,7 +381,7 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
     p.rows_bytes = std::max(route_rows, (size_t)4 * 16 * row);  // two stages of 16 tokens at least
     p.stage_tokens = (int)(p.rows_bytes / (4 * row)) / 16 * 16;
     p.attn_warps = 1;
-    p.smem_per_query = route_smem_layout(D, (int)cmax, beam, p.rows_bytes, narrow_wpq(cmax)).total;
+    p.smem_per_query = route_smem_layout(D, (int)cmax, beam, p.rows_bytes, kNarrowMaxWpq).total;
     p.fused = p.smem_per_query <= kRouteSmemCap && p.stage_tokens >= 16 && 2LL * p.stage_tokens >= tokens;
     return p;
   }
@@ -406,7 +441,8 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
 cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
                           const long long* d_positions, const void* d_K, const void* d_V, float scale,
                           int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
-                          zha_dtype o_dtype, cudaStream_t stream, bool* unsupported) {
+                          zha_dtype o_dtype, cudaStream_t stream, bool* unsupported, long long prefix_pos,
+                          int buf_tokens) {
   *unsupported = false;
   RouteArgs a = route_args(t, d_Q, q_dtype, q_heads, nq, beam, d_leaf_idx, d_leaf_score, d_trace);
   const int D = t->desc.head_dim;
@@ -425,7 +461,7 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
     nbuf = dp.nbuf;
     stage_tokens = dp.stage_tokens;
     if (!wide) {
-      const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
+      const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N) + buf_tokens;
       rows = std::max(rows, std::min((size_t)2 * row * (size_t)tokens, (size_t)64 * 1024));
       stage_tokens = (int)(rows / (4 * row)) / 16 * 16;
     }
@@ -442,7 +478,10 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
   a.O = d_O;
   a.o_bf16 = o_dtype == ZHA_BF16;
   a.positions = d_positions;
-  const int pw_warps = wide ? kRouteMaxWarps : narrow_wpq(a.cmax);
+  a.prefix_pos = prefix_pos;
+  a.buf_leaf0 = (prefix_pos + 1) / t->desc.leaf_block;
+  a.buf_tokens = buf_tokens;
+  const int pw_warps = wide ? kRouteMaxWarps : kNarrowMaxWpq;
   const size_t route_part = route_smem_layout(D, a.cmax, beam, (size_t)a.rows_bytes, pw_warps).total;
   const size_t path_bytes = path_smem_layout(D, row, sum_bytes(t), (int)a.lb, a.b, t->L).total;
   a.path_smem_off = (long long)route_align(route_part, 128);

@@ -49,8 +49,14 @@ struct RouteArgs {
   long long path_leaf;       // the leaf that received the new tokens
   int path_tokens;           // its tokens after the append
   long long path_smem_off;   // byte offset of the path region in a query's shared memory
-  // causal routing (kPathPrefix): query qg routes over tokens 0 .. positions[qg % nq]
+  // causal routing (kPathPrefix): query qg routes over tokens 0 .. positions[qg % nq], or
+  // over tokens 0 .. prefix_pos when positions is null
   const long long* positions;
+  long long prefix_pos;
+  // append buffer: the attention also covers buf_tokens tokens from leaf buf_leaf0 on (the
+  // tokens after the routed prefix, which then ends on a leaf boundary)
+  long long buf_leaf0;
+  int buf_tokens;
 };
 
 struct NoKV {};  // route only: no attention epilogue

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   long long Nq = a.N;
   bool live = valid;  // a query with a position outside the tree routes nowhere
   if constexpr (PREFIX) {
-    const long long pos = valid ? a.positions[qg % a.nq] : 0;
+    const long long pos = !valid ? 0 : a.positions ? a.positions[qg % a.nq] : a.prefix_pos;
     if (valid && (pos < 0 || pos >= a.N)) {
       if (wq == 0 && lane == 0) atomicOr(a.err, kDevErrBadLeaf);
       live = false;
@@ -278,7 +278,10 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
     }
     qsync();
-    if (C > 0 && C <= 128 && C <= 64 * nw) {  // C is the same for the whole group
+    // C is the same for the whole group.  Up to 64 candidates: one warp's register selection
+    // (no shared-memory ranks, no group barriers inside); up to 128: ranks over the group;
+    // wider: the group's radix selection, or one warp's register selection.
+    if (C > 64 && C <= 128 && C <= 64 * nw) {
       const int kept =
           select_rank_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red, wq, lane, nw, bar_id);
       qsync();
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;
         for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
       }
-    } else if (GROUPED && C <= 32 * nw) {  // radix selection over the group
+    } else if (GROUPED && C > 64 && C <= 32 * nw) {  // radix selection over the group
       const int kept = select_radix_group(keys, cand, C, a.beam, nxt, leaf_sc, l == 0, red,
                                           reinterpret_cast<unsigned*>(base + Ls.hist), wq, lane, nw, bar_id);
       group_sync(bar_id, bar_n);
@@ -328,8 +331,10 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     using S = AttnShape<TKV, D>;
     StagedAttn sa;
     sa.leaves = cur;
+    sa.m = m;
+    sa.buf_leaf0 = a.buf_leaf0;
     sa.lb = (int)a.lb;
-    sa.total = leaf_tokens(cur, m, a.lb, Nq);
+    sa.total = leaf_tokens(cur, m, a.lb, Nq) + (live ? a.buf_tokens : 0);
     sa.TS = a.stage_tokens;
     sa.nbuf = a.attn_nbuf;
     sa.sb = base + Ls.rows;  // the candidate rows (and the append path) are no longer needed
@@ -346,7 +351,8 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     const int nst = (sa.total + sa.TS - 1) / sa.TS;
     if (wq == 0)
       for (int st = 0; st < min(nst, sa.nbuf); ++st)
-        attn_issue_stage<S::ROWB>(cur, sa.lb, sa.total, sa.TS, st, sa.nbuf, sa.sb, sa.Ku, sa.Vu, bar, lane);
+        attn_issue_stage<S::ROWB>(cur, m, sa.buf_leaf0, sa.lb, sa.total, sa.TS, st, sa.nbuf, sa.sb, sa.Ku, sa.Vu,
+                                  bar, lane);
     float qa[S::CPL][S::VEC];
     if (valid) attn_load_q<TKV, D>(a.Q, a.q_bf16 != 0, qg, lane, qa);
     float* pw = reinterpret_cast<float*>(base + Ls.pw) + wq * 16;

@@ -248,10 +248,13 @@ zha_status zha_decode_step(zha_tree* t, const void* d_K, const void* d_V, long l
                     d_trace, d_O, o_dtype, stream);
 }
 
+// d_positions null: every query at position prefix_pos, with buf_tokens buffered tokens
+// after it attended as well (zha_decode_buffered).
 static zha_status causal_call(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
                               const long long* d_positions, int beam, const void* d_K, const void* d_V,
                               float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
-                              zha_dtype o_dtype, void* stream) {
+                              zha_dtype o_dtype, void* stream, long long prefix_pos = -1,
+                              int buf_tokens = 0) {
   if (!t || !dtype_ok(q_dtype) || !dtype_ok(o_dtype) || q_heads < 1 || nq < 0) return ZHA_ERR_INVALID_ARG;
   if (q_heads % t->desc.kv_heads != 0) return ZHA_ERR_INVALID_ARG;
   if (beam < 1 || beam > kMaxBeam) return ZHA_ERR_INVALID_ARG;
@@ -259,7 +262,8 @@ static zha_status causal_call(const zha_tree* t, const void* d_Q, zha_dtype q_dt
   if (t->N == 0) return ZHA_ERR_INVALID_ARG;
   if (d_O && !(scale == scale)) return ZHA_ERR_INVALID_ARG;
   if (nq == 0) return ZHA_OK;
-  if (!d_Q || !d_K || !d_positions || !d_leaf_idx || (d_O && !d_V)) return ZHA_ERR_INVALID_ARG;
+  if (!d_Q || !d_K || (!d_positions && prefix_pos < 0) || !d_leaf_idx || (d_O && !d_V))
+    return ZHA_ERR_INVALID_ARG;
   if (!aligned(d_Q, 16) || !aligned(d_K, 16) || !aligned(d_positions, 8) || !aligned(d_leaf_idx, 4) ||
       (d_O && (!aligned(d_O, 16) || !aligned(d_V, 16))) || (d_leaf_score && !aligned(d_leaf_score, 4)) ||
       (d_trace && !aligned(d_trace, 4)))
@@ -267,7 +271,7 @@ static zha_status causal_call(const zha_tree* t, const void* d_Q, zha_dtype q_dt
   bool unsupported = false;
   const cudaError_t e = launch_causal(const_cast<zha_tree*>(t), d_Q, q_dtype, q_heads, nq, beam, d_positions,
                                       d_K, d_V, scale, d_leaf_idx, d_leaf_score, d_trace, d_O, o_dtype,
-                                      static_cast<cudaStream_t>(stream), &unsupported);
+                                      static_cast<cudaStream_t>(stream), &unsupported, prefix_pos, buf_tokens);
   if (unsupported) return ZHA_ERR_UNSUPPORTED;
   return cuda_status(e);
 }
@@ -286,6 +290,20 @@ zha_status zha_decode_causal(const zha_tree* t, const void* d_Q, zha_dtype q_dty
   if (!d_O) return ZHA_ERR_INVALID_ARG;
   return causal_call(t, d_Q, q_dtype, q_heads, nq, d_positions, beam, d_K, d_V, scale, d_leaf_idx,
                      d_leaf_score, d_trace, d_O, o_dtype, stream);
+}
+
+zha_status zha_decode_buffered(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq,
+                               int beam, const void* d_K, const void* d_V, long long n_routed,
+                               long long n_tokens, float scale, int* d_leaf_idx, float* d_leaf_score,
+                               int* d_trace, void* d_O, zha_dtype o_dtype, void* stream) {
+  if (!t || !d_O) return ZHA_ERR_INVALID_ARG;
+  const long long lb = t->desc.leaf_block;
+  if (n_routed < 1 || n_routed % lb != 0 || n_routed > t->N) return ZHA_ERR_INVALID_ARG;
+  if (n_tokens < n_routed) return ZHA_ERR_INVALID_ARG;
+  if (n_tokens > t->desc.capacity_tokens) return ZHA_ERR_CAPACITY;
+  if (n_tokens - n_routed > (1LL << 30)) return ZHA_ERR_UNSUPPORTED;
+  return causal_call(t, d_Q, q_dtype, q_heads, nq, nullptr, beam, d_K, d_V, scale, d_leaf_idx, d_leaf_score,
+                     d_trace, d_O, o_dtype, stream, n_routed - 1, (int)(n_tokens - n_routed));
 }
 
 size_t zha_tree_radii_bytes(const zha_tree* t) {

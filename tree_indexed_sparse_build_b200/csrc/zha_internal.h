@@ -98,12 +98,15 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
                           long long append_leaf = -1);
 
 // Causal routing (route.cu): query qg of every head routes over the tree of tokens
-// 0 .. positions[qg % nq], and attends over its leaves' tokens in that prefix when d_O is
-// given.  *unsupported: the shape does not fit the staged kernel (nothing launched).
+// 0 .. positions[qg % nq] (0 .. prefix_pos for every query when d_positions is null), and
+// attends over its leaves' tokens in that prefix when d_O is given -- and over the
+// buf_tokens tokens after the prefix (an append buffer; prefix_pos + 1 a multiple of the
+// leaf block).  *unsupported: the shape does not fit the staged kernel (nothing launched).
 cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
                           const long long* d_positions, const void* d_K, const void* d_V, float scale,
                           int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
-                          zha_dtype o_dtype, cudaStream_t stream, bool* unsupported);
+                          zha_dtype o_dtype, cudaStream_t stream, bool* unsupported,
+                          long long prefix_pos = -1, int buf_tokens = 0);
 
 // Bounding-sphere radii (radii.cu): recompute leaves [lo, hi] of every unit and all their
 // ancestors (no-op without radii attached).

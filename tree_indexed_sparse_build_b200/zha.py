@@ -28,7 +28,7 @@ EXPORTED = [
     "zha_tree_level_offset", "zha_tree_unit_rows", "zha_tree_summaries", "zha_tree_launch_count",
     "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
     "zha_decode", "zha_decode_step", "zha_route_causal", "zha_decode_causal",
-    "zha_tree_radii_bytes", "zha_tree_attach_radii", "zha_threshold_route",
+    "zha_tree_radii_bytes", "zha_tree_attach_radii", "zha_threshold_route", "zha_decode_buffered",
 ]
 
 
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "zha_threshold_route": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P]),
             "zha_decode_causal": (_I, [_P, _P, _I, _I, _I, _P, _I, _P, _P, ctypes.c_float, _P, _P, _P,
                                        _P, _I, _P]),
+            "zha_decode_buffered": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _LL, _LL, ctypes.c_float, _P, _P,
+                                         _P, _P, _I, _P]),
             "zha_tree_check": (_I, [_P, _P]),
             "zha_tree_seq_len": (_LL, [_P]),
             "zha_tree_levels": (_I, [_P]),
@@ -231,6 +233,18 @@ def zha_decode_causal(handle, Q: torch.Tensor, positions: torch.Tensor, beam: in
     _check(lib().zha_decode_causal(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions), beam,
                                    _ptr(K), _ptr(V), scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
                                    _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_causal")
+
+
+def zha_decode_buffered(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: torch.Tensor, n_routed: int,
+                        n_tokens: int, scale: float, leaf_idx: torch.Tensor, O: torch.Tensor,
+                        leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
+                        stream=None) -> None:
+    """Route over the tree of the first n_routed tokens, attend over the routed leaves and the
+    buffered tokens n_routed .. n_tokens - 1, one launch."""
+    B, Hq, nq, _ = Q.shape
+    _check(lib().zha_decode_buffered(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
+                                     n_routed, n_tokens, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
+                                     _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_buffered")
 
 
 def zha_tree_radii_bytes(handle) -> int:
@@ -434,6 +448,18 @@ class Tree:
         O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
         zha_decode_causal(self.handle, Q, positions, beam, K, V, scale, idx, O, None, None, stream)
         return O, idx
+
+    def decode_buffered(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, n_routed: int, n_tokens: int,
+                        beam: int, scale: float, out_dtype: torch.dtype = torch.bfloat16, trace: bool = False,
+                        stream=None):
+        """Decode with an append buffer; returns (O, leaf_idx) or (O, leaf_idx, trace)."""
+        B, Hq, nq, d = Q.shape
+        idx = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=Q.device)
+        O = torch.empty((B, Hq, nq, d), dtype=out_dtype, device=Q.device)
+        tr = (torch.empty((B, Hq, nq, self.levels, beam), dtype=torch.int32, device=Q.device)
+              if trace else None)
+        zha_decode_buffered(self.handle, Q, beam, K, V, n_routed, n_tokens, scale, idx, O, None, tr, stream)
+        return (O, idx, tr) if trace else (O, idx)
 
     def attach_radii(self, K: torch.Tensor | None, stream=None) -> torch.Tensor:
         """Allocate and attach the bounding-sphere radii; returns them ([units, unit_rows])."""
