@@ -397,6 +397,73 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     return res
 
 
+def run_buffered(w, W, K, rank, dev, flush, buf_leaves=2):
+    """128K decode steps with an append buffer: each step writes one token into the buffer
+    (tokens after the committed prefix) and runs zha_decode_buffered; when buf_leaves full
+    leaves have accumulated, the step also commits them (zha_tree_append on a second stream,
+    forked from the step and joined at its end, so the commit overlaps that step's decode).
+    One CUDA graph per step, start and end events on the decode stream around the fork and
+    the join; L2 flushed between steps."""
+    import torch
+    from tree_indexed_sparse_build_b200 import ranks, synth, zha
+
+    lb = w.leaf_block
+    N, cap = w.seq_len, w.seq_len + W + K
+    w = w.with_(seed=ranks.rank_seed(w.seed, rank))
+    Qs = np.stack([synth.queries(w, step=s) for s in range(W + K)])
+    Kd = synth.to_torch(synth.keys(w, capacity=cap), dev)
+    Vd = synth.to_torch(synth.values(w, capacity=cap), dev)
+    Qd = synth.to_torch(Qs, dev)
+    B, Hq, d, beam = w.batch, w.q_heads, w.head_dim, w.beam
+    tree = zha.Tree(B, w.kv_heads, d, w.branching, lb, cap, torch.bfloat16)
+    tree.build(Kd, N)
+    torch.cuda.synchronize()
+    O = torch.empty((W + K, B, Hq, 1, d), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((W + K, B, Hq, 1, beam), dtype=torch.int32, device=dev)
+    main, side = torch.cuda.Stream(), torch.cuda.Stream()
+    plan, n_routed, commits = [], N, 0
+    for s in range(W + K):  # (tokens after this step's write, routed prefix, commit target or None)
+        n_tok = N + s + 1
+        full = (n_tok - n_routed) // lb
+        target = n_routed + buf_leaves * lb if full >= buf_leaves else None
+        plan.append((n_tok, n_routed, target))
+        if target is not None:
+            n_routed = target
+    graphs, evs = [], []
+    l0 = tree.launches
+    for s, (n_tok, nr, target) in enumerate(plan):
+        e = _graph_events(2)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=main, capture_error_mode="thread_local"):
+            e[0].record()
+            if target is not None:
+                side.wait_stream(main)
+                zha.zha_tree_append(tree.handle, Kd, target, side)
+            zha.zha_decode_buffered(tree.handle, Qd[s], beam, Kd, Vd, nr, n_tok, w.scale, idx[s], O[s],
+                                    None, None, main)
+            if target is not None:
+                main.wait_stream(side)
+            e[1].record()
+        graphs.append(g)
+        evs.append(e)
+    launches = (tree.launches - l0) / len(plan)
+    for s in range(W):
+        graphs[s].replay()
+    torch.cuda.synchronize()
+    for s in range(W, W + K):
+        flush.zero_()
+        graphs[s].replay()
+    torch.cuda.synchronize()
+    assert tree.check() == zha.ZHA_OK, "device error word set during the buffered steps"
+    t = np.array([evs[s][0].elapsed_time(evs[s][1]) for s in range(W, W + K)])
+    commits = sum(1 for s in range(W, W + K) if plan[s][2] is not None)
+    tree.close()
+    return {"ms_per_step": float(t.mean()), "qps": B * Hq / (t.mean() * 1e-3),
+            "commit_step_ms": float(np.mean([t[i] for i in range(K) if plan[W + i][2] is not None] or [0.0])),
+            "plain_step_ms": float(np.mean([t[i] for i in range(K) if plan[W + i][2] is None] or [0.0])),
+            "commits": commits, "buffer_leaves": buf_leaves, "launches_per_step": launches}
+
+
 def run_1m(W, K, rank, dev, flush, eager=False, summary_dtype=None):
     """1M-token cache, 8 KV heads: route + attend with 64 queries per head (throughput)
     and with 1 query per head (single step).  summary_dtype: the tree's summary storage
@@ -906,6 +973,12 @@ def main():
         "decode_kernel_gbs": dec_b / (float(rb["decode_ms"].mean()) * 1e-3) / 1e9,
         "decode_kernel_bytes": int(dec_b), "route_bytes": int(rb["route_bytes"]),
         "summaries_per_query": rb["summaries_per_query"], "clocks": rb["clocks"]}
+
+    # the same 128K steps with an append buffer (decode reads the buffer; commits overlap)
+    bu = run_buffered(w, W, K, rank, dev, flush)
+    line["decode_128k_buffered"] = {
+        "qps": ranks.weak_scaling_rate(w.batch * w.q_heads, world, max_over_ranks(bu["ms_per_step"])), **bu,
+        "call": "zha_decode_buffered per step; zha_tree_append of 2 leaves on a second stream when full"}
 
     if not args.no_1m:
         line["ctx_1m"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager))

@@ -436,8 +436,9 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
 
 // Causal routing (and, with d_O, attention): query qg routes over the tree of tokens
 // 0 .. positions[qg % nq] (kPathPrefix).  Each query's shared memory holds the route's region
-// (grown for the attention's stages when attending, as planned by plan_decode) followed by
-// the path region of its prefix's right edge.
+// (grown for the attention's stages when attending, as planned by plan_decode) and the path
+// region of its prefix's right edge: inside the row region after the route's candidate rows
+// when it fits there, else after the route's region.
 cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads, int nq, int beam,
                           const long long* d_positions, const void* d_K, const void* d_V, float scale,
                           int* d_leaf_idx, float* d_leaf_score, int* d_trace, void* d_O,
@@ -484,8 +485,13 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
   const int pw_warps = wide ? kRouteMaxWarps : kNarrowMaxWpq;
   const size_t route_part = route_smem_layout(D, a.cmax, beam, (size_t)a.rows_bytes, pw_warps).total;
   const size_t path_bytes = path_smem_layout(D, row, sum_bytes(t), (int)a.lb, a.b, t->L).total;
-  a.path_smem_off = (long long)route_align(route_part, 128);
-  const size_t per_query = (size_t)a.path_smem_off + path_bytes;
+  // The path is needed during the route only, so it goes inside the row region after the
+  // route's candidate rows when it fits there (the attention's stages overwrite it once the
+  // route is done), else after the query's route layout.
+  const size_t path_in_rows = route_align(route_rows_bytes(D, a.cmax, sum_bytes(t)), 128);
+  const bool inside = path_in_rows + path_bytes <= (size_t)a.rows_bytes;
+  a.path_smem_off = (long long)(inside ? path_in_rows : route_align(route_part, 128));
+  const size_t per_query = inside ? route_part : (size_t)a.path_smem_off + path_bytes;
   if ((attend && stage_tokens < 16) || per_query > (wide ? kCtaSmemCap : kRouteSmemCap)) {
     *unsupported = true;
     return cudaSuccess;

@@ -213,6 +213,9 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         }
         return;
       }
+      // every thread has seen the path's copies land: the path barrier's life ends here, as
+      // its memory may later hold the attention's stages
+      if (wq == 0 && lane == 0) mbar_inval(pbar);
       if constexpr (HASPATH) {
         if (live) {
           // fused append: the first query of each unit stores the path
@@ -308,6 +311,11 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
     }
     m = min(C, a.beam);
+    // This level's generic shared-memory writes (the path's rows and values, the patched
+    // candidate row) lie where bulk copies land next: the next level's rows, or the
+    // attention's stages.  Each thread orders its own writes before those copies (a proxy
+    // fence by the writing thread, then the barrier the copies follow).
+    fence_proxy_async_smem();
     qsync();
     int* tmp = cur;
     cur = nxt;
