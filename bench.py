@@ -397,13 +397,13 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     return res
 
 
-def run_buffered(w, W, K, rank, dev, flush, buf_leaves=2):
+def run_buffered(w, W, K, rank, dev, flush, buf_leaves=2, eager=False):
     """128K decode steps with an append buffer: each step writes one token into the buffer
     (tokens after the committed prefix) and runs zha_decode_buffered; when buf_leaves full
     leaves have accumulated, the step also commits them (zha_tree_append on a second stream,
     forked from the step and joined at its end, so the commit overlaps that step's decode).
-    One CUDA graph per step, start and end events on the decode stream around the fork and
-    the join; L2 flushed between steps."""
+    One CUDA graph per step (eager: the same launches without graphs), start and end events
+    on the decode stream around the fork and the join; L2 flushed between steps."""
     import torch
     from tree_indexed_sparse_build_b200 import ranks, synth, zha
 
@@ -429,30 +429,49 @@ def run_buffered(w, W, K, rank, dev, flush, buf_leaves=2):
         plan.append((n_tok, n_routed, target))
         if target is not None:
             n_routed = target
+    def step(s, e):
+        n_tok, nr, target = plan[s]
+        e[0].record(main)
+        if target is not None:
+            side.wait_stream(main)
+            zha.zha_tree_append(tree.handle, Kd, target, side)
+        zha.zha_decode_buffered(tree.handle, Qd[s], beam, Kd, Vd, nr, n_tok, w.scale, idx[s], O[s],
+                                None, None, main)
+        if target is not None:
+            main.wait_stream(side)
+        e[1].record(main)
+
     graphs, evs = [], []
     l0 = tree.launches
-    for s, (n_tok, nr, target) in enumerate(plan):
-        e = _graph_events(2)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=main, capture_error_mode="thread_local"):
-            e[0].record()
-            if target is not None:
-                side.wait_stream(main)
-                zha.zha_tree_append(tree.handle, Kd, target, side)
-            zha.zha_decode_buffered(tree.handle, Qd[s], beam, Kd, Vd, nr, n_tok, w.scale, idx[s], O[s],
-                                    None, None, main)
-            if target is not None:
-                main.wait_stream(side)
-            e[1].record()
-        graphs.append(g)
-        evs.append(e)
-    launches = (tree.launches - l0) / len(plan)
-    for s in range(W):
-        graphs[s].replay()
+    if eager:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in plan]
+        runs = [(lambda s=s: step(s, evs[s])) for s in range(len(plan))]
+        with torch.cuda.stream(main):  # the step's launches, outside any graph
+            for s in range(W):
+                runs[s]()
+        torch.cuda.synchronize()
+        launches = (tree.launches - l0) / W if W else 0.0
+    else:
+        for s in range(len(plan)):
+            e = _graph_events(2)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=main, capture_error_mode="thread_local"):
+                step(s, e)
+            graphs.append(g)
+            evs.append(e)
+        launches = (tree.launches - l0) / len(plan)
+        runs = [g.replay for g in graphs]
+        for s in range(W):
+            runs[s]()
     torch.cuda.synchronize()
     for s in range(W, W + K):
         flush.zero_()
-        graphs[s].replay()
+        if eager:
+            torch.cuda.synchronize()
+            with torch.cuda.stream(main):
+                runs[s]()
+        else:
+            runs[s]()
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_OK, "device error word set during the buffered steps"
     t = np.array([evs[s][0].elapsed_time(evs[s][1]) for s in range(W, W + K)])
@@ -837,6 +856,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-1m", action="store_true")
     ap.add_argument("--no-build", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the 128K variants (bf16 summaries, append buffer) and the 1M bf16-summary run")
     ap.add_argument("--profile-case", choices=["deep_1m_2kv"], default=None,
                     help="run only a small case for ncu captures: the 1M-token tree at 2 of its "
                          "8 KV heads (1,024 queries, 64 per head), zha_decode, eager launches")
@@ -962,30 +983,32 @@ def main():
         one["launches_per_step"] = {k: m[k]["launches_per_step"] for k in ("throughput", "single")}
         return one
 
-    # the same 128K decode steps over bf16-stored summaries (device-timed pass only)
-    rb = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager, mode=args.mode,
-                    summary_dtype=torch.bfloat16, e2e=False)
-    ms_b = max_over_ranks(float(rb["step_ms"].mean()))
-    dec_b = rb["route_bytes"] + rb["attend_bytes"] + (rb["append_bytes"] if fused_append else 0)
-    line["decode_128k_bf16_summaries"] = {
-        "qps": ranks.weak_scaling_rate(rb["queries_per_step"], world, ms_b), "ms_per_step": ms_b,
-        "decode_kernel_ms": float(rb["decode_ms"].mean()),
-        "decode_kernel_gbs": dec_b / (float(rb["decode_ms"].mean()) * 1e-3) / 1e9,
-        "decode_kernel_bytes": int(dec_b), "route_bytes": int(rb["route_bytes"]),
-        "summaries_per_query": rb["summaries_per_query"], "clocks": rb["clocks"]}
+    if not args.no_extras:
+        # the same 128K decode steps over bf16-stored summaries (device-timed pass only)
+        rb = run_decode(w, W, K, rank, dev, flush, sampler, eager=args.eager, mode=args.mode,
+                        summary_dtype=torch.bfloat16, e2e=False)
+        ms_b = max_over_ranks(float(rb["step_ms"].mean()))
+        dec_b = rb["route_bytes"] + rb["attend_bytes"] + (rb["append_bytes"] if fused_append else 0)
+        line["decode_128k_bf16_summaries"] = {
+            "qps": ranks.weak_scaling_rate(rb["queries_per_step"], world, ms_b), "ms_per_step": ms_b,
+            "decode_kernel_ms": float(rb["decode_ms"].mean()),
+            "decode_kernel_gbs": dec_b / (float(rb["decode_ms"].mean()) * 1e-3) / 1e9,
+            "decode_kernel_bytes": int(dec_b), "route_bytes": int(rb["route_bytes"]),
+            "summaries_per_query": rb["summaries_per_query"], "clocks": rb["clocks"]}
 
-    # the same 128K steps with an append buffer (decode reads the buffer; commits overlap)
-    bu = run_buffered(w, W, K, rank, dev, flush)
-    line["decode_128k_buffered"] = {
-        "qps": ranks.weak_scaling_rate(w.batch * w.q_heads, world, max_over_ranks(bu["ms_per_step"])), **bu,
-        "call": "zha_decode_buffered per step; zha_tree_append of 2 leaves on a second stream when full"}
+        # the same 128K steps with an append buffer (decode reads the buffer; commits overlap)
+        bu = run_buffered(w, W, K, rank, dev, flush, eager=args.eager)
+        line["decode_128k_buffered"] = {
+            "qps": ranks.weak_scaling_rate(w.batch * w.q_heads, world, max_over_ranks(bu["ms_per_step"])), **bu,
+            "call": "zha_decode_buffered per step; zha_tree_append of 2 leaves on a second stream when full"}
 
     if not args.no_1m:
         line["ctx_1m"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager))
-        # the same step over bf16-stored summaries (half the route's bytes; routing then
-        # follows the bf16 tree, so the leaf sets may differ from the fp32 tree's)
-        line["ctx_1m_bf16_summaries"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager,
-                                                      summary_dtype=torch.bfloat16))
+        if not args.no_extras:
+            # the same step over bf16-stored summaries (half the route's bytes; routing then
+            # follows the bf16 tree, so the leaf sets may differ from the fp32 tree's)
+            line["ctx_1m_bf16_summaries"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager,
+                                                          summary_dtype=torch.bfloat16))
 
     if not args.no_build and rank == 0:
         line["build_256k"] = run_build_256k(W, K, dev, flush)
