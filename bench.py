@@ -360,35 +360,58 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
         return res
 
     # End to end through the public API: per step, H2D of the new K/V rows and the query
-    # from pinned memory, append + route + attend, D2H of the output, synchronize.
-    tree.build(Kd, N)
-    hk = torch.from_numpy(np.ascontiguousarray(Kn[:, :, N:N + W + K])).view(torch.bfloat16).pin_memory()
-    hv = torch.from_numpy(np.ascontiguousarray(Vn[:, :, N:N + W + K])).view(torch.bfloat16).pin_memory()
+    # from pinned memory, append + route + attend, D2H of the output, synchronize.  Measured
+    # twice: each step's calls issued eagerly, and each step's calls (copies included)
+    # captured in one CUDA graph per step, as a serving loop would replay them (the value
+    # reported as e2e).
+    # host staging step-major ([step, batch, kv_heads, d]), so a step's rows are one contiguous
+    # pinned block (graph capture copies only from pinned, contiguous host memory)
+    hk = torch.from_numpy(np.ascontiguousarray(np.moveaxis(Kn[:, :, N:N + W + K], 2, 0))).view(
+        torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(np.ascontiguousarray(np.moveaxis(Vn[:, :, N:N + W + K], 2, 0))).view(
+        torch.bfloat16).pin_memory()
     hq = torch.from_numpy(Qs).view(torch.bfloat16).pin_memory()
     ho = torch.empty((K, B, Hq, nq, d), dtype=torch.bfloat16).pin_memory()
     qbuf = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
     obuf = torch.empty((B, Hq, nq, d), dtype=torch.bfloat16, device=dev)
     ibuf = torch.empty((B, Hq, nq, beam), dtype=torch.int32, device=dev)
 
-    def e2e_step(s, out_slot):
+    def e2e_calls(s, out_slot):
         pos = N + s
-        Kd[:, :, pos].copy_(hk[:, :, s], non_blocking=True)
-        Vd[:, :, pos].copy_(hv[:, :, s], non_blocking=True)
+        Kd[:, :, pos].copy_(hk[s], non_blocking=True)
+        Vd[:, :, pos].copy_(hv[s], non_blocking=True)
         qbuf.copy_(hq[s], non_blocking=True)
         decode_call(pos + 1, qbuf, ibuf, obuf, None)
         if out_slot is not None:
             ho[out_slot].copy_(obuf, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
 
-    for s in range(W):
-        e2e_step(s, None)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for s in range(K):
-        e2e_step(W + s, s)
-    e1.record()
-    torch.cuda.synchronize()
-    res["e2e_ms_per_step"] = e0.elapsed_time(e1) / K
+    def timed_e2e(run):
+        for s in range(W):
+            run(s, None)
+            torch.cuda.current_stream().synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(K):
+            run(W + s, s)
+            torch.cuda.current_stream().synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+    tree.build(Kd, N)
+    res["e2e_eager_ms_per_step"] = timed_e2e(e2e_calls)
+    if not eager:
+        tree.build(Kd, N)  # the same starting tree; the graphs replay the same steps
+        egraphs = []
+        for s in range(W + K):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream, capture_error_mode="thread_local"):
+                e2e_calls(s, s - W if s >= W else None)
+            egraphs.append(g)
+        res["e2e_ms_per_step"] = timed_e2e(lambda s, slot: egraphs[s].replay())
+        del egraphs
+    else:
+        res["e2e_ms_per_step"] = res["e2e_eager_ms_per_step"]
     res["h2d_bytes_per_step"] = int(2 * B * w.kv_heads * d * 2 + B * Hq * nq * d * 2)
     res["d2h_bytes_per_step"] = int(B * Hq * nq * d * 2)
     # parity spot check of the last e2e output against the graph run is not meaningful
@@ -953,7 +976,12 @@ def main():
         "keys_per_query": r["keys_per_query"], "summaries_per_query": r["summaries_per_query"],
         "e2e": {"value": r["queries_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": r["h2d_bytes_per_step"],
-                "d2h_bytes_per_step": r["d2h_bytes_per_step"]},
+                "d2h_bytes_per_step": r["d2h_bytes_per_step"],
+                "launch": "one CUDA graph per step: H2D of the step's K/V rows and query from pinned "
+                          "memory, zha_decode_step, D2H of O; host synchronizes every step"},
+        "e2e_eager": {"value": r["queries_per_step"] * world / (max_over_ranks(r["e2e_eager_ms_per_step"]) * 1e-3),
+                      "unit": UNIT, "ms_per_step": max_over_ranks(r["e2e_eager_ms_per_step"]),
+                      "launch": "the same calls issued eagerly each step"},
         "gpu_launches": int(round(r["launches_per_step"] * K)),
         "launch_mode": "eager" if args.eager else "cuda_graph_per_step",
         "decode_call": {"step": "zha_decode_step (append + route + attention, one launch)",

@@ -22,7 +22,7 @@ namespace zha {
 // Shared memory of the path, for head_dim D, token rows of row_bytes, summary elements of
 // sum_bytes, leaf block lb, branching b and (at most) L levels below the root.
 struct PathSmem {
-  size_t tok, sib, pv, pf, node, kpos, qn, bar, total;
+  size_t tok, sib, pf, node, kpos, qn, bar, total;
 };
 __host__ __device__ inline size_t path_align(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int sum_bytes, int lb, int b,
@@ -33,8 +33,6 @@ __host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int s
   o = path_align(o + (size_t)lb * row_bytes, 16);
   s.sib = o;   // for l = 1..L: the children of path node l, stored rows [b][D]
   o += (size_t)L * b * D * sum_bytes;
-  s.pv = o;    // fp64 values of the path node at two consecutive levels [2][D]
-  o += (size_t)2 * D * 8;
   s.pf = o;    // the stored path rows, levels 0..L [L + 1][D]
   o = path_align(o + (size_t)(L + 1) * D * sum_bytes, 8);
   s.node = o;  // path node index per level [L + 1]
@@ -75,13 +73,15 @@ __device__ void path_issue(const PathSmem& P, unsigned char* pb, const char* Ku,
 }
 
 // Threads tid < D of the group (nt threads in all): the path rows, after pbar completed.
-// sync() synchronises the group.  writer: also store the rows into the unit's summaries.
+// Each thread carries its dims e = tid, tid + nt, .. from the leaf to the root with the
+// kept fp64 value in a register (a level's dim e needs only dim e of the level below), so
+// the levels need no barrier; sync() once at the end makes the rows visible to the group.
+// writer: also store the rows into the unit's summaries.
 template <typename TIn, typename TS, int D, typename Sync>
 __device__ void path_compute(const PathSmem& P, unsigned char* pb, TS* pyr_u, const long long* off,
                              const long long* n, int b, int L, int ntok, bool writer, int tid, int nt,
                              Sync sync) {
   const TIn* tok = reinterpret_cast<const TIn*>(pb + P.tok);
-  double* pv = reinterpret_cast<double*>(pb + P.pv);
   TS* pf = reinterpret_cast<TS*>(pb + P.pf);
   const long long* node = reinterpret_cast<const long long*>(pb + P.node);
   for (int e = tid; e < D; e += nt) {
@@ -92,28 +92,23 @@ __device__ void path_compute(const PathSmem& P, unsigned char* pb, TS* pyr_u, co
       else
         s += (double)tok[(size_t)r * D + e];
     }
-    const double v = s / (double)ntok;
-    pv[e] = SumT<TS>::kept(v);
+    double v = s / (double)ntok;
+    double kept = SumT<TS>::kept(v);
     pf[e] = SumT<TS>::store(v);
     if (writer) pyr_u[(off[0] + node[0]) * D + e] = pf[e];
-  }
-  sync();
-  for (int l = 1; l <= L; ++l) {
-    const double* cur = pv + (size_t)((l - 1) & 1) * D;
-    double* nxt = pv + (size_t)(l & 1) * D;
-    const TS* sib = reinterpret_cast<const TS*>(pb + P.sib + (size_t)(l - 1) * b * D * sizeof(TS));
-    const long long c0 = node[l] * b, c1 = min(c0 + (long long)b, n[l - 1]);
-    for (int e = tid; e < D; e += nt) {
-      double s = 0.0;
+    for (int l = 1; l <= L; ++l) {
+      const TS* sib = reinterpret_cast<const TS*>(pb + P.sib + (size_t)(l - 1) * b * D * sizeof(TS));
+      const long long c0 = node[l] * b, c1 = min(c0 + (long long)b, n[l - 1]);
+      double t = 0.0;
       for (long long c = c0; c < c1; ++c)
-        s += c == node[l - 1] ? cur[e] : (double)SumT<TS>::load(sib[(c - c0) * D + e]);
-      const double v = s / (double)(c1 - c0);
-      nxt[e] = SumT<TS>::kept(v);
+        t += c == node[l - 1] ? kept : (double)SumT<TS>::load(sib[(c - c0) * D + e]);
+      v = t / (double)(c1 - c0);
+      kept = SumT<TS>::kept(v);
       pf[(size_t)l * D + e] = SumT<TS>::store(v);
       if (writer) pyr_u[(off[l] + node[l]) * D + e] = pf[(size_t)l * D + e];
     }
-    sync();
   }
+  sync();
 }
 
 }  // namespace zha
