@@ -138,11 +138,14 @@ def test_threshold_frontier_overflow_is_reported_per_query(dev):
     assert (toks == -1).all()
 
 
-def test_radii_follow_appends_and_decode_steps(dev):
+@pytest.mark.parametrize("sdt", ["f32", "bf16"])
+def test_radii_follow_appends_and_decode_steps(dev, sdt):
     # radii kept current by append and zha_decode_step equal a fresh computation bit for bit
+    # (fp32 and bf16 summaries: the centers are the stored summaries either way)
     w = _wl("th_grow", 1, 2, 4, 64, 1024, "f32", 2, 16, 2, 1, 306)
     cap = 1024 + 80
-    tree, (Qn, Kn, Vn), (Q, K, V) = _setup(w, dev, 1, capacity=cap)
+    tree, (Qn, Kn, Vn), (Q, K, V) = _setup(w, dev, 1, capacity=cap,
+                                           summary_dtype=torch.bfloat16 if sdt == "bf16" else None)
     tree.build(K, 700)
     tree.attach_radii(K)
     for n in (701, 703, 760, 1024, 1025):  # crosses leaves and adds a level
