@@ -12,9 +12,12 @@
 //
 // GPU mapping: one CTA of 8 warps per query.  The survivors of a level live in shared
 // memory (at most kFrontierCap); the children of the survivors are tested in chunks of
-// kChunk candidates, one warp per candidate row (each lane head_dim / 32 dims), and the
-// kept ones are compacted in candidate order by a block-wide prefix sum, so survivors and
-// the tokens found stay ascending.  The leaves' tokens go through the same chunked test.
+// kChunk candidates, one thread per candidate row: the thread sums its row's products in
+// dim order with fp64 FMAs against q held in shared memory (fp64, read as a broadcast), so
+// no cross-lane reduction is needed; and since a product of a stored element (bf16 or fp32)
+// and a q element is exact in fp64, that sum is bit for bit the plain sequential fp64 sum.
+// The kept ones are compacted in candidate order by a block-wide prefix sum, so survivors
+// and the tokens found stay ascending.  The leaves' tokens go through the same chunked test.
 #include "device_common.cuh"
 #include "zha_internal.h"
 
@@ -52,6 +55,32 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// dot = sum over dims e in order of q[e] * row[e], and (MAG) mag = sum of |q[e] * row[e]|, in
+// fp64 by one thread: the row read in 16-byte pieces (four in flight), q from shared memory.
+template <typename T, int D, bool MAG>
+__device__ __forceinline__ void row_dot(const T* row, const double* q, double& dot, double& mag) {
+  constexpr int EPC = Vec16<T>::N;
+  dot = 0.0;
+  mag = 0.0;
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += 4 * EPC) {
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = ldg16(row + c0 + i * EPC);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float f[EPC];
+      Vec16<T>::to_f32(v[i], f);
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) {
+        const double qe = q[c0 + i * EPC + e], x = (double)f[e];
+        dot = fma(qe, x, dot);
+        if (MAG) mag += fabs(qe * x);
+      }
+    }
+  }
 }
 
 // Block-wide ordered compaction of one chunk: flags[i] (i < n) -> positions base + prefix.
@@ -94,6 +123,7 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
   int* pos = fb + kFrontierCap;                                     // [kChunk]
   unsigned char* flags = reinterpret_cast<unsigned char*>(pos + kChunk);  // [kChunk]
   int* wsum = reinterpret_cast<int*>(flags + kChunk);               // [kThWarps]
+  double* qs = reinterpret_cast<double*>(wsum + kThWarps + 4);      // [D], 16-byte aligned
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const long long qg = blockIdx.x;
   pdl_wait();
@@ -119,6 +149,9 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
 #pragma unroll
   for (int e = 0; e < DPL; ++e) qn = fma(qv[e], qv[e], qn);
   qn = sqrt(warp_sum_d(qn));
+  if (warp == 0)
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) qs[lane * DPL + e] = qv[e];
 
   int* cur = fa;
   int* nxt = fb;
@@ -134,24 +167,17 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
     int mn = 0;
     for (long long c0 = 0; c0 < total; c0 += kChunk) {
       const int n = (int)min((long long)kChunk, total - c0);
-      for (int k = warp; k < n; k += kThWarps) {
+      for (int k = t; k < n; k += kThThreads) {  // one candidate row per thread
         const long long slot = c0 + k;
         const long long node = (long long)a.b * cur[slot / a.b] + slot % a.b;
         bool keep = false;
         if (node < a.n[l]) {
-          double dot = 0.0, mag = 0.0;
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) {
-            const double c = (double)SumT<TS>::load(S[node * D + lane * DPL + e]);
-            dot = fma(qv[e], c, dot);
-            mag += fabs(qv[e] * c);
-          }
-          dot = warp_sum_d(dot);
-          mag = warp_sum_d(mag);
+          double dot, mag;
+          row_dot<TS, D, true>(S + node * D, qs, dot, mag);
           const double rq = qn * (double)R[node];
           keep = dot + rq >= tau - 1e-9 * (mag + rq + fabs(tau));
         }
-        if (lane == 0) flags[k] = keep ? 1 : 0;
+        flags[k] = keep ? 1 : 0;
       }
       __syncthreads();
       const int kept = chunk_compact(flags, n, pos, wsum);
@@ -183,24 +209,16 @@ __global__ void __launch_bounds__(kThThreads) threshold_kernel(const ThreshArgs 
     const long long total = (long long)m * a.lb;
     for (long long c0 = 0; c0 < total; c0 += kChunk) {
       const int n = (int)min((long long)kChunk, total - c0);
-      for (int k = warp; k < n; k += kThWarps) {
+      for (int k = t; k < n; k += kThThreads) {  // one token per thread
         const long long slot = c0 + k;
         const long long tok = (long long)cur[slot / a.lb] * a.lb + slot % a.lb;
         bool keep = false;
         if (tok < a.N) {
-          double dot = 0.0;
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) {
-            double kx;
-            if constexpr (sizeof(TK) == 2)
-              kx = (double)bf16_bits_to_f32(Ku[tok * D + lane * DPL + e]);
-            else
-              kx = (double)Ku[tok * D + lane * DPL + e];
-            dot = fma(qv[e], kx, dot);
-          }
-          keep = warp_sum_d(dot) >= tau;
+          double dot, mag;
+          row_dot<TK, D, false>(Ku + tok * D, qs, dot, mag);
+          keep = dot >= tau;
         }
-        if (lane == 0) flags[k] = keep ? 1 : 0;
+        flags[k] = keep ? 1 : 0;
       }
       __syncthreads();
       const int kept = chunk_compact(flags, n, pos, wsum);
@@ -268,7 +286,7 @@ cudaError_t launch_threshold(zha_tree* t, const void* d_K, const void* d_Q, zha_
   a.count = d_count;
   a.stats = d_stats;
   a.total_queries = (long long)t->desc.batch * q_heads * nq;
-  const size_t smem = (size_t)2 * kFrontierCap * 4 + kChunk * 4 + kChunk + kThWarps * 4;
+  const size_t smem = (size_t)2 * kFrontierCap * 4 + kChunk * 4 + kChunk + kThWarps * 4 + 16 + (size_t)D * 8;
   cudaError_t e;
   if (sbf)
     e = bf ? (D == 128 ? run_threshold<uint16_t, uint16_t, 128>(a, smem, stream)
