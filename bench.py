@@ -580,6 +580,8 @@ def run_1m(W, K, rank, dev, flush, eager=False, summary_dtype=None):
         step_ms = times[2][:, 0]
         pb = path_bytes(idx.cpu().numpy(), tr.cpu().numpy(), counts, N, w.leaf_block,
                         w.branching, d, 2, w.group, 2, sum_bytes=sum_bytes)
+        if mode == "throughput":  # the needles were planted for these 64 queries per head
+            out["needle_recall"] = needle_recall(w, Qn, idx.cpu().numpy())
         out[mode] = {"route_ms": tr_ms, "attend_ms": at_ms, "step_ms": step_ms,
                      "queries_per_step": w.batch * w.q_heads * nq, "launches_per_step": launches, **pb}
         del runs
@@ -634,6 +636,39 @@ def run_build_256k(W, K, dev, flush):
            "qps": q / (np.mean(ra_ms) * 1e-3)}
     tree.close()
     return res
+
+
+def needle_recall(w, Qn, idx) -> dict:
+    """Planted needles whose leaf the assigned query's routed leaves include (a reported figure,
+    not a pass mark: mean pooling over a leaf block dilutes a single key).  idx: the route's
+    leaf indices [batch, q_heads, nq, beam] for the queries Qn the needles were planted with."""
+    from tree_indexed_sparse_build_b200 import synth
+    hits = total = 0
+    for u, lst in enumerate(synth.needles(w, Qn)):
+        b = u // w.kv_heads
+        for p, hq, qi in lst:
+            total += 1
+            hits += int((idx[b, hq, qi] == p // w.leaf_block).any())
+    return {"needles": total, "retrieved": hits, "recall": hits / total if total else None}
+
+
+def run_needles(dev) -> dict:
+    """Needle recall of zha_route on the workloads with planted needles (tiny_fp32: 4 needles
+    = 3 q_hat + N(0, 0.1^2); gqa_32k: 16 per KV head = 4 q_hat + N(0, 0.2^2))."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+    out = {}
+    for name in ("tiny_fp32", "gqa_32k"):
+        w = workloads.get(name)
+        Qn = synth.queries(w)
+        Kn = synth.keys(w, Q=Qn)
+        tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len,
+                        torch.float32 if w.kv_dtype == "f32" else torch.bfloat16)
+        tree.build(synth.to_torch(Kn, dev), w.seq_len)
+        idx, _, _ = tree.route(synth.to_torch(Qn, dev), w.beam)
+        out[name] = needle_recall(w, Qn, idx.cpu().numpy())
+        tree.close()
+    return out
 
 
 def run_causal(W, K, dev, flush):
@@ -1009,6 +1044,7 @@ def main():
         one["workload"] = ("deep_1m: 1 x 8 KV heads x 64 query heads, d 128, 1,048,576 bf16 tokens, "
                            "b 8, leaf block 4, beam 8; throughput = 64 queries per head per step")
         one["launches_per_step"] = {k: m[k]["launches_per_step"] for k in ("throughput", "single")}
+        one["needle_recall"] = m["needle_recall"]
         return one
 
     if not args.no_extras:
@@ -1041,6 +1077,7 @@ def main():
     if not args.no_build and rank == 0:
         line["build_256k"] = run_build_256k(W, K, dev, flush)
         line["causal"] = run_causal(W, min(K, 10), dev, flush)
+        line["needle_recall"] = run_needles(dev)
         line["threshold"] = run_threshold(W, min(K, 10), dev, flush)
 
     if rank == 0 and world == 1:
