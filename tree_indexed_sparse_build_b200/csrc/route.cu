@@ -4,7 +4,9 @@
 //
 // Survivors start as {root}.  For l = L-1 .. 0 every existing child c of a survivor is
 // scored by q . S_l[c] in fp32, and the top-min(beam, #candidates) are kept, ordered by
-// score descending with the lower node index first on equal scores.
+// score descending with the lower node index first on equal scores.  Levels with at most
+// beam nodes below the root are kept whole without scoring (the route starts at the
+// highest level with more than beam nodes, from every node of the level above it).
 //
 // GPU mapping.  A candidate's key packs (order-preserving score bits, inverted node
 // index) into 64 bits, so "greater key" is exactly "ranks first".  Candidates are the
@@ -16,15 +18,17 @@
 // one contiguous run of rows -- all completing on the query's mbarrier, so a level costs
 // one memory round trip whatever its width and holds no registers while in flight.
 // Few queries ("wide"): one query per CTA with up to 16 warps scoring from shared memory.
-// Many queries ("narrow"): several queries per CTA, one warp each, no CTA barriers.
-// Four lanes score one row from shared memory against q held in registers (each lane a
-// quarter of the dims; the chunk order alternates between neighbouring rows so the two
-// rows of a shared-memory phase use opposite bank halves), two rows per lane in flight.
-// One warp per query then holds the candidate keys in registers, finds the B-th largest
-// by a binary search on the key bits with ballot-based warp counts (starting below the
-// common prefix of the largest and smallest score, stopping as soon as exactly B keys
-// remain), and compacts the kept candidates with ballots in candidate order, which keeps
-// the survivors ascending without a sort.
+// Many queries ("narrow"): several queries per CTA, 1-4 warps each on a named barrier per
+// query, sized so the most queries stay resident per SM.  Four lanes score one row from
+// shared memory against q held in registers (each lane a quarter of the dims; the chunk
+// order alternates between neighbouring rows so the two rows of a shared-memory phase use
+// opposite bank halves), two rows per lane in flight.  Selection: up to 64 candidates, one
+// warp holds the keys in registers, finds the B-th largest by a binary search on the key
+// bits with ballot-based warp counts (starting below the common prefix of the largest and
+// smallest score, stopping as soon as exactly B keys remain) and compacts the kept ones
+// with ballots in candidate order, which keeps the survivors ascending without a sort;
+// 65-128, ranks counted over the query's threads; wider, a radix select over the group
+// (route_common.cuh).
 //
 // Fallback kernel (route_reg_kernel) for levels too wide to stage in shared memory:
 // the same selection, with candidate rows loaded into registers in batches.

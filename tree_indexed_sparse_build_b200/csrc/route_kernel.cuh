@@ -22,18 +22,19 @@ namespace zha {
 //
 // With TKV = the KV storage type (not NoKV) the kernel is the fused decode: once the
 // last level is selected, the query's warps attend over the tokens of its leaves.  The
-// candidate-row region, free after the leaf-level scoring, becomes two K/V stage buffers
-// filled by one bulk copy per leaf piece (K and V) on the two mbarriers; the warps run
-// the online softmax of attn_core.cuh over each stage, merge their states through shared
-// memory and write O.  No leaf list goes through global memory and nothing is launched
-// between the route and the attention.
+// candidate-row region, free after the leaf-level scoring, becomes two or three K/V stage
+// buffers filled by one bulk copy per leaf piece (K and V) on their "full" mbarriers and
+// refilled as the warps release them (decode_attn.cuh); the warps run the online softmax
+// of attn_core.cuh over each stage, merge their states through shared memory and write O.
+// No leaf list goes through global memory and nothing is launched between the route and
+// the attention.  With buf_tokens the attention also covers the append buffer's tokens.
 // NARROW instantiations are built for CTAs of at most 8 warps, three per SM (register cap).
 // PATH (decode_append.cuh; needs TKV, the type of the K rows the path reads):
 //  kPathAppend (fused decode, one query per CTA) -- the kernel first extends the tree by
 //    the tokens appended to one leaf, and stores the path (one CTA per unit);
-//  kPathPrefix (causal routing) -- query qg routes over the tree of tokens 0 .. p, p =
-//    positions[qg % nq]: its own depth and node counts, and its prefix's right edge
-//    recomputed into shared memory (never stored).
+//  kPathPrefix (causal routing, append-buffer decode) -- query qg routes over the tree of
+//    tokens 0 .. p, p = positions[qg % nq] (or prefix_pos): its own depth and node counts,
+//    and its prefix's right edge recomputed into shared memory (never stored).
 // With a KV type, the query then attends over its leaves unless O is null.
 // TS: the summaries' storage (float, or bf16 bits in uint16_t); rows are staged as stored
 // and widened to fp32 as they are scored.
