@@ -117,3 +117,61 @@ def test_random_shape_matches_oracle(dev, seed):
     assert checked > 0
     assert worst <= (1e-5 if (w.kv_dtype == "f32" and w.out_dtype == "f32") else 2e-2), worst
     tree.close()
+
+
+@pytest.mark.parametrize("seed", CASES[:12])
+def test_random_shape_causal_and_buffered(dev, seed):
+    # causal routing at random positions, and the append-buffer decode over a committed prefix
+    from tree_indexed_sparse_build_b200 import zha
+    w, sdt = _case(seed)
+    summary = "bf16" if sdt == "bf16" else "f64"
+    Qn, Kn, Vn = make_inputs(w)
+    Q, K, V = torch_of(Qn, dev), torch_of(Kn, dev), torch_of(Vn, dev)
+    tdt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, w.seq_len, tdt,
+                    summary_dtype=torch.bfloat16 if sdt == "bf16" else torch.float32)
+    n_routed = max(w.leaf_block, (w.seq_len // 2) // w.leaf_block * w.leaf_block)
+    tree.build(K, n_routed)
+    rng = np.random.default_rng(1000 + seed)
+    pos = rng.integers(0, n_routed, size=w.nq).astype(np.int64)
+    try:
+        cidx, ctr = tree.route_causal(K, Q, torch.from_numpy(pos).to(dev), w.beam, trace=True)
+        Ob, bidx = tree.decode_buffered(Q, K, V, n_routed, w.seq_len, w.beam, w.scale, out_dtype=odt)
+    except zha.ZhaError as e:  # a level too wide for the staged kernel: the call says so
+        assert e.status == zha.ZHA_ERR_UNSUPPORTED
+        pytest.skip("shape outside the staged kernel")
+    torch.cuda.synchronize()
+    assert tree.check() == zha.ZHA_OK
+    cidx, ctr, bidx, got = cidx.cpu().numpy(), ctr.cpu().numpy(), bidx.cpu().numpy(), out_to_f64(Ob)
+    checked = 0
+    worst = 0.0
+    for u in (0, w.units - 1):
+        bb, h = divmod(u, w.kv_heads)
+        otb = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching, summary=summary).build(Kn[bb, h], n_routed)
+        for hq in range(h * w.group, (h + 1) * w.group):
+            q64 = synth.to_f64(Qn[bb, hq])
+            resb = otb.route(q64, w.beam)
+            okb = oracle.well_conditioned(resb["bounds"])
+            for i in range(q64.shape[0]):
+                # causal: the tree of the prefix 0 .. pos[i]
+                ot = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching, summary=summary).build(
+                    Kn[bb, h], int(pos[i]) + 1)
+                res = ot.route(q64[i:i + 1], w.beam)
+                if oracle.well_conditioned(res["bounds"])[0]:
+                    np.testing.assert_array_equal(cidx[bb, hq, i], res["leaves"][0])
+                    L = ctr.shape[3]
+                    np.testing.assert_array_equal(ctr[bb, hq, i, L - ot.L:], res["survivors"][0])
+                    checked += 1
+                # buffered: routed over the first n_routed tokens, the rest attended
+                if okb[i]:
+                    np.testing.assert_array_equal(bidx[bb, hq, i], resb["leaves"][i])
+                ref, _ = oracle.attend_buffered(q64[i], Kn[bb, h], Vn[bb, h], bidx[bb, hq, i], n_routed, w.seq_len,
+                                                w.leaf_block, w.scale)
+                if w.kv_dtype == "f32" and w.out_dtype == "f32":
+                    worst = max(worst, float(np.abs(got[bb, hq, i] - ref).max()))
+                else:
+                    worst = max(worst, rel_l2(got[bb, hq, i], ref))
+    assert checked > 0
+    assert worst <= (1e-5 if (w.kv_dtype == "f32" and w.out_dtype == "f32") else 2e-2), worst
+    tree.close()
