@@ -293,3 +293,35 @@ def test_host_errors_leave_tree_usable(dev):
     idx, _, _ = tree.route(Q, w.beam)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_OK
+
+
+@pytest.mark.parametrize("kv", ["f32", "bf16"])
+def test_largest_beam_keeps_every_leaf(dev, kv):
+    # beam 1024 with beam * b = 4096 (the limits): a tree of 1,000 leaves keeps them all, so
+    # routing returns every leaf in order (then -1) and attention equals dense attention over
+    # the whole cache.  The levels above the leaves are kept whole; the 1,000 leaf rows are
+    # too many to stage, so they are scored by the register route and attended by a second
+    # launch
+    from tree_indexed_sparse_build_b200 import zha
+    w = _wl(f"beam1024_{kv}", 1, 1, 2, 64, 3000, kv, 4, 3, 1024, 2, 118)
+    tree, (Qn, Kn, Vn), (Q, K, V) = _setup(w, dev)
+    tree.build(K, w.seq_len)
+    n0 = tree.level_nodes(0)
+    assert n0 == 1000
+    idx, _, _ = tree.route(Q, w.beam)
+    expect = torch.cat([torch.arange(n0, dtype=torch.int32), torch.full((w.beam - n0,), -1, dtype=torch.int32)])
+    assert (idx.cpu() == expect).all()
+    odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    O, didx = tree.decode(Q, K, V, w.beam, w.scale, out_dtype=odt)[:2]
+    torch.cuda.synchronize()
+    assert tree.check() == zha.ZHA_OK
+    assert torch.equal(didx, idx)
+    got = out_to_f64(O)
+    for hq in range(w.q_heads):
+        q64 = synth.to_f64(Qn[0, hq])
+        for i in range(q64.shape[0]):
+            ref = oracle.dense(q64[i], Kn[0, 0], Vn[0, 0], w.seq_len, w.scale)
+            if kv == "f32":
+                assert np.abs(got[0, hq, i] - ref).max() <= 1e-5
+            else:
+                assert rel_l2(got[0, hq, i], ref) <= 2e-2
