@@ -39,13 +39,17 @@ __device__ __forceinline__ void attn_load_q(const void* Q, bool q_bf16, long lon
 #pragma unroll
     for (int j = 0; j < S::CPL; ++j) {
       const int c = 4 * (j ^ par) + sub;
-#pragma unroll
-      for (int e = 0; e < S::VEC; e += 8) {
-        const uint4 v = ldg16(qrow + (size_t)(c * S::VEC + e) * 2);
+      if constexpr (S::VEC == 8) {  // bf16 K: a chunk is 16 bytes of q as well
         float f[8];
-        Vec16<uint16_t>::to_f32(v, f);
+        Vec16<uint16_t>::to_f32(ldg16(qrow + (size_t)c * 16), f);
 #pragma unroll
-        for (int k = 0; k < 8 && e + k < S::VEC; ++k) qv[j][e + k] = f[k];
+        for (int k = 0; k < 8; ++k) qv[j][k] = f[k];
+      } else {  // fp32 K: four bf16 elements, 8 bytes (8-byte aligned only)
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(qrow + (size_t)c * 8));
+        qv[j][0] = bf16_bits_to_f32(v.x & 0xFFFFu);
+        qv[j][1] = bf16_bits_to_f32(v.x >> 16);
+        qv[j][2] = bf16_bits_to_f32(v.y & 0xFFFFu);
+        qv[j][3] = bf16_bits_to_f32(v.y >> 16);
       }
     }
   } else {
