@@ -285,9 +285,11 @@ def test_host_errors_leave_tree_usable(dev):
     with pytest.raises(zha.ZhaError) as e:
         tree.route(Q, 1024)  # beam * b > 4096
     assert e.value.status == zha.ZHA_ERR_UNSUPPORTED
-    with pytest.raises(zha.ZhaError):
-        zha.zha_route(tree.handle, Q[:, :3].contiguous(), w.beam,
-                      torch.empty(1, dtype=torch.int32, device=dev))  # 3 heads % 2 kv heads
+    Q3 = Q[:, :3].contiguous()
+    with pytest.raises(zha.ZhaError):  # 3 heads % 2 kv heads
+        zha.zha_route(tree.handle, Q3, w.beam, torch.empty(Q3.shape[:3] + (w.beam,), dtype=torch.int32, device=dev))
+    with pytest.raises(ValueError):  # a leaf-index buffer too small for the queries: refused
+        zha.zha_route(tree.handle, Q, w.beam, torch.empty(1, dtype=torch.int32, device=dev))
     idx, _, _ = tree.route(Q[:, :, :0].contiguous(), w.beam)  # nq == 0 is a no-op
     assert idx.numel() == 0
     idx, _, _ = tree.route(Q, w.beam)

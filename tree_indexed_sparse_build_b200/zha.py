@@ -119,6 +119,40 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _expect(t: torch.Tensor | None, what: str, numel: int, dtypes: tuple) -> None:
+    """Refuse a buffer the library would read or write past, or read as another type: the C
+    calls take plain pointers, so sizes are checked here (they follow from Q's shape)."""
+    if t is None:
+        return
+    if t.dtype not in dtypes:
+        raise ValueError(f"{what}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if t.numel() != numel:
+        raise ValueError(f"{what}: {t.numel()} elements, expected {numel}")
+
+
+_I32, _I64, _F32 = (torch.int32,), (torch.int64,), (torch.float32,)
+_OUT = (torch.float32, torch.bfloat16)
+
+
+def _route_buffers(handle, Q: torch.Tensor, beam: int, leaf_idx, leaf_score=None, trace=None,
+                   O=None, appending: bool = False) -> None:
+    """leaf_idx / leaf_score [batch, q_heads, nq, beam], trace [.., levels, beam], O like Q.
+    appending: the call first appends, so the trace has the levels of the grown tree (at
+    least the current ones)."""
+    B, Hq, nq, _ = Q.shape
+    n = B * Hq * nq * int(beam)
+    _expect(leaf_idx, "leaf_idx", n, _I32)
+    _expect(leaf_score, "leaf_score", n, _F32)
+    _expect(O, "O", Q.numel(), _OUT)
+    if trace is not None:
+        L = max(zha_tree_levels(handle), 1)
+        if not appending:
+            _expect(trace, "trace", n * L, _I32)
+        elif trace.dtype != torch.int32 or n == 0 or trace.numel() % n or trace.numel() // n < L:
+            raise ValueError(f"trace: {trace.numel()} {trace.dtype} elements, expected int32 "
+                             f"[batch, q_heads, nq, levels >= {L}, beam]")
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -163,6 +197,7 @@ def zha_route(handle, Q: torch.Tensor, beam: int, leaf_idx: torch.Tensor,
               leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
               stream=None) -> None:
     B, Hq, nq, _ = Q.shape
+    _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace)
     _check(lib().zha_route(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(leaf_idx),
                            _ptr(leaf_score), _ptr(trace), _stream(stream)), "zha_route")
 
@@ -175,6 +210,7 @@ def zha_sparse_attn_decode(handle, Q: torch.Tensor, K: torch.Tensor, V: torch.Te
                            leaf_idx: torch.Tensor, beam: int, scale: float, O: torch.Tensor,
                            scratch: torch.Tensor | None = None, stream=None) -> None:
     B, Hq, nq, _ = Q.shape
+    _route_buffers(handle, Q, beam, leaf_idx, O=O)
     nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
     _check(lib().zha_sparse_attn_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(K),
                                         _ptr(V), _ptr(leaf_idx), beam, scale, _ptr(O),
@@ -187,6 +223,7 @@ def zha_sparse_attn_decode_noalloc(handle, Q: torch.Tensor, K: torch.Tensor, V: 
                                    O: torch.Tensor, stream=None) -> None:
     """zha_sparse_attn_decode with the library's own fixed scratch (no caller buffer)."""
     B, Hq, nq, _ = Q.shape
+    _route_buffers(handle, Q, beam, leaf_idx, O=O)
     _check(lib().zha_sparse_attn_decode_noalloc(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq,
                                                 _ptr(K), _ptr(V), _ptr(leaf_idx), beam, scale,
                                                 _ptr(O), dtype_code(O.dtype), _stream(stream)),
@@ -198,6 +235,7 @@ def zha_decode(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: torch.Ten
                trace: torch.Tensor | None = None, stream=None) -> None:
     """Route + attention in one call (one launch when the levels fit shared memory)."""
     B, Hq, nq, _ = Q.shape
+    _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O)
     _check(lib().zha_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
                             scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _ptr(O),
                             dtype_code(O.dtype), _stream(stream)), "zha_decode")
@@ -209,6 +247,7 @@ def zha_decode_step(handle, K: torch.Tensor, V: torch.Tensor, new_seq_len: int, 
                     stream=None) -> None:
     """Append up to new_seq_len, then route + attention (one launch for one-leaf appends)."""
     B, Hq, nq, _ = Q.shape
+    _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O, appending=True)
     _check(lib().zha_decode_step(handle, _ptr(K), _ptr(V), new_seq_len, _ptr(Q), dtype_code(Q.dtype),
                                  Hq, nq, beam, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
                                  _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_step")
@@ -219,6 +258,8 @@ def zha_route_causal(handle, K: torch.Tensor, Q: torch.Tensor, positions: torch.
                      trace: torch.Tensor | None = None, stream=None) -> None:
     """Query i of every head routes over the tree of tokens 0 .. positions[i] (int64, device)."""
     B, Hq, nq, _ = Q.shape
+    _expect(positions, "positions", nq, _I64)
+    _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace)
     _check(lib().zha_route_causal(handle, _ptr(K), _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions),
                                   beam, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _stream(stream)),
            "zha_route_causal")
@@ -230,6 +271,8 @@ def zha_decode_causal(handle, Q: torch.Tensor, positions: torch.Tensor, beam: in
                       stream=None) -> None:
     """Causal routing + attention over each query's prefix, one launch."""
     B, Hq, nq, _ = Q.shape
+    _expect(positions, "positions", nq, _I64)
+    _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O)
     _check(lib().zha_decode_causal(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions), beam,
                                    _ptr(K), _ptr(V), scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
                                    _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_causal")
@@ -242,6 +285,7 @@ def zha_decode_buffered(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: 
     """Route over the tree of the first n_routed tokens, attend over the routed leaves and the
     buffered tokens n_routed .. n_tokens - 1, one launch."""
     B, Hq, nq, _ = Q.shape
+    _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O)
     _check(lib().zha_decode_buffered(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
                                      n_routed, n_tokens, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
                                      _ptr(O), dtype_code(O.dtype), _stream(stream)), "zha_decode_buffered")
@@ -261,6 +305,10 @@ def zha_threshold_route(handle, K: torch.Tensor, Q: torch.Tensor, tau: torch.Ten
                         tokens: torch.Tensor, count: torch.Tensor, stats: torch.Tensor | None = None,
                         stream=None) -> None:
     B, Hq, nq, _ = Q.shape
+    _expect(tau, "tau", B * Hq * nq, _F32)
+    _expect(tokens, "tokens", B * Hq * nq * int(max_tokens), _I32)
+    _expect(count, "count", B * Hq * nq, _I32)
+    _expect(stats, "stats", B * Hq * nq * 2, _I32)
     _check(lib().zha_threshold_route(handle, _ptr(K), _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(tau),
                                      max_tokens, _ptr(tokens), _ptr(count), _ptr(stats), _stream(stream)),
            "zha_threshold_route")
