@@ -11,6 +11,8 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 import bench
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -48,7 +50,6 @@ def test_reference_other_ranks_exit_quietly():
 
 def test_cuda_arm_fails_loudly_without_a_gpu():
     # no CPU fallback: without a GPU the CUDA arm exits non-zero and prints no result line
-    import pytest
     torch = pytest.importorskip("torch")
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
