@@ -147,9 +147,10 @@ zha_status zha_sparse_attn_decode(const zha_tree* tree, const void* d_Q, zha_dty
  * device array inside this library of zha_noalloc_scratch_capacity() bytes (128 KiB),
  * which every GPU that loads the library holds until the process exits.  Shapes whose
  * partials need more return ZHA_ERR_CAPACITY (use zha_sparse_attn_decode for them).
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- * with the tree's device current) and caches it; make that first call before any stream
- * capture.  No call allocates or frees device memory.  All calls share the one array and
+ * The tree's device must be current (ZHA_ERR_INVALID_ARG otherwise).  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches it for the
+ * life of the process; make that first call before any stream capture.  A cudaDeviceReset
+ * invalidates the cached address, so do not call this entry point after one.  No call allocates or frees device memory.  All calls share the one array and
  * nothing in it needs clearing between calls, so calls whose kernels overlap on the GPU
  * (other streams, other threads) race on it: order them. */
 zha_status zha_sparse_attn_decode_noalloc(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype,
@@ -278,6 +279,11 @@ long long zha_tree_unit_rows(const zha_tree* tree);               /* rows per un
 const void* zha_tree_summaries(const zha_tree* tree);
 /* Kernel launches issued through this handle since zha_tree_init (all calls). */
 long long zha_tree_launch_count(const zha_tree* tree);
+/* Copies the geometry the tree was created with into *out (bindings use it to check
+ * buffer shapes before a call).  ZHA_ERR_INVALID_ARG on a null argument. */
+zha_status zha_tree_get_desc(const zha_tree* tree, zha_tree_desc* out);
+/* The CUDA device that was current when the tree was created; -1 on a null handle. */
+int zha_tree_device(const zha_tree* tree);
 
 const char* zha_status_string(zha_status status);
 

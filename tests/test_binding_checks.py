@@ -68,3 +68,75 @@ def test_right_sizes_reach_the_device_check():
     # sizes and types right: the next refusal is the binding's device-tensor check
     with pytest.raises(ValueError, match="device tensors"):
         zha.zha_route(None, _q(), BEAM, _idx(), torch.zeros(B * HQ * NQ * BEAM, dtype=torch.float32))
+
+
+# Q, K and V against the tree's geometry.  No tree can be created without a GPU, so the
+# binding's desc getter is replaced by a fixed geometry: batch 2, 2 KV heads, d 64,
+# capacity 16 tokens, bf16 caches.
+TREE = zha.zha_tree_desc(2, 2, 64, 4, 4, 16, zha.ZHA_BF16, zha.ZHA_F32)
+HANDLE = object()
+
+
+@pytest.fixture()
+def fake_tree(monkeypatch):
+    monkeypatch.setattr(zha, "zha_tree_get_desc", lambda h: TREE)
+
+
+def _cache(dtype=torch.bfloat16, n=2 * 2 * 16 * 64):
+    return torch.zeros(n, dtype=dtype)
+
+
+def _q2(b=2, hq=4, nq=3, d=64, dtype=torch.bfloat16):
+    return torch.zeros((b, hq, nq, d), dtype=dtype)
+
+
+def _out(q):
+    return torch.zeros(q.shape, dtype=torch.bfloat16)
+
+
+def _ix(q, beam=BEAM):
+    return torch.zeros(q.shape[:3] + (beam,), dtype=torch.int32)
+
+
+def test_query_must_fit_the_tree(fake_tree):
+    for bad in (_q2(b=1), _q2(b=3), _q2(d=128)):
+        with pytest.raises(ValueError, match="does not fit the tree"):
+            zha.zha_route(HANDLE, bad, BEAM, _ix(bad))
+        with pytest.raises(ValueError, match="does not fit the tree"):
+            zha.zha_decode(HANDLE, bad, BEAM, _cache(), _cache(), 0.1, _ix(bad), _out(bad))
+        with pytest.raises(ValueError, match="does not fit the tree"):
+            zha.zha_sparse_attn_decode_noalloc(HANDLE, bad, _cache(), _cache(), _ix(bad), BEAM, 0.1, _out(bad))
+    flat = torch.zeros((2, 4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="expected \\[batch, q_heads, nq, head_dim\\]"):
+        zha.zha_route(HANDLE, flat, BEAM, torch.zeros(2 * 4 * BEAM, dtype=torch.int32))
+    with pytest.raises(ValueError, match="Q: dtype torch.float16"):
+        q = _q2(dtype=torch.float16)
+        zha.zha_route(HANDLE, q, BEAM, _ix(q))
+
+
+def test_caches_must_fit_the_tree(fake_tree):
+    q = _q2()
+    for K, V, what in ((_cache(torch.float32), _cache(), "K: dtype"), (_cache(n=100), _cache(), "K: 100"),
+                       (_cache(), _cache(n=2 * 2 * 17 * 64), "V: 4352"), (_cache(), _cache(torch.float32), "V: dtype")):
+        with pytest.raises(ValueError, match=what):
+            zha.zha_decode(HANDLE, q, BEAM, K, V, 0.1, _ix(q), _out(q))
+        with pytest.raises(ValueError, match=what):
+            zha.zha_decode_step(HANDLE, K, V, 10, q, BEAM, 0.1, _ix(q), _out(q))
+        with pytest.raises(ValueError, match=what):
+            zha.zha_sparse_attn_decode(HANDLE, q, K, V, _ix(q), BEAM, 0.1, _out(q))
+        with pytest.raises(ValueError, match=what):
+            zha.zha_decode_buffered(HANDLE, q, BEAM, K, V, 4, 9, 0.1, _ix(q), _out(q))
+    with pytest.raises(ValueError, match="K: 100"):
+        zha.zha_tree_build(HANDLE, _cache(n=100), 8)
+    with pytest.raises(ValueError, match="K: dtype"):
+        zha.zha_tree_append(HANDLE, _cache(torch.float32), 8)
+    with pytest.raises(ValueError, match="K: 100"):
+        zha.zha_route_causal(HANDLE, _cache(n=100), q, torch.zeros(3, dtype=torch.int64), BEAM, _ix(q))
+
+
+def test_fitting_buffers_reach_the_device_check(fake_tree):
+    q = _q2()
+    with pytest.raises(ValueError, match="device tensors"):
+        zha.zha_decode(HANDLE, q, BEAM, _cache(), _cache(), 0.1, _ix(q), _out(q))
+    with pytest.raises(ValueError, match="device tensors"):
+        zha.zha_tree_build(HANDLE, _cache(), 8)

@@ -67,6 +67,11 @@ extern "C" zha_status zha_sparse_attn_decode_noalloc(const zha_tree* t, const vo
   if (!aligned16(d_Q) || !aligned16(d_K) || !aligned16(d_V) || !aligned16(d_O) ||
       (reinterpret_cast<uintptr_t>(d_leaf_idx) & 3u) != 0)
     return ZHA_ERR_INVALID_ARG;
+  // The array's address is looked up (and cached) for the current device, and the kernels
+  // launch there: both must be the tree's device.
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZHA_ERR_CUDA;
+  if (dev != t->device) return ZHA_ERR_INVALID_ARG;
   const zha::AttnPlan plan = zha::plan_attention(t, q_heads, nq, beam);
   if (plan.smem_bytes > 227 * 1024) return ZHA_ERR_UNSUPPORTED;
   if (plan.scratch_bytes > kNoAllocScratchBytes) return ZHA_ERR_CAPACITY;

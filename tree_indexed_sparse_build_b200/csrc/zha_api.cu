@@ -367,6 +367,12 @@ long long zha_tree_level_offset(const zha_tree* t, int level) {
 long long zha_tree_unit_rows(const zha_tree* t) { return t ? t->unit_rows : 0; }
 const void* zha_tree_summaries(const zha_tree* t) { return t ? t->pyr : nullptr; }
 long long zha_tree_launch_count(const zha_tree* t) { return t ? t->launches : -1; }
+zha_status zha_tree_get_desc(const zha_tree* t, zha_tree_desc* out) {
+  if (!t || !out) return ZHA_ERR_INVALID_ARG;
+  *out = t->desc;
+  return ZHA_OK;
+}
+int zha_tree_device(const zha_tree* t) { return t ? t->device : -1; }
 
 const char* zha_status_string(zha_status s) {
   switch (s) {

@@ -29,6 +29,7 @@ EXPORTED = [
     "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
     "zha_decode", "zha_decode_step", "zha_route_causal", "zha_decode_causal",
     "zha_tree_radii_bytes", "zha_tree_attach_radii", "zha_threshold_route", "zha_decode_buffered",
+    "zha_tree_get_desc", "zha_tree_device",
 ]
 
 
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
             "zha_tree_unit_rows": (_LL, [_P]),
             "zha_tree_summaries": (_P, [_P]),
             "zha_tree_launch_count": (_LL, [_P]),
+            "zha_tree_get_desc": (_I, [_P, ctypes.POINTER(zha_tree_desc)]),
+            "zha_tree_device": (_I, [_P]),
             "zha_status_string": (ctypes.c_char_p, [_I]),
         }
         for name, (res, args) in sig.items():
@@ -132,6 +135,53 @@ def _expect(t: torch.Tensor | None, what: str, numel: int, dtypes: tuple) -> Non
 
 _I32, _I64, _F32 = (torch.int32,), (torch.int64,), (torch.float32,)
 _OUT = (torch.float32, torch.bfloat16)
+_TORCH_DT = {ZHA_F32: torch.float32, ZHA_BF16: torch.bfloat16}
+
+
+def zha_tree_get_desc(handle) -> zha_tree_desc:
+    d = zha_tree_desc()
+    _check(lib().zha_tree_get_desc(handle, ctypes.byref(d)), "zha_tree_get_desc")
+    return d
+
+
+def zha_tree_device(handle) -> int:
+    return int(lib().zha_tree_device(handle))
+
+
+def _check_q(handle, Q: torch.Tensor, what: str = "Q") -> None:
+    """Refuse a query tensor that does not fit the tree: the kernels size their reads of Q,
+    and their writes of every per-query output, from the tree's batch and head_dim and the
+    call's q_heads and nq, so a Q of another batch or head_dim would be read past its end.
+    (A null handle is left to the library, which refuses it.)"""
+    if handle is None:
+        return
+    d = zha_tree_get_desc(handle)
+    if Q.dim() != 4:
+        raise ValueError(f"{what}: expected [batch, q_heads, nq, head_dim], got shape {tuple(Q.shape)}")
+    if Q.dtype not in _OUT:
+        raise ValueError(f"{what}: dtype {Q.dtype}, expected torch.float32 or torch.bfloat16")
+    B, _, _, hd = Q.shape  # q_heads % kv_heads is checked by the library itself
+    if B != d.batch or hd != d.head_dim:
+        raise ValueError(f"{what}: shape {tuple(Q.shape)} does not fit the tree "
+                         f"(batch {d.batch}, head_dim {d.head_dim})")
+
+
+def _check_kv(handle, *caches) -> None:
+    """Refuse a K or V cache of another type or size than the tree's
+    [batch, kv_heads, capacity_tokens, head_dim] in kv_dtype (None entries are skipped): the
+    kernels address rows by the tree's capacity, so any other size is read past or mis-strided."""
+    if handle is None:
+        return
+    d = zha_tree_get_desc(handle)
+    n = d.batch * d.kv_heads * d.capacity_tokens * d.head_dim
+    for name, t in zip("KV", caches):
+        if t is None:
+            continue
+        if t.dtype != _TORCH_DT[d.kv_dtype]:
+            raise ValueError(f"{name}: dtype {t.dtype}, the tree's caches are {_TORCH_DT[d.kv_dtype]}")
+        if t.numel() != n:
+            raise ValueError(f"{name}: {t.numel()} elements, the tree's [batch, kv_heads, capacity, "
+                             f"head_dim] cache has {n}")
 
 
 def _route_buffers(handle, Q: torch.Tensor, beam: int, leaf_idx, leaf_score=None, trace=None,
@@ -186,16 +236,19 @@ def zha_tree_destroy(handle) -> None:
 
 
 def zha_tree_build(handle, K: torch.Tensor, seq_len: int, stream=None) -> None:
+    _check_kv(handle, K)
     _check(lib().zha_tree_build(handle, _ptr(K), seq_len, _stream(stream)), "zha_tree_build")
 
 
 def zha_tree_append(handle, K: torch.Tensor, new_seq_len: int, stream=None) -> None:
+    _check_kv(handle, K)
     _check(lib().zha_tree_append(handle, _ptr(K), new_seq_len, _stream(stream)), "zha_tree_append")
 
 
 def zha_route(handle, Q: torch.Tensor, beam: int, leaf_idx: torch.Tensor,
               leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
               stream=None) -> None:
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
     _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace)
     _check(lib().zha_route(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(leaf_idx),
@@ -209,7 +262,9 @@ def zha_attn_scratch_bytes(handle, q_heads: int, nq: int, beam: int) -> int:
 def zha_sparse_attn_decode(handle, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                            leaf_idx: torch.Tensor, beam: int, scale: float, O: torch.Tensor,
                            scratch: torch.Tensor | None = None, stream=None) -> None:
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
+    _check_kv(handle, K, V)
     _route_buffers(handle, Q, beam, leaf_idx, O=O)
     nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
     _check(lib().zha_sparse_attn_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(K),
@@ -222,7 +277,9 @@ def zha_sparse_attn_decode_noalloc(handle, Q: torch.Tensor, K: torch.Tensor, V: 
                                    leaf_idx: torch.Tensor, beam: int, scale: float,
                                    O: torch.Tensor, stream=None) -> None:
     """zha_sparse_attn_decode with the library's own fixed scratch (no caller buffer)."""
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
+    _check_kv(handle, K, V)
     _route_buffers(handle, Q, beam, leaf_idx, O=O)
     _check(lib().zha_sparse_attn_decode_noalloc(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq,
                                                 _ptr(K), _ptr(V), _ptr(leaf_idx), beam, scale,
@@ -234,7 +291,9 @@ def zha_decode(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: torch.Ten
                leaf_idx: torch.Tensor, O: torch.Tensor, leaf_score: torch.Tensor | None = None,
                trace: torch.Tensor | None = None, stream=None) -> None:
     """Route + attention in one call (one launch when the levels fit shared memory)."""
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
+    _check_kv(handle, K, V)
     _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O)
     _check(lib().zha_decode(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
                             scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _ptr(O),
@@ -246,7 +305,9 @@ def zha_decode_step(handle, K: torch.Tensor, V: torch.Tensor, new_seq_len: int, 
                     leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
                     stream=None) -> None:
     """Append up to new_seq_len, then route + attention (one launch for one-leaf appends)."""
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
+    _check_kv(handle, K, V)
     _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O, appending=True)
     _check(lib().zha_decode_step(handle, _ptr(K), _ptr(V), new_seq_len, _ptr(Q), dtype_code(Q.dtype),
                                  Hq, nq, beam, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
@@ -257,8 +318,10 @@ def zha_route_causal(handle, K: torch.Tensor, Q: torch.Tensor, positions: torch.
                      leaf_idx: torch.Tensor, leaf_score: torch.Tensor | None = None,
                      trace: torch.Tensor | None = None, stream=None) -> None:
     """Query i of every head routes over the tree of tokens 0 .. positions[i] (int64, device)."""
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
     _expect(positions, "positions", nq, _I64)
+    _check_kv(handle, K)
     _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace)
     _check(lib().zha_route_causal(handle, _ptr(K), _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions),
                                   beam, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace), _stream(stream)),
@@ -270,8 +333,10 @@ def zha_decode_causal(handle, Q: torch.Tensor, positions: torch.Tensor, beam: in
                       leaf_score: torch.Tensor | None = None, trace: torch.Tensor | None = None,
                       stream=None) -> None:
     """Causal routing + attention over each query's prefix, one launch."""
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
     _expect(positions, "positions", nq, _I64)
+    _check_kv(handle, K, V)
     _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O)
     _check(lib().zha_decode_causal(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, _ptr(positions), beam,
                                    _ptr(K), _ptr(V), scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
@@ -284,7 +349,9 @@ def zha_decode_buffered(handle, Q: torch.Tensor, beam: int, K: torch.Tensor, V: 
                         stream=None) -> None:
     """Route over the tree of the first n_routed tokens, attend over the routed leaves and the
     buffered tokens n_routed .. n_tokens - 1, one launch."""
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
+    _check_kv(handle, K, V)
     _route_buffers(handle, Q, beam, leaf_idx, leaf_score, trace, O)
     _check(lib().zha_decode_buffered(handle, _ptr(Q), dtype_code(Q.dtype), Hq, nq, beam, _ptr(K), _ptr(V),
                                      n_routed, n_tokens, scale, _ptr(leaf_idx), _ptr(leaf_score), _ptr(trace),
@@ -296,6 +363,7 @@ def zha_tree_radii_bytes(handle) -> int:
 
 
 def zha_tree_attach_radii(handle, radii: torch.Tensor | None, K: torch.Tensor | None, stream=None) -> None:
+    _check_kv(handle, K)
     nbytes = 0 if radii is None else radii.numel() * radii.element_size()
     _check(lib().zha_tree_attach_radii(handle, _ptr(radii), nbytes, _ptr(K), _stream(stream)),
            "zha_tree_attach_radii")
@@ -304,7 +372,9 @@ def zha_tree_attach_radii(handle, radii: torch.Tensor | None, K: torch.Tensor | 
 def zha_threshold_route(handle, K: torch.Tensor, Q: torch.Tensor, tau: torch.Tensor, max_tokens: int,
                         tokens: torch.Tensor, count: torch.Tensor, stats: torch.Tensor | None = None,
                         stream=None) -> None:
+    _check_q(handle, Q)
     B, Hq, nq, _ = Q.shape
+    _check_kv(handle, K)
     _expect(tau, "tau", B * Hq * nq, _F32)
     _expect(tokens, "tokens", B * Hq * nq * int(max_tokens), _I32)
     _expect(count, "count", B * Hq * nq, _I32)
