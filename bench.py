@@ -352,7 +352,11 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
         for k in pb:
             acc[k] += pb[k] / K
     del graphs, graphs2
-    res = {"step_ms": t_step, "append_ms": t_app, "decode_ms": t_dec,
+    # the last kernel-pass step (tokens N + W + 2K) against the oracle, first and last unit
+    sl = 2 * K - 1
+    par = parity_sample(w, Qs[W + sl], Kn, Vn, N + W + sl + 1, idx_n[sl], tr_n[sl], O[sl].float().cpu().numpy(),
+                        (0, w.units - 1), summary="bf16" if sum_bytes == 2 else "f64")
+    res = {"parity": par, "step_ms": t_step, "append_ms": t_app, "decode_ms": t_dec,
            "queries_per_step": B * Hq * nq, "launches_per_step": launches, "clocks": smp.summary(),
            **acc}
     if not e2e:
@@ -543,6 +547,7 @@ def run_1m(W, K, rank, dev, flush, eager=False, summary_dtype=None):
     Kn = synth.keys(w, Q=Qn)
     Vn = synth.values(w)
     Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
+    K0, V0 = np.ascontiguousarray(Kn[:1, :1]), np.ascontiguousarray(Vn[:1, :1])  # unit 0, for parity
     del Kn, Vn
     d, beam, N = w.head_dim, w.beam, w.seq_len
     summary_dtype = summary_dtype or torch.float32
@@ -605,7 +610,9 @@ def run_1m(W, K, rank, dev, flush, eager=False, summary_dtype=None):
                         w.branching, d, 2, w.group, 2, sum_bytes=sum_bytes)
         if mode == "throughput":  # the needles were planted for these 64 queries per head
             out["needle_recall"] = needle_recall(w, Qn, idx.cpu().numpy())
-        out[mode] = {"route_ms": tr_ms, "attend_ms": at_ms, "step_ms": step_ms,
+        par = parity_sample(w, Qn[:, :, :nq], K0, V0, N, idx.cpu().numpy(), tr.cpu().numpy(),
+                            O.float().cpu().numpy(), (0,), summary="bf16" if sum_bytes == 2 else "f64")
+        out[mode] = {"route_ms": tr_ms, "attend_ms": at_ms, "step_ms": step_ms, "parity": par,
                      "queries_per_step": w.batch * w.q_heads * nq, "launches_per_step": launches, **pb}
         del runs
     out["dense_bytes_per_step"] = int(2 * N * d * 2 * w.kv_heads * w.batch)
@@ -625,7 +632,6 @@ def run_build_256k(W, K, dev, flush):
     Kn = synth.keys(w)
     Vn = synth.values(w)
     Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
-    del Kn, Vn
     d, N, cap = w.head_dim, w.seq_len, w.capacity
     tree = zha.Tree(w.batch, w.kv_heads, d, w.branching, w.leaf_block, cap, torch.bfloat16)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
@@ -641,7 +647,7 @@ def run_build_256k(W, K, dev, flush):
         ev[3].record()
         flush.zero_()
         ev[4].record()
-        tree.decode(Qd, Kd, Vd, w.beam, w.scale)
+        last = tree.decode(Qd, Kd, Vd, w.beam, w.scale)
         ev[5].record()
         torch.cuda.synchronize()
         if it >= W:
@@ -652,7 +658,12 @@ def run_build_256k(W, K, dev, flush):
     rows = sum(counts)
     build_bytes = N * d * 2 * w.units + rows * d * 4 * w.units
     q = w.batch * w.q_heads * w.nq
-    res = {"build_ms": float(np.mean(build_ms)), "build_bytes": int(build_bytes),
+    O, idx = last[0], last[1]
+    par = parity_sample(w, Qn, Kn, Vn, cap, idx.cpu().numpy(), None, O.float().cpu().numpy(),
+                        (0, w.units - 1),
+                        gpu_levels=lambda u: [tree.level(l)[u].float().cpu().numpy() for l in range(tree.levels + 1)])
+    del Kn, Vn
+    res = {"parity": par, "build_ms": float(np.mean(build_ms)), "build_bytes": int(build_bytes),
            "build_gbs": build_bytes / (np.mean(build_ms) * 1e-3) / 1e9,
            "append_4096_ms": float(np.mean(append_ms)), "levels_after_append": tree.levels,
            "route_attend_ms": float(np.mean(ra_ms)), "queries": q,
@@ -820,14 +831,158 @@ def run_profile_case(case: str, W: int, K: int):
     return {"case": case, "queries": w.batch * w.q_heads * nq, "zha_decode_ms": float(np.mean(ms))}
 
 
+# ----------------------------------------------------------------------------- parity sample
+
+def parity_sample(w, Q, K, V, N, idx, trace, O, units, summary="f64", gpu_levels=None):
+    """A sampled check of one call's results against the fp64 oracle, reported (not raised).
+
+    Per sampled (batch, KV head) unit: the oracle's tree over tokens [0, N) (fp64 summaries,
+    or bf16-stored ones with summary="bf16"), its beam descent for every query of the unit,
+    and exact attention over the leaves the GPU selected.  A query is well-conditioned when
+    its fp64 margins between the beam-th and next score exceed 1e-3 |score| at every level;
+    its leaves and per-level survivors must then equal the oracle's (counted in "exact").
+    The other queries' leaf sets may differ and are counted as mismatches.  Q: stored queries
+    [B, Hq, nq, d]; K, V: stored caches [B, H_kv, >= N, d]; idx, trace, O: the call's outputs
+    as numpy arrays (trace may be None; O as floats).  gpu_levels(unit), when given, returns
+    the GPU tree's levels of that unit (numpy, leaves first); each node must then be within
+    1e-6 normwise relative error of the oracle's (bit-exact for bf16-stored summaries)."""
+    import oracle
+    from tree_indexed_sparse_build_b200 import synth
+
+    t0 = time.perf_counter()
+    Q64 = synth.to_f64(Q)
+    O64 = np.asarray(O, dtype=np.float64)
+    g = w.group
+    wc = exact = ill = ill_mis = n = 0
+    max_abs = max_rel = 0.0
+    sum_err, sum_ok = 0.0, True
+    for u in units:
+        b, h = divmod(u, w.kv_heads)
+        ot = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching, summary=summary).build(K[b, h], N)
+        if gpu_levels is not None:
+            got_levels = gpu_levels(u)
+            sum_ok &= len(got_levels) == len(ot.levels)
+            for got, ref in zip(got_levels, ot.levels):
+                got = np.asarray(got, dtype=np.float64)
+                sum_ok &= got.shape == ref.shape
+                if got.shape != ref.shape:
+                    continue
+                if summary == "bf16":
+                    sum_ok &= bool(np.array_equal(got, ref))
+                den = np.linalg.norm(ref, axis=-1)
+                rel = np.linalg.norm(got - ref, axis=-1) / np.where(den > 0, den, 1.0)
+                sum_err = max(sum_err, float(rel.max()) if rel.size else 0.0)
+        flat = ot.flat()
+        for hq in range(h * g, (h + 1) * g):
+            res = ot.route(Q64[b, hq], w.beam, flat=flat)
+            ok = oracle.well_conditioned(res["bounds"])
+            got = idx[b, hq]
+            same = (got == res["leaves"]).all(axis=-1)
+            if trace is not None:
+                same &= (trace[b, hq] == res["survivors"]).all(axis=(-2, -1))
+            n += got.shape[0]
+            wc += int(ok.sum())
+            exact += int((same & ok).sum())
+            ill += int((~ok).sum())
+            ill_mis += int((~same & ~ok).sum())
+            for i in range(got.shape[0]):
+                ref, _ = oracle.attend(Q64[b, hq, i], K[b, h], V[b, h], N, w.leaf_block,
+                                       got[i].astype(np.int64), w.scale)
+                err = O64[b, hq, i] - ref
+                max_abs = max(max_abs, float(np.abs(err).max()))
+                max_rel = max(max_rel, float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300)))
+    fp32 = w.kv_dtype == "f32" and w.out_dtype == "f32"
+    attn_ok = max_abs <= 1e-5 if fp32 else max_rel <= 2e-2
+    extra = {}
+    if gpu_levels is not None:
+        sum_ok &= sum_err <= 1e-6
+        extra = {"summary_max_rel_err": sum_err, "summaries_ok": bool(sum_ok)}
+        attn_ok &= bool(sum_ok)
+    return {**extra, "units": list(units), "summaries": "bf16" if summary == "bf16" else "fp32", "queries": n,
+            "well_conditioned": wc, "exact": exact, "ill_conditioned": ill, "ill_mismatch": ill_mis,
+            "ill_mismatch_rate": ill_mis / max(n, 1), "attn_max_abs": max_abs, "attn_max_rel_l2": max_rel,
+            "attn_bar": "max-abs 1e-5" if fp32 else "rel L2 2e-2",
+            "pass": bool(exact == wc and attn_ok), "oracle_s": time.perf_counter() - t0}
+
+
+def parity_brief(p) -> str:
+    """One short line of a parity_sample result."""
+    if not p:
+        return "not checked"
+    err = f"abs {p['attn_max_abs']:.1e}" if p["attn_bar"].startswith("max") else f"rl2 {p['attn_max_rel_l2']:.1e}"
+    return (f"{'ok' if p['pass'] else 'FAIL'} {p['exact']}/{p['well_conditioned']} exact, "
+            f"ill {p['ill_mismatch']}/{p['ill_conditioned']} differ, {err}")
+
+
+# ----------------------------------------------------------------------------- small workloads
+
+def run_small(name, W, K, dev, flush):
+    """One zha_decode call (route + attention, one launch) over a tree built on the workload's
+    cache, replayed from a CUDA graph with start and end events, L2 flushed between calls:
+    tiny_fp32 (1,024 fp32 tokens, 16 queries, fp32 output) and gqa_32k (one decode step: 8 x
+    32 query heads, one query each, over 32,768 bf16 tokens)."""
+    import torch
+    from tree_indexed_sparse_build_b200 import synth, workloads, zha
+
+    w = workloads.get(name)
+    Qn = synth.queries(w)
+    Kn = synth.keys(w, Q=Qn if w.needles else None)
+    Vn = synth.values(w)
+    Kd, Vd, Qd = synth.to_torch(Kn, dev), synth.to_torch(Vn, dev), synth.to_torch(Qn, dev)
+    tdt = torch.float32 if w.kv_dtype == "f32" else torch.bfloat16
+    odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    d, N, beam = w.head_dim, w.seq_len, w.beam
+    tree = zha.Tree(w.batch, w.kv_heads, d, w.branching, w.leaf_block, N, tdt)
+    tree.build(Kd, N)
+    idx = torch.empty((w.batch, w.q_heads, w.nq, beam), dtype=torch.int32, device=dev)
+    tr = torch.empty((w.batch, w.q_heads, w.nq, tree.levels, beam), dtype=torch.int32, device=dev)
+    O = torch.empty((w.batch, w.q_heads, w.nq, d), dtype=odt, device=dev)
+    e = _graph_events(2)
+    g = torch.cuda.CUDAGraph()
+    l0 = tree.launches
+    with torch.cuda.graph(g, stream=torch.cuda.Stream(), capture_error_mode="thread_local"):
+        e[0].record()
+        zha.zha_decode(tree.handle, Qd, beam, Kd, Vd, w.scale, idx, O, None, tr)
+        e[1].record()
+    launches = tree.launches - l0
+    for _ in range(W):
+        g.replay()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(K):
+        flush.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        ms.append(e[0].elapsed_time(e[1]))
+    assert tree.check() == zha.ZHA_OK, f"device error word set during {name}"
+    kvb = 4 if w.kv_dtype == "f32" else 2
+    ob = 4 if w.out_dtype == "f32" else 2
+    idx_n, tr_n = idx.cpu().numpy(), tr.cpu().numpy()
+    pb = path_bytes(idx_n, tr_n, level_counts(N, w.leaf_block, w.branching), N, w.leaf_block,
+                    w.branching, d, kvb, w.group, ob)
+    t = float(np.mean(ms))
+    q = w.batch * w.q_heads * w.nq
+    peak, _ = hbm_peak()
+    byts = pb["route_bytes"] + pb["attend_bytes"]
+    units = range(w.units) if w.units <= 8 else range(0, w.units, w.units // 8)
+    par = parity_sample(w, Qn, Kn, Vn, N, idx_n, tr_n, O.float().cpu().numpy(), units)
+    del g
+    tree.close()
+    return {"call": "zha_decode (route + attention, one launch)", "queries": q, "ms": t,
+            "qps": q / (t * 1e-3), "bytes": int(byts), "gbs": byts / (t * 1e-3) / 1e9,
+            "frac_of_peak": byts / (t * 1e-3) / 1e9 / peak, "keys_per_query": pb["keys_per_query"],
+            "summaries_per_query": pb["summaries_per_query"], "launches": launches, "parity": par}
+
+
 # ----------------------------------------------------------------------------- oracle arm
 
 def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), warmup: int = 0,
                          start=None):
     """Time the fp64 oracle on decode steps of `w` for a few units (single thread).
 
-    Setup (not timed): each sampled unit's tree over the first N tokens.  Timed: per step
-    and unit, append one token, route the unit's query heads, attend each.
+    Setup (not timed): each sampled unit's tree over the first N tokens and every step's
+    queries.  Timed: per step and unit, append one token, route the unit's query heads,
+    attend each.
     """
     import oracle
     from tree_indexed_sparse_build_b200 import synth
@@ -840,8 +995,11 @@ def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), 
     trees = {u: oracle.OracleTree(w.head_dim, w.leaf_block, w.branching).build(
         Kn[u // w.kv_heads, u % w.kv_heads], N) for u in units}
 
+    # every step's queries are drawn before the clock starts (drawing them is not oracle work)
+    Qsteps = [synth.queries(w, step=s) for s in range(warmup + max_steps)]
+
     def step(s):
-        q = synth.queries(w, step=s)
+        q = Qsteps[s]
         n = 0
         for u in units:
             b, h = divmod(u, w.kv_heads)
@@ -872,34 +1030,107 @@ def oracle_decode_sample(w, seconds: float, max_steps: int, units=(0, 1, 2, 3), 
             "per_step_s": per_step}
 
 
-def _host_parallel_worker(i, w, seconds, max_steps, start, out):
-    """One process of oracle_host_parallel: a single-unit replica of w (its own seed)."""
-    wi = w.with_(batch=1, kv_heads=1, q_heads=w.group, seed=w.seed + 104729 * (i + 1))
-    r = oracle_decode_sample(wi, seconds=seconds, max_steps=max_steps, units=(0,), start=start)
-    out.put((i, r["queries"], r["seconds"], r["steps"]))
+def oracle_route_attend_sample(w, seconds: float, nq: int, units=(0,), N=None, start=None):
+    """Time the fp64 oracle's route + attention over prebuilt trees (single thread).
+
+    Setup (not timed): the sampled units' caches, their trees over tokens [0, N) (N defaults to
+    the workload's), the stacked levels the descent reads, and nq queries per query head.
+    Timed: every query of the units' heads routed and attended, unit after unit, repeated
+    until `seconds` have passed (at least one pass)."""
+    import oracle
+    from tree_indexed_sparse_build_b200 import synth
+
+    N = N or w.seq_len
+    units = list(units)
+    Qn = synth.queries(w, nq=nq)
+    Kn = synth.keys(w, capacity=N, Q=Qn if w.needles else None, units=units)
+    Vn = synth.values(w, capacity=N, units=units)
+    Q64 = synth.to_f64(Qn)
+    trees, flats = {}, {}
+    for u in units:
+        b, h = divmod(u, w.kv_heads)
+        trees[u] = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching).build(Kn[b, h], N)
+        flats[u] = trees[u].flat()
+    g = w.group
+    if start is not None:  # processes of a host-parallel run begin their timed work together
+        start.wait()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        for u in units:
+            b, h = divmod(u, w.kv_heads)
+            for hq in range(h * g, (h + 1) * g):
+                res = trees[u].route(Q64[b, hq], w.beam, flat=flats[u])
+                for i in range(nq):
+                    oracle.attend(Q64[b, hq, i], Kn[b, h], Vn[b, h], N, w.leaf_block, res["leaves"][i], w.scale)
+                n += nq
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n / el, "queries": n, "seconds": el, "units": len(units)}
 
 
-def oracle_host_parallel(w, seconds: float, max_steps: int):
-    """The fp64 oracle on every host core: one process per core (started with spawn, so it
-    is safe after CUDA initialisation), each a single-threaded oracle instance routing one
-    (batch, KV head) unit of w's shape with its own seed.  Setup (the unit's tree over the
-    first N tokens) is untimed; all processes then start together and run decode steps;
-    rate = all processes' queries / the slowest process's time."""
+def oracle_build_sample(w, N_build: int, N_final: int):
+    """The fp64 oracle's build of one unit over N_build tokens and its append up to N_final
+    (single thread): seconds of each."""
+    import oracle
+    from tree_indexed_sparse_build_b200 import synth
+
+    wi = w.with_(batch=1, kv_heads=1, q_heads=w.group)
+    Kn = synth.keys(wi, capacity=N_final)
+    t0 = time.perf_counter()
+    ot = oracle.OracleTree(w.head_dim, w.leaf_block, w.branching).build(Kn[0, 0], N_build)
+    t1 = time.perf_counter()
+    ot.append(Kn[0, 0], N_final)
+    t2 = time.perf_counter()
+    return {"build_s": t1 - t0, "append_s": t2 - t1}
+
+
+def _replica(w, i):
+    """A single-unit copy of workload w's shape with its own seed (host-parallel process i)."""
+    return w.with_(batch=1, kv_heads=1, q_heads=w.group, seed=w.seed + 104729 * (i + 1))
+
+
+def _host_parallel_worker(i, jobs, start, out):
+    """One process of oracle_host_parallel: every job in turn on its own single-unit replica,
+    each started together with the other processes."""
+    for j, (kind, w, nq, N, seconds, max_steps) in enumerate(jobs):
+        wi = _replica(w, i)
+        try:
+            if kind == "decode":
+                r = oracle_decode_sample(wi, seconds=seconds, max_steps=max_steps, units=(0,), start=start)
+            else:
+                r = oracle_route_attend_sample(wi, seconds, nq, units=(0,), N=N, start=start)
+            out.put((j, i, r["queries"], r["seconds"]))
+        except Exception as e:  # report and keep the barrier count right for the others
+            out.put((j, i, None, repr(e)))
+            try:
+                start.wait()
+            except Exception:
+                pass
+
+
+def oracle_host_parallel(jobs, timeout_s: float = 300.0):
+    """The fp64 oracle on every host core: one process per core (spawned, so safe after CUDA
+    initialisation), each a single-threaded oracle working on its own single-unit replica of
+    each job's workload.  jobs: (kind, workload, nq, N, seconds, max_steps) with kind "decode"
+    (append + route + attend steps) or "route_attend" (prebuilt tree).  Setup is untimed; the
+    processes start each job's timed work together.  Per job: rate = all processes' queries /
+    the slowest process's time."""
     import multiprocessing as mp
+    import queue as _queue
 
     cores = os.cpu_count() or 1
     n = min(cores, 64)
     ctx = mp.get_context("spawn")
-    start = ctx.Barrier(n)
+    start = ctx.Barrier(n, timeout=timeout_s)
     out = ctx.Queue()
-    procs = [ctx.Process(target=_host_parallel_worker, args=(i, w, seconds, max_steps, start, out))
-             for i in range(n)]
+    procs = [ctx.Process(target=_host_parallel_worker, args=(i, jobs, start, out)) for i in range(n)]
     for p in procs:
         p.start()
     res = []
-    deadline = time.time() + 20 * seconds + 120
-    import queue as _queue
-    while len(res) < n:
+    deadline = time.time() + timeout_s + sum(j[4] for j in jobs) * 2
+    while len(res) < n * len(jobs):
         try:
             res.append(out.get(timeout=5))
         except _queue.Empty:
@@ -910,10 +1141,17 @@ def oracle_host_parallel(w, seconds: float, max_steps: int):
                 raise RuntimeError("host-parallel oracle processes failed or timed out")
     for p in procs:
         p.join(timeout=60)
-    q = sum(r[1] for r in res)
-    t = max(r[2] for r in res)
-    return {"value": q / t, "queries": q, "seconds": t, "threads": n, "cores": cores,
-            "steps": min(r[3] for r in res)}
+    per_job = []
+    for j in range(len(jobs)):
+        rows = [r for r in res if r[0] == j]
+        bad = [r for r in rows if r[2] is None]
+        if bad:
+            per_job.append({"value": None, "error": bad[0][3]})
+            continue
+        q = sum(r[2] for r in rows)
+        t = max(r[3] for r in rows)
+        per_job.append({"value": q / t, "queries": q, "seconds": t, "processes": n, "cores": cores})
+    return per_job
 
 
 # ----------------------------------------------------------------------------- main
@@ -1049,6 +1287,8 @@ def main():
         "clocks": r["clocks"],
     }
 
+    line["parity"] = r["parity"]
+
     def ctx_1m(m):
         one = {}
         for mode in ("throughput", "single"):
@@ -1063,7 +1303,7 @@ def main():
                          "attend_gbs": x["attend_bytes"] / (x["attend_ms"].mean() * 1e-3) / 1e9,
                          "bytes_per_step": int(byts), "keys_per_query": x["keys_per_query"],
                          "summaries_per_query": x["summaries_per_query"],
-                         "queries_per_step": x["queries_per_step"]}
+                         "queries_per_step": x["queries_per_step"], "parity": x["parity"]}
         one["dense_bytes_per_step"] = m["dense_bytes_per_step"]
         one["workload"] = ("deep_1m: 1 x 8 KV heads x 64 query heads, d 128, 1,048,576 bf16 tokens, "
                            "b 8, leaf block 4, beam 8; throughput = 64 queries per head per step")
@@ -1082,13 +1322,21 @@ def main():
             "decode_kernel_ms": float(rb["decode_ms"].mean()),
             "decode_kernel_gbs": dec_b / (float(rb["decode_ms"].mean()) * 1e-3) / 1e9,
             "decode_kernel_bytes": int(dec_b), "route_bytes": int(rb["route_bytes"]),
-            "summaries_per_query": rb["summaries_per_query"], "clocks": rb["clocks"]}
+            "summaries_per_query": rb["summaries_per_query"], "clocks": rb["clocks"], "parity": rb["parity"]}
 
         # the same 128K steps with an append buffer (decode reads the buffer; commits overlap)
         bu = run_buffered(w, W, K, rank, dev, flush, eager=args.eager)
         line["decode_128k_buffered"] = {
             "qps": ranks.weak_scaling_rate(w.batch * w.q_heads, world, max_over_ranks(bu["ms_per_step"])), **bu,
             "call": "zha_decode_buffered per step; zha_tree_append of 2 leaves on a second stream when full"}
+
+    if not args.no_build and rank == 0:
+        line["tiny_fp32"] = run_small("tiny_fp32", W, K, dev, flush)
+        line["gqa_32k"] = run_small("gqa_32k", W, K, dev, flush)
+        line["build_256k"] = run_build_256k(W, K, dev, flush)
+        line["causal"] = run_causal(W, min(K, 10), dev, flush)
+        line["needle_recall"] = run_needles(dev)
+        line["threshold"] = run_threshold(W, min(K, 10), dev, flush)
 
     if not args.no_1m:
         line["ctx_1m"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager))
@@ -1098,12 +1346,7 @@ def main():
             line["ctx_1m_bf16_summaries"] = ctx_1m(run_1m(W, K, rank, dev, flush, eager=args.eager,
                                                           summary_dtype=torch.bfloat16))
 
-    if not args.no_build and rank == 0:
-        line["build_256k"] = run_build_256k(W, K, dev, flush)
-        line["causal"] = run_causal(W, min(K, 10), dev, flush)
-        line["needle_recall"] = run_needles(dev)
-        line["threshold"] = run_threshold(W, min(K, 10), dev, flush)
-
+    oracle_1c, oracle_hp = {}, {}
     if rank == 0 and world == 1:
         try:
             cb = oracle_decode_sample(w, seconds=args.cpu_seconds, max_steps=64,
@@ -1112,24 +1355,98 @@ def main():
                                     "sample": f"{cb['units']} (batch, KV head) unit(s) x {cb['steps']} "
                                               f"decode steps x {w.group} query heads of decode_128k, "
                                               "single-threaded fp64 C oracle"}
+            oracle_1c["decode_128k"] = cb["value"]
         except Exception as e:  # the baseline must never sink the GPU number
             line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle",
                                     "sample": f"failed: {e}"}
         if args.cpu_seconds > 0:
+            sec = max(1.0, args.cpu_seconds / 5)
+            from tree_indexed_sparse_build_b200 import workloads as _wl
+            ra_jobs = {"tiny_fp32": (_wl.get("tiny_fp32"), 16, None),
+                       "gqa_32k": (_wl.get("gqa_32k"), 1, None),
+                       "deep_1m": (_wl.get("deep_1m"), _wl.THROUGHPUT_NQ, None),
+                       "build_256k": (_wl.get("build_256k"), 64, _wl.get("build_256k").capacity)}
+            detail = {}
+            for name, (wj, nqj, Nj) in ra_jobs.items():
+                try:
+                    r1 = oracle_route_attend_sample(wj, sec, nqj, units=(0,), N=Nj)
+                    oracle_1c[name] = r1["value"]
+                    detail[name] = {"qps": r1["value"], "queries": r1["queries"], "seconds": r1["seconds"]}
+                except Exception as e:
+                    detail[name] = {"qps": None, "error": repr(e)}
             try:
-                hp = oracle_host_parallel(w, seconds=args.cpu_seconds, max_steps=64)
+                wb = _wl.get("build_256k")
+                bs = oracle_build_sample(wb, wb.seq_len, wb.capacity)
+                rows = sum(level_counts(wb.seq_len, wb.leaf_block, wb.branching))
+                detail["build_256k"].update({"build_s_per_unit": bs["build_s"], "append_4096_s_per_unit": bs["append_s"],
+                                             "build_gbs": (wb.seq_len * wb.head_dim * 2 + rows * wb.head_dim * 4)
+                                             / bs["build_s"] / 1e9})
+            except Exception as e:
+                detail["build_256k"]["build_error"] = repr(e)
+            line["oracle_1core"] = {"kind": "oracle", "cores": 1, "seconds_per_config": sec,
+                                    "what": "route + attention of every query of one (batch, KV head) unit over "
+                                            "its prebuilt tree (decode_128k: cpu_baseline's decode steps)",
+                                    **detail}
+            try:
+                jobs = [("route_attend", _wl.get("tiny_fp32"), 16, None, sec, 0),
+                        ("route_attend", _wl.get("gqa_32k"), 1, None, sec, 0),
+                        ("decode", w, 1, None, sec, 64),
+                        ("route_attend", _wl.get("deep_1m"), _wl.THROUGHPUT_NQ, None, sec, 0),
+                        ("route_attend", _wl.get("build_256k"), 64, _wl.get("build_256k").capacity, sec, 0)]
+                names = ["tiny_fp32", "gqa_32k", "decode_128k", "deep_1m", "build_256k"]
+                hp = oracle_host_parallel(jobs)
+                oracle_hp = {n: h.get("value") for n, h in zip(names, hp)}
                 line["cpu_baseline_host_parallel"] = {
-                    "value": hp["value"], "unit": UNIT, "cores": hp["threads"], "host_cores": hp["cores"],
-                    "kind": "oracle",
-                    "sample": f"{hp['threads']} processes, each one (batch, KV head) unit of "
-                              f"decode_128k's shape with its own seed, single-threaded fp64 C oracle, "
-                              f">= {hp['steps']} decode steps each"}
+                    "value": hp[2].get("value"), "unit": UNIT, "cores": hp[2].get("processes"),
+                    "host_cores": hp[2].get("cores"), "kind": "oracle",
+                    "sample": "one spawned process per host core, each a single-threaded fp64 C oracle on its "
+                              "own single-unit replica (own seed) of each workload; value = decode_128k",
+                    "per_config": dict(zip(names, hp))}
             except Exception as e:
                 line["cpu_baseline_host_parallel"] = {"value": None, "sample": f"failed: {e}"}
+
     if rank == 0:
+        line["configs"] = config_summary(line, oracle_1c, oracle_hp)
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
+
+
+def config_summary(line, oracle_1c, oracle_hp):
+    """The five workloads in one short object (it ends the JSON line): GPU queries/s, time per
+    call, fraction of the measured HBM peak on algorithmic bytes, keys read per query, the
+    parity sample in one phrase, and the oracle's queries/s on 1 core and on every host core."""
+    def r(x, n=3):
+        return None if x is None else float(f"{x:.{n}g}")
+
+    out = {}
+    o1, oh = oracle_1c or {}, oracle_hp or {}
+    for name in ("tiny_fp32", "gqa_32k"):
+        x = line.get(name)
+        if x:
+            out[name] = {"qps": r(x["qps"]), "us": r(x["ms"] * 1e3), "frac": r(x["frac_of_peak"], 2),
+                         "keys_q": r(x["keys_per_query"]), "parity": parity_brief(x["parity"]),
+                         "oracle_qps": [r(o1.get(name)), r(oh.get(name))]}
+    ro = line.get("roofline", {})
+    out["decode_128k"] = {"qps": r(line.get("value")), "us": r(line.get("ms_per_step", 0) * 1e3),
+                          "frac": r(ro.get("frac"), 2), "keys_q": r(line.get("keys_per_query")),
+                          "parity": parity_brief(line.get("parity")),
+                          "oracle_qps": [r(o1.get("decode_128k")), r(oh.get("decode_128k"))]}
+    for key, tag in (("ctx_1m", "deep_1m"), ("ctx_1m_bf16_summaries", "deep_1m_bf16sum")):
+        x = line.get(key)
+        if x:
+            t, s1 = x["throughput"], x["single"]
+            out[tag] = {"qps": r(t["qps"]), "us": r(t["ms_per_step"] * 1e3), "frac": r(t["frac_of_peak"], 2),
+                        "single_us": r(s1["ms_per_step"] * 1e3), "keys_q": r(t["keys_per_query"]),
+                        "parity": parity_brief(t["parity"])}
+            if tag == "deep_1m":
+                out[tag]["oracle_qps"] = [r(o1.get("deep_1m")), r(oh.get("deep_1m"))]
+    x = line.get("build_256k")
+    if x:
+        out["build_256k"] = {"build_gbs": r(x["build_gbs"]), "append_us": r(x["append_4096_ms"] * 1e3),
+                             "qps": r(x["qps"]), "parity": parity_brief(x.get("parity")),
+                             "oracle_qps": [r(o1.get("build_256k")), r(oh.get("build_256k"))]}
+    return out
 
 
 if __name__ == "__main__":
