@@ -122,19 +122,17 @@ __global__ void __launch_bounds__(kRouteMaxWarps * 32) route_reg_kernel(const Ro
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        float s = 0.f;
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         if (node[u] >= 0) {
 #pragma unroll
           for (int j = 0; j < NJ; ++j) {
             float f[EPC];
             Vec16<TS>::to_f32(v[u][j], f);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) s = fmaf(q[EPC * j + e], f[e], s);
+            for (int e = 0; e < EPC; e += 4) score_fma(q + EPC * j + e, f + e, acc0, acc1);
           }
         }
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        const float s = score_reduce8(acc0, acc1);
         const int k = k0 + 4 * u + grp;
         if (l8 == 0 && k < C) keys[k] = route_key(s, node[u]);
       }
@@ -321,6 +319,12 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
   const long long cmax = a.cmax;
   cudaError_t e;
 
+  // Many queries: one warp per query, rows loaded into registers.
+  if (a.total_queries > 2LL * t->sms && route_warp_fits(t, a.cmax, beam)) {
+    e = launch_route_warp(t, a, false, stream);
+    ++t->launches;
+    return e;
+  }
   a.rows_bytes = (int)route_rows_bytes(D, a.cmax, sum_bytes(t));
   // Staged kernel when a query's widest level fits in shared memory.
   const size_t per_query = route_smem_layout(D, a.cmax, beam, a.rows_bytes, 0).total;
@@ -369,7 +373,7 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
 // call is fused only when the query's tokens then fit in at most two stages; otherwise
 // fused = false and the route and the attention run as two launches.  Stages hold a
 // multiple of 16 tokens (the attention's rounds), at least 16.
-DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
+DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam, bool allow_warp) {
   DecodePlan p{};
   const int D = t->desc.head_dim;
   const int row = D * (t->desc.kv_dtype == ZHA_BF16 ? 2 : 4);
@@ -380,6 +384,11 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam) {
     cmax = std::max(cmax, std::min(std::min((long long)beam, t->n[l + 1]) * t->desc.branching, t->n[l]));
   const long long tokens = std::min((long long)beam * t->desc.leaf_block, t->N);
   const size_t route_rows = route_rows_bytes(D, (int)cmax, sum_bytes(t));
+  if (allow_warp && !wide && route_warp_fits(t, (int)cmax, beam)) {  // one warp per query (route_warp.cu)
+    p.warp = true;
+    p.fused = true;
+    return p;
+  }
   if (!wide) {
     p.nbuf = 2;
     p.rows_bytes = std::max(route_rows, (size_t)4 * 16 * row);  // two stages of 16 tokens at least
@@ -420,6 +429,13 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
   a.lb = t->desc.leaf_block;
   a.N = t->N;
   a.qk_scale = scale * 1.4426950408889634f;
+  a.O = d_O;
+  a.o_bf16 = o_dtype == ZHA_BF16;
+  if (p.warp) {
+    const cudaError_t e = launch_route_warp(t, a, true, stream);
+    ++t->launches;
+    return e;
+  }
   a.stage_tokens = p.stage_tokens;
   a.attn_nbuf = p.nbuf;
   a.O = d_O;
@@ -454,7 +470,7 @@ cudaError_t launch_causal(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q
   const bool bf = t->desc.kv_dtype == ZHA_BF16;
   const int row = D * (bf ? 2 : 4);
   const bool attend = d_O != nullptr;
-  const DecodePlan dp = plan_decode(t, q_heads, nq, beam);
+  const DecodePlan dp = plan_decode(t, q_heads, nq, beam, false);
   const bool wide = a.total_queries <= 2LL * t->sms;
   // Route only: the route's rows.  Attending: the decode plan's row region; in narrow
   // launches grown up to 64 KB, and any number of stages is accepted (the attention

@@ -82,6 +82,14 @@ ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_f32_s16);
 
 constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
+// Warp-per-query kernel (route_warp.cu) for launches with many queries: each warp routes one
+// query with its candidate rows loaded straight into registers and, when attending, reads
+// its leaves' K/V rows the same way.  It fits when its per-warp shared memory (candidate ids,
+// keys, survivors) stays small and a query attends to at most kWarpMaxTokens tokens.
+constexpr int kWarpMaxTokens = 256;
+bool route_warp_fits(const zha_tree* t, int cmax, int beam);
+cudaError_t launch_route_warp(zha_tree* t, const RouteArgs& a, bool attend, cudaStream_t s);
+
 // Shared-memory layout of one query in the staged kernel.
 struct RouteSmem {
   size_t rows, keys, cand, surv_a, surv_b, leaf_sc, red, hist, pw, bar, total;
@@ -120,6 +128,24 @@ __host__ __device__ inline RouteSmem route_smem_layout(int D, int cmax, int beam
               // then the three buffers' "empty"
   o += 48;
   s.total = route_align(o, 128);
+  return s;
+}
+
+// The scoring order every route kernel uses, so that all of them give the same fp32 score
+// for a (query, row) pair bit for bit: eight lanes share a row, lane l8 takes the row's
+// 16-byte chunks l8, l8 + 8, ... in that order; within a chunk, elements 4i and 4i + 1 go to
+// one packed accumulator and 4i + 2, 4i + 3 to another (score_fma); the lane's partial is
+// (acc0.x + acc0.y) + (acc1.x + acc1.y), and the eight partials are summed by xor shuffles
+// over lane distances 4, 2, 1 (score_reduce8).
+__device__ __forceinline__ void score_fma(const float* q, const float* v, float2& acc0, float2& acc1) {
+  acc0 = __ffma2_rn(make_float2(q[0], q[1]), make_float2(v[0], v[1]), acc0);
+  acc1 = __ffma2_rn(make_float2(q[2], q[3]), make_float2(v[2], v[3]), acc1);
+}
+__device__ __forceinline__ float score_reduce8(float2 acc0, float2 acc1) {
+  float s = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
   return s;
 }
 
@@ -333,6 +359,64 @@ __device__ __forceinline__ int select_compact(const unsigned long long* keys, co
     kept += __popc(bal);
   }
   return kept;
+}
+
+// One warp: top-min(beam, C) of keys[0, C) for C <= 64 (two keys per lane), by beam rounds
+// that each take the largest remaining key (warp max of the score words, then of the index
+// words among the keys with that score: keys are distinct, so exactly one lane holds it).
+// The beam-th key taken is the threshold T; the kept candidates (key >= T) are compacted in
+// candidate order as in select_compact.  Fewer steps than the bit search when beam is small.
+// Returns the number kept.
+__device__ __forceinline__ int select_extract(const unsigned long long* keys, const int* cand, int C, int beam,
+                                              int lane, int* nxt, float* leaf_sc, bool leaf) {
+  const unsigned long long k0 = lane < C ? keys[lane] : 0ull;
+  const unsigned long long k1 = lane + 32 < C ? keys[lane + 32] : 0ull;
+  unsigned long long T = 0ull;
+  if (C > beam) {
+    // each lane's two keys, larger first; a taken key is replaced by the lane's other one
+    unsigned long long r0 = k0 > k1 ? k0 : k1, r1 = k0 > k1 ? k1 : k0;
+    for (int it = 0; it < beam; ++it) {
+      const uint32_t hi = (uint32_t)(r0 >> 32);
+      const uint32_t mh = __reduce_max_sync(0xffffffffu, hi);
+      const unsigned at = __ballot_sync(0xffffffffu, hi == mh);
+      uint32_t ml;
+      if (__builtin_expect((at & (at - 1u)) == 0u, 1)) {  // one lane holds the top score
+        ml = __shfl_sync(0xffffffffu, (uint32_t)r0, __ffs(at) - 1);
+      } else {  // equal scores: the largest index word among them
+        ml = __reduce_max_sync(0xffffffffu, hi == mh ? (uint32_t)r0 : 0u);
+      }
+      T = ((unsigned long long)mh << 32) | ml;
+      if (r0 == T) {
+        r0 = r1;
+        r1 = 0ull;
+      }
+    }
+  }
+  int kept = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int k = lane + 32 * i;
+    const unsigned long long key = i == 0 ? k0 : k1;
+    const bool keep = k < C && key >= T;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = kept + __popc(bal & ((1u << lane) - 1u));
+      nxt[pos] = cand[k];
+      if (leaf) leaf_sc[pos] = key_score(key);
+    }
+    kept += __popc(bal);
+  }
+  return kept;
+}
+
+// One warp's exact top-min(beam, C) selection, compacted in candidate order: the extract
+// rounds for small levels and beams, else the bit search.
+__device__ __forceinline__ int select_warp(const unsigned long long* keys, const int* cand, int C, int beam,
+                                           int lane, int* nxt, float* leaf_sc, bool leaf) {
+  if (C <= 64 && beam <= 16) return select_extract(keys, cand, C, beam, lane, nxt, leaf_sc, leaf);
+  return C <= 64    ? select_compact<2>(keys, cand, C, beam, lane, nxt, leaf_sc, leaf)
+         : C <= 128 ? select_compact<4>(keys, cand, C, beam, lane, nxt, leaf_sc, leaf)
+                    : select_compact<8>(keys, cand, C, beam, lane, nxt, leaf_sc, leaf);
 }
 
 // Rank selection for small levels (C <= 64 nw, at most two candidates per thread of the

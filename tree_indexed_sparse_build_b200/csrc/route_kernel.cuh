@@ -46,10 +46,9 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   constexpr bool PREFIX = PATH == kPathPrefix;
   constexpr bool HASPATH = PATH != kPathNone;
   static_assert(!HASPATH || ATTEND, "the path reads K rows of type TKV");
-  constexpr int EPC = 16 / (int)sizeof(TS);      // summary elements per 16-byte chunk
-  constexpr int CPL = D * (int)sizeof(TS) / 64;  // 16-byte chunks of a row per lane (4 lanes per row)
+  constexpr int EPC = 16 / (int)sizeof(TS);       // summary elements per 16-byte chunk
+  constexpr int CPL = D * (int)sizeof(TS) / 128;  // 16-byte chunks of a row per lane (8 lanes per row)
   constexpr uint32_t SROW = D * (uint32_t)sizeof(TS);  // bytes of a summary row
-  constexpr int R = 8;         // candidate keys held per lane in the selecting warp
   extern __shared__ __align__(128) unsigned char rsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = GROUPED ? a.wpq : 1;  // warps of this query
@@ -148,9 +147,10 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
   }
   qsync();
 
-  // Four lanes per row: lane (rg = lane / 4, sub = lane % 4) reads chunks 4 (j ^ par) + sub,
-  // par = rg & 1, so the two rows of a shared-memory phase use opposite bank halves.
-  const int sub = lane & 3, rg = lane >> 2, par = rg & 1;
+  // Eight lanes per row, in the scoring order of score_fma / score_reduce8 (route_common.cuh):
+  // lane (rg = lane / 8, l8 = lane % 8) reads chunks l8 + 8 j, so each row of a shared-memory
+  // phase is one 128-byte run.
+  const int l8 = lane & 7, rg = lane >> 3;
   float qv[CPL][EPC];
   int* cur = surv_a;
   int* nxt = surv_b;
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       const long long qo = qg * D;
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
-        const int c = 4 * (j ^ par) + sub;
+        const int c = l8 + 8 * j;
 #pragma unroll
         for (int e = 0; e < EPC; ++e)
           qv[j][e] = a.q_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.Q)[qo + EPC * c + e])
@@ -248,13 +248,12 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
     }
 
-    // score: rows r = 8 (wq + nw t) + rg, two rows per lane in flight
-    for (int r0 = 8 * wq; r0 < C; r0 += 16 * nw) {
-      // four running sums per row (dims 4c + e for e = 0..3), updated pairwise by packed FMAs
+    // score: rows r = 4 (wq + nw t) + rg, two rows per lane in flight
+    for (int r0 = 4 * wq; r0 < C; r0 += 8 * nw) {
       float2 acc[2][2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int r = r0 + 8 * nw * u + rg;
+        const int r = r0 + 4 * nw * u + rg;
         acc[u][0] = make_float2(0.f, 0.f);
         acc[u][1] = make_float2(0.f, 0.f);
         if (r < C) {
@@ -262,23 +261,17 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
 #pragma unroll
           for (int j = 0; j < CPL; ++j) {
             float v[EPC];
-            Vec16<TS>::to_f32(row[4 * (j ^ par) + sub], v);
+            Vec16<TS>::to_f32(row[l8 + 8 * j], v);
 #pragma unroll
-            for (int e = 0; e < EPC; e += 4) {
-              acc[u][0] = __ffma2_rn(make_float2(qv[j][e], qv[j][e + 1]), make_float2(v[e], v[e + 1]), acc[u][0]);
-              acc[u][1] =
-                  __ffma2_rn(make_float2(qv[j][e + 2], qv[j][e + 3]), make_float2(v[e + 2], v[e + 3]), acc[u][1]);
-            }
+            for (int e = 0; e < EPC; e += 4) score_fma(qv[j] + e, v + e, acc[u][0], acc[u][1]);
           }
         }
       }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        float s = (acc[u][0].x + acc[u][0].y) + (acc[u][1].x + acc[u][1].y);
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        const int r = r0 + 8 * nw * u + rg;
-        if (sub == 0 && r < C) keys[r] = route_key(s, cand[r]);
+        const float s = score_reduce8(acc[u][0], acc[u][1]);
+        const int r = r0 + 4 * nw * u + rg;
+        if (l8 == 0 && r < C) keys[r] = route_key(s, cand[r]);
       }
     }
     qsync();
@@ -302,9 +295,7 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         for (int k = lane; k < a.beam; k += 32) tr[k] = k < kept ? nxt[k] : -1;
       }
     } else if (wq == 0 && C > 0) {
-      const int kept = C <= 64    ? select_compact<2>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
-                       : C <= 128 ? select_compact<4>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0)
-                                  : select_compact<R>(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0);
+      const int kept = select_warp(keys, cand, C, a.beam, lane, nxt, leaf_sc, l == 0);
       __syncwarp();
       if (a.trace && valid) {
         int* tr = a.trace + (qg * a.L + (a.L - 1 - l)) * a.beam;

@@ -82,6 +82,7 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
 // requires append_ok).
 struct DecodePlan {
   bool fused;
+  bool warp;              // many queries: the warp-per-query kernel (route_warp.cu)
   size_t rows_bytes;      // candidate-row / K-V stage region per query
   int stage_tokens;       // tokens per stage buffer
   int nbuf;               // stage buffers (2 or 3)
@@ -90,7 +91,9 @@ struct DecodePlan {
   bool append_ok;         // a one-leaf append can ride along (wide launches)
   size_t path_off, path_bytes;  // that append's region inside the row region
 };
-DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam);
+// allow_warp = false: the staged kernel's plan only (the causal and buffered calls run the
+// staged kernel whatever the launch shape).
+DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam, bool allow_warp = true);
 cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
                           int q_heads, int nq, int beam, const void* d_K, const void* d_V,
                           float scale, int* d_leaf_idx, float* d_leaf_score, int* d_trace,
