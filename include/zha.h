@@ -285,6 +285,17 @@ zha_status zha_tree_get_desc(const zha_tree* tree, zha_tree_desc* out);
 /* The CUDA device that was current when the tree was created; -1 on a null handle. */
 int zha_tree_device(const zha_tree* tree);
 
+/* Failure-path testing (the source pages have no counterpart).  Every kernel that waits for
+ * its own bulk copies bounds that wait (about a second of SM clock); a wait that runs out
+ * records ZHA_ERR_TIMEOUT in the device error word, waits for the copies it issued with the
+ * same default bound, marks the affected queries' outputs as lost (leaf indices -1, scores
+ * and O NaN) and returns; the context stays usable.  This call lowers the first of those two
+ * bounds to `cycles` SM clock cycles for every later call on this tree, so a test can make a
+ * wait run out on demand; 0 restores the default.  After a call whose wait ran out, the
+ * summaries that call was writing (a build or append) are unspecified until the tree is
+ * rebuilt.  ZHA_ERR_INVALID_ARG on a null tree or negative cycles. */
+zha_status zha_tree_set_wait_limit(zha_tree* tree, long long cycles);
+
 const char* zha_status_string(zha_status status);
 
 #ifdef __cplusplus

@@ -39,7 +39,7 @@ namespace zha {
 
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = kAttnThreads / 32;
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+constexpr long long kWaitCycles = kCopyWaitCycles;  // ~1 s at 1.9 GHz
 
 struct AttnArgs {
   const void* Q;
@@ -57,6 +57,7 @@ struct AttnArgs {
   float* partial;  // scratch path: [queries][splits][D + 2]
   unsigned* err;
   long long total_items;
+  long long first_wait;  // bound of a first wait for a stage's copies
 };
 
 // Shared-memory layout, identical on host and device.
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(const AttnArgs a) 
   for (int s = 0; s < nstages; ++s) {
     const int buf = a.nbuf == 2 ? (s & 1) : 0;
     const uint32_t parity = (uint32_t)((a.nbuf == 2 ? (s >> 1) : s) & 1);
-    const bool ok = mbar_wait_bounded(&bar[buf], parity, a.err, kDevErrTimeout, kWaitCycles);
+    const bool ok = mbar_wait_bounded(&bar[buf], parity, a.err, kDevErrTimeout, a.first_wait);
     // one barrier per stage: the stage's data is visible to all, every warp has finished
     // the previous stage (whose buffer the next copy may now overwrite)
     if (__syncthreads_or(!ok)) {
@@ -466,6 +467,7 @@ cudaError_t launch_attention(zha_tree* t, const AttnPlan& plan, const void* d_Q,
   a.o_bf16 = o_dtype == ZHA_BF16;
   a.partial = static_cast<float*>(d_scratch);
   a.err = t->d_err;
+  a.first_wait = first_wait_cycles(t);
   const long long queries = (long long)t->desc.batch * q_heads * nq;
   a.total_items = queries * plan.splits;
   cudaError_t e;

@@ -69,7 +69,8 @@ struct StagedAttn {
   void* O;               // output row qg of [queries, D]
   int o_bf16;
   unsigned* err;
-  long long wait_cycles;
+  long long wait_cycles;   // bound of a first wait for a stage's copies
+  long long drain_cycles;  // bound of the waits that let copies land after a failure
 };
 
 // Called by every thread of the query's nw warps (warp wq, lane), after warp 0 issued
@@ -109,7 +110,7 @@ __device__ bool attend_staged(const StagedAttn& s, long long qg, bool valid,
     // previous use of its buffer was released, so no warp's "empty" arrival below can count
     // toward that earlier release.
     if (ok) ok = mbar_wait_bounded(&s.bars[b], phase(st), s.err, kDevErrTimeout, s.wait_cycles);
-    __syncwarp();
+    ok = __all_sync(0xffffffffu, ok);  // one outcome per warp before its full-warp shuffles
     if (ok && r0 < rounds) {
       const unsigned char* Ks = s.sb + (size_t)b * 2 * stage_bytes;
       attn_tokens<TKV, D>(Ks, Ks + stage_bytes, cnt, 16 * r0, 8, 16 * nw, qv, s.qk_scale, pw, m_w, l_w,
@@ -120,7 +121,7 @@ __device__ bool attend_staged(const StagedAttn& s, long long qg, bool valid,
     if (wq == 0 && st + s.nbuf < nst && ok) {
       // refill buffer b once every warp is past stage st
       ok = mbar_wait_bounded(&s.empty[b], (uint32_t)((st / s.nbuf) & 1), s.err, kDevErrTimeout,
-                             s.wait_cycles);
+                             s.drain_cycles);
       __syncwarp();
       if (ok) {
         attn_issue_stage<ROWB>(s.leaves, s.m, s.buf_leaf0, s.lb, s.total, s.TS, st + s.nbuf, s.nbuf, s.sb, s.Ku, s.Vu,
@@ -136,7 +137,7 @@ __device__ bool attend_staged(const StagedAttn& s, long long qg, bool valid,
     // the error word
     if (wq == 0 && lane == 0)
       for (int st = max(0, issued - s.nbuf); st < issued; ++st)
-        mbar_wait_bounded(&s.bars[st % s.nbuf], phase(st), s.err, kDevErrTimeout, s.wait_cycles);
+        mbar_wait_bounded(&s.bars[st % s.nbuf], phase(st), s.err, kDevErrTimeout, s.drain_cycles);
     if (valid && wq == 0)
       for (int e = lane; e < D; e += 32) {
         if (s.o_bf16)

@@ -128,10 +128,38 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// Non-blocking test of phase `parity` of `bar` (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounds below this many SM clocks (set only to test the failure path) poll with test_wait:
+// try_wait suspends the thread until the phase completes or a hardware time limit passes, so
+// a tiny bound would never be noticed before the copies land.
+constexpr long long kPollWaitBelow = 1000000;
+
 // Bounded wait on phase `parity` of `bar`.  Gives up after ~max_cycles SM clocks,
 // records kDevErrTimeout-style `flag` in *err and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned* err,
                                                   unsigned flag, long long max_cycles) {
+  if (max_cycles < kPollWaitBelow) {
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity)) {
+      if (clock64() - t0 > max_cycles) {
+        atomicOr(err, flag);
+        return false;
+      }
+    }
+    return true;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {

@@ -233,6 +233,7 @@ RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int 
   a.leaf_score = d_leaf_score;
   a.trace = d_trace;
   a.err = t->d_err;
+  a.first_wait = first_wait_cycles(t);
   return a;
 }
 

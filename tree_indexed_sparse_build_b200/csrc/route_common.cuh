@@ -57,6 +57,7 @@ struct RouteArgs {
   // tokens after the routed prefix, which then ends on a leaf boundary)
   long long buf_leaf0;
   int buf_tokens;
+  long long first_wait;      // bound of a first wait for copies (kCopyWaitCycles unless testing)
 };
 
 struct NoKV {};  // route only: no attention epilogue
@@ -80,7 +81,7 @@ ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_f32_s16);
 #undef ZHA_ROUTE_LAUNCH_DECL
 
 
-constexpr long long kRouteWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+constexpr long long kRouteWaitCycles = kCopyWaitCycles;  // ~1 s at 1.9 GHz
 
 // Warp-per-query kernel (route_warp.cu) for launches with many queries: each warp routes one
 // query with its candidate rows loaded straight into registers and, when attending, reads

@@ -38,6 +38,21 @@ namespace zha {
 // With a KV type, the query then attends over its leaves unless O is null.
 // TS: the summaries' storage (float, or bf16 bits in uint16_t); rows are staged as stored
 // and widened to fp32 as they are scored.
+// A query whose copies did not arrive (a bounded wait ran out, the error word is set): no
+// leaves, NaN scores and output, so the loss shows in the results as well.  Called by one warp.
+template <bool ATTEND, int D>
+__device__ __forceinline__ void route_poison(const RouteArgs& a, long long qg, int lane) {
+  for (int k = lane; k < a.beam; k += 32) {
+    if (a.leaf_idx) a.leaf_idx[qg * a.beam + k] = -1;
+    if (a.leaf_score) a.leaf_score[qg * a.beam + k] = __int_as_float(0x7fc00000);
+  }
+  if (ATTEND && a.O != nullptr)
+    for (int e = lane; e < D; e += 32) {
+      if (a.o_bf16) static_cast<uint16_t*>(a.O)[qg * D + e] = 0x7FC0u;
+      else static_cast<float*>(a.O)[qg * D + e] = __int_as_float(0x7fc00000);
+    }
+}
+
 template <int D, bool GROUPED, typename TKV, bool NARROW, int PATH, typename TS>
 __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3 : 1)
     route_tma_kernel(const RouteArgs a) {
@@ -205,13 +220,14 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     }
     if (HASPATH && l == l_first) {
       // the path rows, while the first level's copies are in flight
-      const bool pok = !live || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
+      const bool pok = !live || mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, a.first_wait);
       const bool pfail = GROUPED ? group_any(bar_id, bar_n, !pok) : __any_sync(0xffffffffu, !pok);
       if (pfail) {
         if (wq == 0 && lane == 0) {  // let all copies land before the CTA exits
           if (live) mbar_wait_bounded(pbar, 0, a.err, kDevErrTimeout, kRouteWaitCycles);
           if (C > 0) mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
         }
+        if (wq == 0 && valid) route_poison<ATTEND, D>(a, qg, lane);
         return;
       }
       // every thread has seen the path's copies land: the path barrier's life ends here, as
@@ -227,11 +243,12 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
         }
       }
     }
-    const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+    const bool ok = C == 0 || mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, a.first_wait);
     const bool failed = GROUPED ? group_any(bar_id, bar_n, !ok) : __any_sync(0xffffffffu, !ok);
     if (failed) {
       if (wq == 0 && lane == 0 && C > 0)  // let the copies land before the CTA exits
         mbar_wait_bounded(bar, parity, a.err, kDevErrTimeout, kRouteWaitCycles);
+      if (wq == 0 && valid) route_poison<ATTEND, D>(a, qg, lane);
       return;  // the whole group leaves together
     }
     if (!GROUPED) __syncwarp();  // candidate ids written by other lanes
@@ -347,7 +364,8 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
     sa.O = a.O;
     sa.o_bf16 = a.o_bf16;
     sa.err = a.err;
-    sa.wait_cycles = kRouteWaitCycles;
+    sa.wait_cycles = a.first_wait;
+    sa.drain_cycles = kRouteWaitCycles;
     const int nst = (sa.total + sa.TS - 1) / sa.TS;
     if (wq == 0)
       for (int st = 0; st < min(nst, sa.nbuf); ++st)

@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kPassThreads) pyramid_pass_kernel(const PassAr
 constexpr int kPathMaxLeaves = 8;
 constexpr int kPathThreads = 256;
 constexpr size_t kPathSmemCap = 160 * 1024;
-constexpr long long kPathWaitCycles = 2000000000LL;
+constexpr long long kPathWaitCycles = kCopyWaitCycles;
 
 struct AppendPathArgs {
   const char* K;               // unit 0, token 0
@@ -197,6 +197,7 @@ struct AppendPathArgs {
   int fp64_off;                // byte offset of the two fp64 node buffers
   int bar_off;
   unsigned* err;
+  long long first_wait;        // bound of the first wait for the copies
 };
 
 template <typename TIn, typename TS, int D>
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kPathThreads) append_path_kernel(const AppendP
                       (uint32_t)a.sib_rows[l] * D * (uint32_t)sizeof(TS), bar);
   }
   __syncthreads();
-  const bool ok = mbar_wait_bounded(bar, 0, a.err, kDevErrTimeout, kPathWaitCycles);
+  const bool ok = mbar_wait_bounded(bar, 0, a.err, kDevErrTimeout, a.first_wait);
   if (__syncthreads_or(!ok)) {
     if (threadIdx.x == 0) mbar_wait_bounded(bar, 0, a.err, kDevErrTimeout, kPathWaitCycles);
     return;
@@ -343,6 +344,7 @@ cudaError_t launch_pyramid(zha_tree* t, const void* d_K, long long N, long long 
     a.lo = lo;
     a.hi = hi;
     a.err = t->d_err;
+    a.first_wait = first_wait_cycles(t);
     a.tok_rows = (int)(std::min((hi + 1) * a.lb, N) - lo * a.lb);
     size_t o = (size_t)a.tok_rows * D * esz;
     long long clo = lo, chi = hi;

@@ -373,6 +373,11 @@ zha_status zha_tree_get_desc(const zha_tree* t, zha_tree_desc* out) {
   return ZHA_OK;
 }
 int zha_tree_device(const zha_tree* t) { return t ? t->device : -1; }
+zha_status zha_tree_set_wait_limit(zha_tree* t, long long cycles) {
+  if (!t || cycles < 0) return ZHA_ERR_INVALID_ARG;
+  t->wait_limit = cycles;
+  return ZHA_OK;
+}
 
 const char* zha_status_string(zha_status s) {
   switch (s) {

@@ -16,6 +16,12 @@ constexpr int kMaxCandidates = 4096;  // beam * branching bound for the route ke
 // Bits of the device error word.
 enum : unsigned { kDevErrTimeout = 1u, kDevErrBadLeaf = 2u };
 
+// Bound, in SM clock cycles, on every wait for a kernel's bulk copies (about a second).  A wait
+// that runs out records kDevErrTimeout; the kernel then waits for the copies it issued with
+// this same bound before it leaves.  zha_tree_set_wait_limit lowers the first bound (not
+// the second) so tests can make a wait run out.
+constexpr long long kCopyWaitCycles = 2000000000LL;
+
 // Launch `kern` with programmatic stream serialization (see pdl_wait in
 // device_common.cuh): the kernel may begin while its predecessor drains.
 template <typename... KArgs, typename... Args>
@@ -54,9 +60,15 @@ struct zha_tree {
   float* radii;                // caller's bounding-sphere radii [units][unit_rows], or null
   int sms;                     // SMs of the device the tree was created on
   int device;
+  long long wait_limit;        // > 0: bound on a kernel's first wait for its copies (testing)
 };
 
 namespace zha {
+
+// The bound of a kernel's first wait for its copies on this tree.
+inline long long first_wait_cycles(const zha_tree* t) {
+  return t->wait_limit > 0 ? t->wait_limit : kCopyWaitCycles;
+}
 
 // Bytes of one stored summary element (desc.summary_dtype).
 inline int sum_bytes(const zha_tree* t) { return t->desc.summary_dtype == ZHA_BF16 ? 2 : 4; }

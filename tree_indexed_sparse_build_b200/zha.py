@@ -29,7 +29,7 @@ EXPORTED = [
     "zha_status_string", "zha_sparse_attn_decode_noalloc", "zha_noalloc_scratch_capacity",
     "zha_decode", "zha_decode_step", "zha_route_causal", "zha_decode_causal",
     "zha_tree_radii_bytes", "zha_tree_attach_radii", "zha_threshold_route", "zha_decode_buffered",
-    "zha_tree_get_desc", "zha_tree_device",
+    "zha_tree_get_desc", "zha_tree_device", "zha_tree_set_wait_limit",
 ]
 
 
@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
             "zha_tree_launch_count": (_LL, [_P]),
             "zha_tree_get_desc": (_I, [_P, ctypes.POINTER(zha_tree_desc)]),
             "zha_tree_device": (_I, [_P]),
+            "zha_tree_set_wait_limit": (_I, [_P, _LL]),
             "zha_status_string": (ctypes.c_char_p, [_I]),
         }
         for name, (res, args) in sig.items():
@@ -146,6 +147,11 @@ def zha_tree_get_desc(handle) -> zha_tree_desc:
 
 def zha_tree_device(handle) -> int:
     return int(lib().zha_tree_device(handle))
+
+
+def zha_tree_set_wait_limit(handle, cycles: int) -> None:
+    """Test hook: bound the first wait for a kernel's copies to `cycles` SM clocks (0: default)."""
+    _check(lib().zha_tree_set_wait_limit(handle, int(cycles)), "zha_tree_set_wait_limit")
 
 
 def _check_q(handle, Q: torch.Tensor, what: str = "Q") -> None:
