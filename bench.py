@@ -447,6 +447,62 @@ def run_decode(w, W, K, rank, dev, flush, sampler_factory, eager=False, mode="st
     return res
 
 
+def run_decode_split(w, W, K, rank, world, dev, flush):
+    """128K decode steps of ONE workload split over the ranks by (batch, KV head) unit: rank r
+    decodes units ranks.unit_range(units, world, r) (its K/V rows and queries are contiguous
+    slices of the full tensors, run as a tree set of batch 1) and the step's outputs are
+    all-gathered into unit order on every rank.  A step = zha_decode_step on the rank's units
+    (one CUDA graph) + the all-gather, bracketed by events on the same stream; L2 flushed
+    between steps.  Returns the rank's per-step times and a parity sample of its first unit."""
+    import torch
+    from tree_indexed_sparse_build_b200 import ranks, synth, zha
+
+    N, cap = w.seq_len, w.seq_len + W + K
+    u0, u1 = ranks.unit_range(w.units, world, rank)
+    nl, g, d, beam = u1 - u0, w.group, w.head_dim, w.beam
+    Qs = np.stack([synth.queries(w, step=s) for s in range(W + K)])  # [steps, B, Hq, 1, d]
+    Kn = synth.keys(w, capacity=cap, units=list(range(u0, u1)))
+    Vn = synth.values(w, capacity=cap, units=list(range(u0, u1)))
+    Kl = ranks.unit_slice(torch.from_numpy(Kn), u0, u1).contiguous().view(torch.bfloat16).to(dev)
+    Vl = ranks.unit_slice(torch.from_numpy(Vn), u0, u1).contiguous().view(torch.bfloat16).to(dev)
+    Ql = torch.stack([ranks.query_slice(torch.from_numpy(Qs[s]), g, u0, u1) for s in range(W + K)]).contiguous()
+    Ql = Ql.view(torch.bfloat16).to(dev)  # [steps, 1, nl * g, 1, d]
+    tree = zha.Tree(1, nl, d, w.branching, w.leaf_block, cap, torch.bfloat16)
+    tree.build(Kl, N)
+    O = torch.empty((W + K, 1, nl * g, 1, d), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((W + K, 1, nl * g, 1, beam), dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream()
+    graphs = []
+    for s in range(W + K):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream, capture_error_mode="thread_local"):
+            zha.zha_decode_step(tree.handle, Kl, Vl, N + s + 1, Ql[s], beam, w.scale, idx[s], O[s])
+        graphs.append(gr)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms, full = [], None
+    for s in range(W + K):
+        flush.zero_()
+        torch.cuda.synchronize()
+        ranks.barrier(world)
+        e0.record()
+        graphs[s].replay()
+        full = ranks.gather_units(O[s].reshape(nl * g, d), w.units, world, rank, g)
+        e1.record()
+        torch.cuda.synchronize()
+        if s >= W:
+            ms.append(e0.elapsed_time(e1))
+    assert tree.check() == zha.ZHA_OK, "device error word set during the split decode steps"
+    assert full.shape == (w.units * g, d)
+    s_last = W + K - 1
+    par = parity_sample(w.with_(batch=1, kv_heads=nl, q_heads=nl * g), Ql[s_last].view(torch.uint16).cpu().numpy(),
+                        ranks.unit_slice(torch.from_numpy(Kn), u0, u1).numpy(),
+                        ranks.unit_slice(torch.from_numpy(Vn), u0, u1).numpy(), N + s_last + 1,
+                        idx[s_last].cpu().numpy(), None, O[s_last].float().cpu().numpy(), (0,))
+    del graphs
+    tree.close()
+    return {"step_ms": np.array(ms), "units": [u0, u1], "parity": par}
+
+
 def run_buffered(w, W, K, rank, dev, flush, buf_leaves=2, eager=False):
     """128K decode steps with an append buffer: each step writes one token into the buffer
     (tokens after the committed prefix) and runs zha_decode_buffered; when buf_leaves full
@@ -1184,6 +1240,10 @@ def main():
                     help="decode step calls: zha_decode_step (one launch); zha_tree_append + "
                          "zha_decode; zha_tree_append + zha_route + zha_sparse_attn_decode")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--shard", choices=["replicas", "units"], default="replicas",
+                    help="N GPUs: independent replicas of the 128K workload (weak scaling), or one "
+                         "128K workload split over the ranks by (batch, KV head) unit with the "
+                         "outputs all-gathered every step (strong scaling)")
     ap.add_argument("--eager", action="store_true",
                     help="launch the same kernels without CUDA graphs (for profilers)")
     args = ap.parse_args()
@@ -1230,6 +1290,26 @@ def main():
         return ranks.max_over_ranks(x, world, dev)
 
     sampler = lambda: ClockSampler(local)  # noqa: E731
+
+    if args.shard == "units":
+        barrier()
+        with sampler() as smp:
+            rs = run_decode_split(w, W, K, rank, world, dev, flush)
+        step_ms = max_over_ranks(float(rs["step_ms"].mean()))
+        q = w.batch * w.q_heads
+        if rank == 0:
+            cfg = dict(workload_config(w), parallelism=f"units{world}",
+                       split="each rank decodes a contiguous range of the 32 (batch, KV head) units; "
+                             "outputs all-gathered into unit order every step")
+            print(json.dumps({"metric": METRIC, "value": q / (step_ms * 1e-3), "unit": UNIT, "n_gpus": world,
+                              "steps": K, "warmup": W, "ms_per_step": step_ms, "higher_is_better": True,
+                              "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                              "config": cfg, "units_rank0": rs["units"], "parity_rank0": rs["parity"],
+                              "clocks": smp.summary(), "launch": "one CUDA graph per step (zha_decode_step) "
+                              "+ an eager all-gather of O, events on the same stream"}))
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     barrier()
     torch.cuda.synchronize()

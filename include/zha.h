@@ -97,17 +97,20 @@ zha_status zha_tree_init(const zha_tree_desc* desc, void* d_workspace, size_t wo
 zha_status zha_tree_destroy(zha_tree* tree);
 
 /* Builds every summary from tokens [0, seq_len) of d_K (replacing any previous
- * state).  seq_len == 0 leaves an empty tree.  ZHA_ERR_CAPACITY if seq_len >
+ * state): the tree of recursively compressed key summaries kept over the KV cache
+ * ("Subquadratic Attention with a Hierarchical Tree-Structured Indexer", abstract).  seq_len == 0 leaves an empty tree.  ZHA_ERR_CAPACITY if seq_len >
  * capacity_tokens. */
 zha_status zha_tree_build(zha_tree* tree, const void* d_K, long long seq_len, void* stream);
 
-/* Extends the tree to tokens [0, new_seq_len): the caller has already written
+/* Extends the tree to tokens [0, new_seq_len) as the cache grows, deepening it when needed
+ * (same abstract: the tree's depth grows with the context): the caller has already written
  * rows [seq_len, new_seq_len) of K.  Recomputes the leaves that received tokens
  * and all of their ancestors; adds levels when the leaves outgrow b^L.
  * new_seq_len must be >= the current seq_len (equal: no-op). */
 zha_status zha_tree_append(zha_tree* tree, const void* d_K, long long new_seq_len, void* stream);
 
-/* Top-down beam routing of nq queries per query head.
+/* Top-down beam routing of nq queries per query head: each query traverses the tree from
+ * the top down to retrieve a sparse subset of keys (same abstract).
  *   d_Q          [batch, q_heads, nq, head_dim] in q_dtype; q_heads % kv_heads == 0
  *   beam         1 .. 1024, and beam * branching <= 4096
  *   d_leaf_idx   out [batch, q_heads, nq, beam] int32: selected leaves, ascending,
@@ -124,7 +127,8 @@ zha_status zha_route(const zha_tree* tree, const void* d_Q, zha_dtype q_dtype, i
  * and the device's SM count, not on seq_len. */
 size_t zha_attn_scratch_bytes(const zha_tree* tree, int q_heads, int nq, int beam);
 
-/* Exact softmax attention of each query over the tokens t < seq_len of its leaves.
+/* Exact softmax attention of each query over the tokens t < seq_len of its leaves: the
+ * final attention over the retrieved subset (same abstract).
  *   d_Q, d_leaf_idx  as produced for / by zha_route (indices < 0 are skipped)
  *   d_K, d_V         the cache the tree was built over
  *   scale            multiplies q . k before the softmax (e.g. 1/sqrt(head_dim))
