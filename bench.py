@@ -855,13 +855,15 @@ def run_threshold(W, K, dev, flush):
 def run_profile_case(case: str, W: int, K: int):
     """A small case of a bench workload for ncu captures (eager launches, no graphs):
     deep_1m_2kv = the 1M-token tree with 2 KV heads and 16 query heads (group 8, 64 queries
-    per head) instead of 8 and 64, so a capture holds about 1.5 GB on the device."""
+    per head) instead of 8 and 64, so a capture holds about 1.5 GB on the device;
+    deep_1m_2kv_q256 = the same with 256 queries per head (4,096 queries, as many per SM as
+    the full batch)."""
     import torch
     from tree_indexed_sparse_build_b200 import synth, workloads, zha
 
     dev = torch.device("cuda", 0)
     w = workloads.get("deep_1m").with_(kv_heads=2, q_heads=16)
-    nq = workloads.THROUGHPUT_NQ
+    nq = workloads.THROUGHPUT_NQ * (4 if case.endswith("_q256") else 1)
     Qn = synth.queries(w, nq=nq)
     Kn = synth.keys(w, Q=Qn)
     Vn = synth.values(w)
@@ -1233,9 +1235,10 @@ def main():
     ap.add_argument("--no-build", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the 128K variants (bf16 summaries, append buffer) and the 1M bf16-summary run")
-    ap.add_argument("--profile-case", choices=["deep_1m_2kv"], default=None,
+    ap.add_argument("--profile-case", choices=["deep_1m_2kv", "deep_1m_2kv_q256"], default=None,
                     help="run only a small case for ncu captures: the 1M-token tree at 2 of its "
-                         "8 KV heads (1,024 queries, 64 per head), zha_decode, eager launches")
+                         "8 KV heads, zha_decode, eager launches; 64 queries per head (1,024), or "
+                         "256 per head (4,096: the full batch's queries per SM)")
     ap.add_argument("--mode", choices=["step", "decode", "two_call"], default="step",
                     help="decode step calls: zha_decode_step (one launch); zha_tree_append + "
                          "zha_decode; zha_tree_append + zha_route + zha_sparse_attn_decode")
