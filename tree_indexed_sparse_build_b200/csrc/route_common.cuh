@@ -362,20 +362,45 @@ __device__ __forceinline__ int select_compact(const unsigned long long* keys, co
   return kept;
 }
 
-// One warp: top-min(beam, C) of keys[0, C) for C <= 64 (two keys per lane), by beam rounds
-// that each take the largest remaining key (warp max of the score words, then of the index
-// words among the keys with that score: keys are distinct, so exactly one lane holds it).
-// The beam-th key taken is the threshold T; the kept candidates (key >= T) are compacted in
-// candidate order as in select_compact.  Fewer steps than the bit search when beam is small.
+// One warp: top-min(beam, C) of keys[0, C) for C <= 64 (two keys per lane), by rounds that
+// each take the largest remaining key (warp max of the score words, then of the index words
+// when several keys share the top score: keys are distinct, so exactly one lane holds it).
+// When fewer keys are dropped than kept (C - beam < beam) it takes the C - beam smallest keys
+// instead, the same way, and keeps the rest.  The kept candidates are compacted in candidate
+// order as in select_compact.  Fewer steps than the bit search when beam or C - beam is small.
 // Returns the number kept.
 __device__ __forceinline__ int select_extract(const unsigned long long* keys, const int* cand, int C, int beam,
                                               int lane, int* nxt, float* leaf_sc, bool leaf) {
   const unsigned long long k0 = lane < C ? keys[lane] : 0ull;
   const unsigned long long k1 = lane + 32 < C ? keys[lane + 32] : 0ull;
-  unsigned long long T = 0ull;
-  if (C > beam) {
+  bool keep0 = lane < C, keep1 = lane + 32 < C;
+  if (C > beam && C - beam < beam) {
+    // drop the C - beam smallest: rounds of warp min, absent keys count as the largest
+    unsigned long long r0 = keep0 ? k0 : ~0ull, r1 = keep1 ? k1 : ~0ull;
+    for (int it = 0; it < C - beam; ++it) {
+      const unsigned long long low = r0 < r1 ? r0 : r1;
+      const uint32_t hi = (uint32_t)(low >> 32);
+      const uint32_t mh = __reduce_min_sync(0xffffffffu, hi);
+      const unsigned at = __ballot_sync(0xffffffffu, hi == mh);
+      uint32_t ml;
+      if (__builtin_expect((at & (at - 1u)) == 0u, 1)) {
+        ml = __shfl_sync(0xffffffffu, (uint32_t)low, __ffs(at) - 1);
+      } else {
+        ml = __reduce_min_sync(0xffffffffu, hi == mh ? (uint32_t)low : 0xFFFFFFFFu);
+      }
+      const unsigned long long T = ((unsigned long long)mh << 32) | ml;
+      if (r0 == T) {
+        r0 = ~0ull;
+        keep0 = false;
+      } else if (r1 == T) {
+        r1 = ~0ull;
+        keep1 = false;
+      }
+    }
+  } else if (C > beam) {
     // each lane's two keys, larger first; a taken key is replaced by the lane's other one
     unsigned long long r0 = k0 > k1 ? k0 : k1, r1 = k0 > k1 ? k1 : k0;
+    unsigned long long T = 0ull;
     for (int it = 0; it < beam; ++it) {
       const uint32_t hi = (uint32_t)(r0 >> 32);
       const uint32_t mh = __reduce_max_sync(0xffffffffu, hi);
@@ -392,13 +417,15 @@ __device__ __forceinline__ int select_extract(const unsigned long long* keys, co
         r1 = 0ull;
       }
     }
+    keep0 = keep0 && k0 >= T;
+    keep1 = keep1 && k1 >= T;
   }
   int kept = 0;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int k = lane + 32 * i;
     const unsigned long long key = i == 0 ? k0 : k1;
-    const bool keep = k < C && key >= T;
+    const bool keep = i == 0 ? keep0 : keep1;
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
     if (keep) {
       const int pos = kept + __popc(bal & ((1u << lane) - 1u));
@@ -414,7 +441,7 @@ __device__ __forceinline__ int select_extract(const unsigned long long* keys, co
 // rounds for small levels and beams, else the bit search.
 __device__ __forceinline__ int select_warp(const unsigned long long* keys, const int* cand, int C, int beam,
                                            int lane, int* nxt, float* leaf_sc, bool leaf) {
-  if (C <= 64 && beam <= 16) return select_extract(keys, cand, C, beam, lane, nxt, leaf_sc, leaf);
+  if (C <= 64 && (beam <= 16 || C - beam <= 16)) return select_extract(keys, cand, C, beam, lane, nxt, leaf_sc, leaf);
   return C <= 64    ? select_compact<2>(keys, cand, C, beam, lane, nxt, leaf_sc, leaf)
          : C <= 128 ? select_compact<4>(keys, cand, C, beam, lane, nxt, leaf_sc, leaf)
                     : select_compact<8>(keys, cand, C, beam, lane, nxt, leaf_sc, leaf);

@@ -265,14 +265,16 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
       }
     }
 
-    // score: rows r = 4 (wq + nw t) + rg, two rows per lane in flight
-    for (int r0 = 4 * wq; r0 < C; r0 += 8 * nw) {
-      float2 acc[2][2];
+    // score: rows r0 + 4 nw u + rg (u = 0 .. 3) per iteration, r0 = 4 (wq + 4 nw t).  Each
+    // lane forms its partial of the four rows, and one transposed butterfly over the eight
+    // lanes of a row (distances 4, 2, 1) sums all four with four shuffles, associating
+    // exactly as score_reduce8 does: lane l8 ends with the sum of row u = l8 / 2.
+    for (int r0 = 4 * wq; r0 < C; r0 += 16 * nw) {
+      float part[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < 4; ++u) {
         const int r = r0 + 4 * nw * u + rg;
-        acc[u][0] = make_float2(0.f, 0.f);
-        acc[u][1] = make_float2(0.f, 0.f);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         if (r < C) {
           const uint4* row = reinterpret_cast<const uint4*>(rows + (size_t)r * D);
 #pragma unroll
@@ -280,16 +282,20 @@ __global__ void __launch_bounds__(NARROW ? 256 : kRouteMaxWarps * 32, NARROW ? 3
             float v[EPC];
             Vec16<TS>::to_f32(row[l8 + 8 * j], v);
 #pragma unroll
-            for (int e = 0; e < EPC; e += 4) score_fma(qv[j] + e, v + e, acc[u][0], acc[u][1]);
+            for (int e = 0; e < EPC; e += 4) score_fma(qv[j] + e, v + e, acc0, acc1);
           }
         }
+        part[u] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
       }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const float s = score_reduce8(acc[u][0], acc[u][1]);
-        const int r = r0 + 4 * nw * u + rg;
-        if (l8 == 0 && r < C) keys[r] = route_key(s, cand[r]);
-      }
+      const bool hi4 = (l8 & 4) != 0, hi2 = (l8 & 2) != 0;
+      const float send0 = hi4 ? part[0] : part[2], send1 = hi4 ? part[1] : part[3];
+      const float keep0 = hi4 ? part[2] : part[0], keep1 = hi4 ? part[3] : part[1];
+      const float b0 = keep0 + __shfl_xor_sync(0xffffffffu, send0, 4);
+      const float b1 = keep1 + __shfl_xor_sync(0xffffffffu, send1, 4);
+      float sc = (hi2 ? b1 : b0) + __shfl_xor_sync(0xffffffffu, hi2 ? b0 : b1, 2);
+      sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+      const int r = r0 + 4 * nw * (l8 >> 1) + rg;
+      if ((l8 & 1) == 0 && r < C) keys[r] = route_key(sc, cand[r]);
     }
     qsync();
     // C is the same for the whole group.  Up to 64 candidates: one warp's register selection
