@@ -1329,9 +1329,9 @@ def main():
     dec_ms = float(r["decode_ms"].mean())
     fused_append = args.mode == "step"
     dec_bytes = r["route_bytes"] + r["attend_bytes"] + (r["append_bytes"] if fused_append else 0)
-    dom_kernel = {"step": "route_tma_kernel (fused append + decode)",
-                  "decode": "route_tma_kernel (fused decode)",
-                  "two_call": "route_tma_kernel + attend_kernel"}[args.mode]
+    dom_kernel = {"step": "route_group_kernel (fused append + route + attention)",
+                  "decode": "route_group_kernel (fused route + attention)",
+                  "two_call": "route_group_kernel (route) + attend_kernel"}[args.mode]
     kern = {"decode": {"ms": dec_ms, "bytes": int(dec_bytes), "gbs": dec_bytes / (dec_ms * 1e-3) / 1e9,
                        "route_bytes": int(r["route_bytes"]), "attend_bytes": int(r["attend_bytes"]),
                        "append_bytes": int(r["append_bytes"]), "includes_append": fused_append},

@@ -14,6 +14,12 @@ were issued a moment before gives up, and check:
 
 Right before each call under the lowered bound the L2 cache is flushed, so the copies come
 from DRAM and are still in flight at the first check (from L2 they can land first).
+
+Which kernels wait: the staged route kernel (every level's rows and the attention's stages
+arrive by bulk copies; it runs the causal and buffered calls, and any shape the other
+kernels do not take), the stand-alone attention, the append kernel, and the CTA-per-query
+kernel's fused append path.  The warp-per-query and CTA-per-query kernels otherwise load
+straight into registers and have no copy to wait for.
 """
 from __future__ import annotations
 
@@ -36,17 +42,23 @@ def dev():
     return torch.device("cuda:0")
 
 
-# 2 units x 8 query heads, one query each: a wide launch (one query per CTA), staged kernel
+# 2 units x 8 query heads, one query each: a wide launch (one query per CTA)
 W = Workload(name="timeout", batch=1, kv_heads=2, q_heads=8, head_dim=128, seq_len=6000, kv_dtype="bf16",
              branching=8, leaf_block=16, beam=8, nq=1, seed=131)
+# The CTA-per-query kernel waits for the fused append's path after scoring the first level
+# (19 leaves here), so the path must still be in flight then: 320-token fp32 leaves make its
+# token copy about 160 KB, several thousand cycles behind the first level's rows.
+W_PATH = Workload(name="timeout_path", batch=1, kv_heads=2, q_heads=8, head_dim=128, seq_len=6071, kv_dtype="f32",
+                  branching=8, leaf_block=320, beam=4, nq=1, seed=132)
 
 
-def _setup(dev, capacity=None):
+def _setup(dev, capacity=None, w=W):
     from tree_indexed_sparse_build_b200 import zha
-    cap = capacity or W.seq_len
-    Qn, Kn, Vn = make_inputs(W, capacity=cap)
+    cap = capacity or w.seq_len
+    Qn, Kn, Vn = make_inputs(w, capacity=cap)
     Q, K, V = torch_of(Qn, dev), torch_of(Kn, dev), torch_of(Vn, dev)
-    tree = zha.Tree(W.batch, W.kv_heads, W.head_dim, W.branching, W.leaf_block, cap, torch.bfloat16)
+    tree = zha.Tree(w.batch, w.kv_heads, w.head_dim, w.branching, w.leaf_block, cap,
+                    torch.float32 if w.kv_dtype == "f32" else torch.bfloat16)
     return tree, Q, K, V
 
 
@@ -69,19 +81,22 @@ def _lost_or_equal(idx, O, idx_ref, O_ref):
     return lost
 
 
-def test_route_and_fused_decode_time_out_and_recover(dev):
+def test_staged_route_and_decode_time_out_and_recover(dev):
+    # the causal calls run the staged kernel; every query at the last position routes over
+    # the whole tree
     from tree_indexed_sparse_build_b200 import zha
     tree, Q, K, V = _setup(dev)
     tree.build(K, W.seq_len)
-    O_ref, idx_ref, _ = tree.decode(Q, K, V, W.beam, W.scale)
+    pos = torch.full((W.nq,), W.seq_len - 1, dtype=torch.int64, device=dev)
+    O_ref, idx_ref = tree.decode_causal(Q, pos, K, V, W.beam, W.scale)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_OK
 
     zha.zha_tree_set_wait_limit(tree.handle, 1)
     _flush_l2(dev)
-    O, idx, _ = tree.decode(Q, K, V, W.beam, W.scale)
+    O, idx = tree.decode_causal(Q, pos, K, V, W.beam, W.scale)
     _flush_l2(dev)
-    ridx, _, _ = tree.route(Q, W.beam)
+    ridx, _ = tree.route_causal(K, Q, pos, W.beam)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_ERR_TIMEOUT
     assert tree.check() == zha.ZHA_OK  # the word was cleared
@@ -90,10 +105,31 @@ def test_route_and_fused_decode_time_out_and_recover(dev):
     assert rlost > 0
 
     zha.zha_tree_set_wait_limit(tree.handle, 0)
-    O2, idx2, _ = tree.decode(Q, K, V, W.beam, W.scale)
+    O2, idx2 = tree.decode_causal(Q, pos, K, V, W.beam, W.scale)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_OK
     assert torch.equal(idx2, idx_ref) and torch.equal(O2, O_ref)
+    tree.close()
+
+
+def test_register_kernels_do_not_wait(dev):
+    # the plain route and decode of this shape load rows straight into registers: a lowered
+    # bound changes nothing
+    from tree_indexed_sparse_build_b200 import zha
+    tree, Q, K, V = _setup(dev)
+    tree.build(K, W.seq_len)
+    O_ref, idx_ref, _ = tree.decode(Q, K, V, W.beam, W.scale)
+    ridx_ref, _, _ = tree.route(Q, W.beam)
+    torch.cuda.synchronize()
+    zha.zha_tree_set_wait_limit(tree.handle, 1)
+    _flush_l2(dev)
+    O, idx, _ = tree.decode(Q, K, V, W.beam, W.scale)
+    _flush_l2(dev)
+    ridx, _, _ = tree.route(Q, W.beam)
+    torch.cuda.synchronize()
+    assert tree.check() == zha.ZHA_OK
+    assert torch.equal(idx, idx_ref) and torch.equal(O, O_ref) and torch.equal(ridx, ridx_ref)
+    zha.zha_tree_set_wait_limit(tree.handle, 0)
     tree.close()
 
 
@@ -129,8 +165,6 @@ def test_append_and_fused_step_time_out_and_recover(dev):
     N = W.seq_len - 40
     tree, Q, K, V = _setup(dev)
     ref, _, _, _ = _setup(dev)
-    ref.build(K, N)
-    O_ref, idx_ref = ref.decode_step(K, V, N + 1, Q, W.beam, W.scale)  # the normal step
     ref.build(K, N + 1)
 
     # the one-leaf append kernel (path staged with one bulk copy round)
@@ -147,17 +181,34 @@ def test_append_and_fused_step_time_out_and_recover(dev):
     for lvl in range(tree.levels + 1):
         assert torch.equal(tree.level(lvl), ref.level(lvl))
 
-    # the fused decode step (append path + route + attention in one launch)
+    tree.close()
+    ref.close()
+
+    # the fused decode step (append path + route + attention in one launch, CTA-per-query
+    # kernel: the path's copies are its one wait)
+    w = W_PATH
+    N = w.seq_len - 1  # the last leaf holds 310 tokens; the step appends the 311th
+    tree, Q, K, V = _setup(dev, w=w)
+    ref, _, _, _ = _setup(dev, w=w)
+    ref.build(K, N)
+    l0 = ref.launches
+    O_ref, idx_ref = ref.decode_step(K, V, N + 1, Q, w.beam, w.scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ref.launches - l0 == 1  # fused
     tree.build(K, N)
     zha.zha_tree_set_wait_limit(tree.handle, 1)
     _flush_l2(dev)
-    O, idx = tree.decode_step(K, V, N + 1, Q, W.beam, W.scale)
+    # the query and the first scored level (the leaves) back in L2, the path's tokens not:
+    # the route's first rows then arrive long before the path's 160 KB of tokens
+    warm = float(Q.sum()) + float(tree.level(0).sum())
+    assert warm == warm
+    O, idx = tree.decode_step(K, V, N + 1, Q, w.beam, w.scale, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_ERR_TIMEOUT
     assert _lost_or_equal(idx, O, idx_ref, O_ref) > 0
     zha.zha_tree_set_wait_limit(tree.handle, 0)
     tree.build(K, N)
-    O2, idx2 = tree.decode_step(K, V, N + 1, Q, W.beam, W.scale)
+    O2, idx2 = tree.decode_step(K, V, N + 1, Q, w.beam, w.scale, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert tree.check() == zha.ZHA_OK
     assert torch.equal(idx2, idx_ref) and torch.equal(O2, O_ref)

@@ -49,14 +49,15 @@ __host__ __device__ inline PathSmem path_smem_layout(int D, int row_bytes, int s
 
 // One thread: path nodes, then the bulk copies of the leaf's tokens and of every level's
 // children of the path node, all completing on pbar.  Ku: the unit's K rows; pyr_u: the
-// unit's summaries; off / n: level offsets and node counts after the append.
+// unit's summaries; off / n: level offsets and node counts after the append.  nodes: the
+// path's nodes at levels 0 .. L when the caller has them (else computed from leaf).
 template <typename TIn, typename TS, int D>
 __device__ void path_issue(const PathSmem& P, unsigned char* pb, const char* Ku, const TS* pyr_u,
                            const long long* off, const long long* n, int b, int L, long long leaf,
-                           int ntok, long long lb, uint64_t* pbar) {
+                           int ntok, long long lb, uint64_t* pbar, const long long* nodes = nullptr) {
   long long* node = reinterpret_cast<long long*>(pb + P.node);
   node[0] = leaf;
-  for (int l = 1; l <= L; ++l) node[l] = node[l - 1] / b;
+  for (int l = 1; l <= L; ++l) node[l] = nodes ? nodes[l] : node[l - 1] / b;
   uint32_t bytes = (uint32_t)ntok * D * sizeof(TIn);
   for (int l = 1; l <= L; ++l) {
     const long long c0 = node[l] * b, c1 = min(c0 + (long long)b, n[l - 1]);

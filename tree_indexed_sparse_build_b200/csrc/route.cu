@@ -13,22 +13,20 @@
 // children of the survivors in ascending node order (survivors ascend, the children of
 // a node are contiguous rows), so candidate k belongs to survivor k / b.
 //
-// Main kernel (route_tma_kernel): each level's candidate rows are staged in shared
-// memory by one 1-D bulk copy (non-multicast TMA) per survivor -- its b children are
-// one contiguous run of rows -- all completing on the query's mbarrier, so a level costs
-// one memory round trip whatever its width and holds no registers while in flight.
-// Few queries ("wide"): one query per CTA with up to 16 warps scoring from shared memory.
-// Many queries ("narrow"): several queries per CTA, 1-4 warps each on a named barrier per
-// query, sized so the most queries stay resident per SM.  Four lanes score one row from
-// shared memory against q held in registers (each lane a quarter of the dims; the chunk
-// order alternates between neighbouring rows so the two rows of a shared-memory phase use
-// opposite bank halves), two rows per lane in flight.  Selection: up to 64 candidates, one
-// warp holds the keys in registers, finds the B-th largest by a binary search on the key
-// bits with ballot-based warp counts (starting below the common prefix of the largest and
-// smallest score, stopping as soon as exactly B keys remain) and compacts the kept ones
-// with ballots in candidate order, which keeps the survivors ascending without a sort;
-// 65-128, ranks counted over the query's threads; wider, a radix select over the group
-// (route_common.cuh).
+// Kernels, by how many queries a call carries per SM:
+//  - at most two (route_group.cuh, route_group_kernel): one CTA of 8 or 16 warps per query;
+//    every level's candidate rows are loaded straight into registers by all the warps (one
+//    memory round trip for up to 64 NW candidates), the keys are gathered in shared memory
+//    and one warp selects; the attention splits the leaves' tokens over the warps and
+//    merges their softmax states; the one-leaf append of a decode step rides along.
+//  - more (route_warp.cu, route_warp_kernel): one warp per query, rows into registers, up
+//    to sixteen queries in flight per SM.
+//  - the causal and buffered calls, and shapes the two above do not take
+//    (route_kernel.cuh, route_tma_kernel): each level's rows staged in shared memory by one
+//    1-D bulk copy (non-multicast TMA) per survivor, scored by the query's warps.
+// Every kernel scores in one shared order (eight lanes per row, route_common.cuh), so
+// scores, survivors and leaves are bit-identical across them.  Selections: exact top-B by
+// thresholds, ranks and ballots (route_common.cuh, route_group.cuh).
 //
 // Fallback kernel (route_reg_kernel) for levels too wide to stage in shared memory:
 // the same selection, with candidate rows loaded into registers in batches.
@@ -37,9 +35,10 @@
 // are read as stored and widened to fp32 for scoring.
 //
 // Files: route_tma_kernel and its launch helpers are in route_kernel.cuh, instantiated per
-// KV type and summary type in route_tma_{nokv,bf16,f32}{,_s16}.cu; this file holds the
-// register kernel and the host-side plans (launch_route, plan_decode, launch_decode,
-// launch_causal).
+// KV type and summary type in route_tma_{nokv,bf16,f32}{,_s16}.cu; route_group_kernel in
+// route_group.cuh, instantiated per KV type in route_group_{nokv,bf16,f32}.cu;
+// route_warp_kernel in route_warp.cu; this file holds the register kernel and the host-side
+// plans (launch_route, plan_decode, launch_decode, launch_causal).
 #include <algorithm>
 #include <type_traits>
 
@@ -48,6 +47,7 @@
 #include "decode_attn.cuh"
 #include "device_common.cuh"
 #include "route_common.cuh"
+#include "route_group.cuh"
 #include "zha_internal.h"
 
 namespace zha {
@@ -234,6 +234,9 @@ RouteArgs route_args(const zha_tree* t, const void* d_Q, zha_dtype q_dtype, int 
   a.trace = d_trace;
   a.err = t->d_err;
   a.first_wait = first_wait_cycles(t);
+  a.l_first = t->L - 1;
+  while (a.l_first >= 1 && t->n[a.l_first] <= beam) --a.l_first;
+  a.m_first = (int)t->n[a.l_first + 1];
   return a;
 }
 
@@ -310,6 +313,29 @@ StagedShape staged_shape(const zha_tree* t, RouteArgs& a, size_t per_query, int 
   sh.grouped = a.wpq > 1;
   return sh;
 }
+// CTA-per-query kernel (route_group.cuh): 16 warps when every query has an SM to itself,
+// else 8 (two CTAs per SM).  It fits when every candidate of a level has a thread (the
+// selection holds one key per thread) and its shared memory (keys, ids, the attention's
+// per-warp states and, appending, the path) fits one CTA.
+int group_warps(const zha_tree* t, long long queries) { return queries <= t->sms ? 16 : 8; }
+size_t group_smem(const zha_tree* t, int cmax, int beam, int nw, bool append) {
+  const int D = t->desc.head_dim;
+  const int row = D * (t->desc.kv_dtype == ZHA_BF16 ? 2 : 4);
+  const size_t path =
+      append ? path_smem_layout(D, row, sum_bytes(t), (int)t->desc.leaf_block, t->desc.branching, t->L).total : 0;
+  return group_smem_layout(D, cmax, beam, nw, path).total;
+}
+bool group_fits(const zha_tree* t, int cmax, int beam, int nw, bool append) {
+  return cmax <= 32 * nw && group_smem(t, cmax, beam, nw, append) <= kCtaSmemCap;
+}
+cudaError_t launch_route_group(zha_tree* t, const RouteArgs& a, int nw, bool attend, bool append, cudaStream_t s) {
+  const int D = t->desc.head_dim;
+  const bool s16 = sum_bf16(t);
+  const size_t smem = group_smem(t, a.cmax, a.beam, nw, append);
+  if (!attend) return route_group_launch_nokv(D, s16, nw, false, a, smem, s);
+  if (t->desc.kv_dtype == ZHA_BF16) return route_group_launch_bf16(D, s16, nw, append, a, smem, s);
+  return route_group_launch_f32(D, s16, nw, append, a, smem, s);
+}
 }  // namespace
 
 cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_heads,
@@ -325,6 +351,15 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
     e = launch_route_warp(t, a, false, stream);
     ++t->launches;
     return e;
+  }
+  // Few queries: one CTA per query, rows loaded into registers by all its warps.
+  if (a.total_queries <= 2LL * t->sms) {
+    const int nw = group_warps(t, a.total_queries);
+    if (group_fits(t, a.cmax, beam, nw, false)) {
+      e = launch_route_group(t, a, nw, false, false, stream);
+      ++t->launches;
+      return e;
+    }
   }
   a.rows_bytes = (int)route_rows_bytes(D, a.cmax, sum_bytes(t));
   // Staged kernel when a query's widest level fits in shared memory.
@@ -390,6 +425,16 @@ DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam, bool al
     p.fused = true;
     return p;
   }
+  if (allow_warp && wide) {  // one CTA per query (route_group.cuh)
+    const int nw = group_warps(t, queries);
+    if (group_fits(t, (int)cmax, beam, nw, false)) {
+      p.group = true;
+      p.group_warps = nw;
+      p.fused = true;
+      p.append_ok = group_fits(t, (int)cmax, beam, nw, true);
+      return p;
+    }
+  }
   if (!wide) {
     p.nbuf = 2;
     p.rows_bytes = std::max(route_rows, (size_t)4 * 16 * row);  // two stages of 16 tokens at least
@@ -437,18 +482,25 @@ cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha
     ++t->launches;
     return e;
   }
+  const bool append = append_leaf >= 0;
+  if (append) {  // the tree already has its new shape
+    a.path_leaf = append_leaf;
+    a.path_tokens = (int)(std::min(append_leaf * a.lb + a.lb, t->N) - append_leaf * a.lb);
+    a.path_node[0] = append_leaf;
+    for (int l = 1; l <= t->L; ++l) a.path_node[l] = a.path_node[l - 1] / t->desc.branching;
+  }
+  if (p.group) {
+    const cudaError_t e = launch_route_group(t, a, p.group_warps, true, append, stream);
+    ++t->launches;
+    return e;
+  }
   a.stage_tokens = p.stage_tokens;
   a.attn_nbuf = p.nbuf;
   a.O = d_O;
   a.o_bf16 = o_dtype == ZHA_BF16;
   a.query_smem_bytes = (int)p.smem_per_query;  // weight area sized for 16 warps when wide
   StagedShape sh = staged_shape(t, a, p.smem_per_query, p.attn_warps);
-  const bool append = append_leaf >= 0;
-  if (append) {  // the tree already has its new shape; the path region follows the route's
-    a.path_leaf = append_leaf;
-    a.path_tokens = (int)(std::min(append_leaf * a.lb + a.lb, t->N) - append_leaf * a.lb);
-    a.path_smem_off = (long long)p.path_off;  // inside the row region, after the route's rows
-  }
+  if (append) a.path_smem_off = (long long)p.path_off;  // inside the row region, after the route's rows
   const cudaError_t e = staged_launch(t, true)(D, sh.grouped, !sh.wide, a, sh.blocks, sh.threads, sh.smem, stream,
                                                append ? kPathAppend : kPathNone);
   ++t->launches;

@@ -58,6 +58,11 @@ struct RouteArgs {
   long long buf_leaf0;
   int buf_tokens;
   long long first_wait;      // bound of a first wait for copies (kCopyWaitCycles unless testing)
+  // the route's first scored level over the whole tree (levels above it are kept whole) and
+  // the number of its parents, every node of the level above
+  int l_first, m_first;
+  // fused append: the path's node at each level 0 .. L (path_leaf, its parent, ...)
+  long long path_node[kMaxLevels];
 };
 
 struct NoKV {};  // route only: no attention epilogue
@@ -82,6 +87,18 @@ ZHA_ROUTE_LAUNCH_DECL(route_tma_launch_f32_s16);
 
 
 constexpr long long kRouteWaitCycles = kCopyWaitCycles;  // ~1 s at 1.9 GHz
+
+// CTA-per-query kernel (route_group.cuh) for launches with at most two queries per SM: one
+// CTA of nw (8 or 16) warps routes a query, every level's rows loaded straight into
+// registers by all its warps, and attends over its leaves the same way; optionally with the
+// one-leaf append path.  route_group_launch_* (route_group_{nokv,bf16,f32}.cu) launch it for
+// one K/V type (s16: bf16 summaries); smem is group_smem_layout's total.
+#define ZHA_GROUP_LAUNCH_DECL(name) \
+  cudaError_t name(int D, bool s16, int nw, bool append, const RouteArgs& a, size_t smem, cudaStream_t s)
+ZHA_GROUP_LAUNCH_DECL(route_group_launch_nokv);
+ZHA_GROUP_LAUNCH_DECL(route_group_launch_bf16);
+ZHA_GROUP_LAUNCH_DECL(route_group_launch_f32);
+#undef ZHA_GROUP_LAUNCH_DECL
 
 // Warp-per-query kernel (route_warp.cu) for launches with many queries: each warp routes one
 // query with its candidate rows loaded straight into registers and, when attending, reads

@@ -20,13 +20,11 @@
 // top-min(beam, C) over the packed (score, inverted node index) keys (select_warp).
 //
 // Attention (TKV = the K/V storage type): the query's warp reads its leaves' K and V rows
-// straight from global memory, LPT lanes per token (one 16-byte chunk each), PP token
-// passes per round with K and V of the round in flight together, and keeps an online
-// softmax in the log2 domain (warp-uniform running max, per-lane sums and output chunks
-// combined across token groups at the end).  K/V rows are read past L1.
+// straight from global memory and keeps an online softmax (attn_regs.cuh).
 #include <algorithm>
 #include <type_traits>
 
+#include "attn_regs.cuh"
 #include "device_common.cuh"
 #include "route_common.cuh"
 #include "zha_internal.h"
@@ -59,118 +57,23 @@ __host__ __device__ inline WarpSmem warp_smem_layout(int cmax, int beam) {
   return s;
 }
 
-// 16 bytes from global memory through the non-coherent path, not kept in L1 (K/V rows a
-// query reads once).
-__device__ __forceinline__ uint4 ldg16_na(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ float load_elem(const void* base, bool bf16, long long i) {
-  return bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(base)[i]) : static_cast<const float*>(base)[i];
-}
-
-// Exact softmax attention of query qg over the tokens of its m leaves (ascending; only the
-// last can be partial), by one warp.  Tokens go LPT lanes each (lane c = lane % LPT holds
-// 16-byte chunk c of the row), TPP = 32 / LPT tokens per pass, PP passes per round.
+// Exact softmax attention of query qg over the tokens of its m leaves by one warp
+// (attn_regs.cuh: every token in this warp's rounds, PP passes per round).
 template <typename TKV, int D, int PP>
 __device__ __forceinline__ void warp_attend(const int* leaves, int m, long long lb, long long N,
                                             const char* Ku, const char* Vu, const void* Q, bool q_bf16,
                                             long long qg, float qk_scale, void* O, bool o_bf16, int lane) {
-  constexpr int E = (int)sizeof(TKV);
-  constexpr int ROWB = D * E;
-  constexpr int VEC = 16 / E;
-  constexpr int LPT = ROWB / 16;
-  constexpr int TPP = 32 / LPT;
-  static_assert(LPT >= 1 && LPT <= 32 && 32 % LPT == 0, "row must split into 16-byte chunks over the warp");
-  const int c = lane % LPT, tg = lane / LPT;
-  float qc[VEC];
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) qc[e] = load_elem(Q, q_bf16, qg * D + c * VEC + e);
-  int total = 0;
-  if (m > 0) {
-    const long long last = leaves[m - 1];
-    total = (m - 1) * (int)lb + (int)(min(last * lb + lb, N) - last * lb);
-  }
+  using A = RegAttn<TKV, D>;
+  float qc[A::VEC];
+  reg_attn_load_q<TKV, D>(Q, q_bf16, qg, lane, qc);
+  const int total = leaf_token_count(leaves, m, lb, N);
   float m_w = -INFINITY, l_w = 0.f;
-  float acc[VEC];
+  float acc[A::VEC];
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-  for (int s0 = 0; s0 < total; s0 += TPP * PP) {
-    uint4 kv[PP], vv[PP];
-#pragma unroll
-    for (int p = 0; p < PP; ++p) {
-      const int s = s0 + p * TPP + tg;
-      if (s < total) {
-        const int j = s / (int)lb;
-        const long long tok = (long long)leaves[j] * lb + (s - j * (int)lb);
-        kv[p] = ldg16_na(Ku + tok * ROWB + c * 16);
-        vv[p] = ldg16_na(Vu + tok * ROWB + c * 16);
-      } else {
-        kv[p] = make_uint4(0u, 0u, 0u, 0u);
-        vv[p] = kv[p];
-      }
-    }
-    float sc[PP];
-    float mg = -INFINITY;
-#pragma unroll
-    for (int p = 0; p < PP; ++p) {
-      float f[VEC];
-      Vec16<TKV>::to_f32(kv[p], f);
-      float2 d01 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < VEC; e += 2)
-        d01 = __ffma2_rn(make_float2(qc[e], qc[e + 1]), make_float2(f[e], f[e + 1]), d01);
-      float d = d01.x + d01.y;
-#pragma unroll
-      for (int o = 1; o < LPT; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-      sc[p] = s0 + p * TPP + tg < total ? d * qk_scale : -INFINITY;
-      mg = fmaxf(mg, sc[p]);
-    }
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
-    const float m_new = fmaxf(m_w, mg);
-    const float alpha = m_w == -INFINITY ? 0.f : exp2f(m_w - m_new);
-    l_w *= alpha;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] *= alpha;
-#pragma unroll
-    for (int p = 0; p < PP; ++p) {
-      const float pr = sc[p] == -INFINITY ? 0.f : exp2f(sc[p] - m_new);
-      l_w += pr;
-      float f[VEC];
-      Vec16<TKV>::to_f32(vv[p], f);
-#pragma unroll
-      for (int e = 0; e < VEC; e += 2) {
-        const float2 r = __ffma2_rn(make_float2(pr, pr), make_float2(f[e], f[e + 1]), make_float2(acc[e], acc[e + 1]));
-        acc[e] = r.x;
-        acc[e + 1] = r.y;
-      }
-    }
-    m_w = m_new;
-  }
-  // every token group holds its own tokens' share of the sum and of each output chunk
-#pragma unroll
-  for (int o = LPT; o < 32; o <<= 1) {
-    l_w += __shfl_xor_sync(0xffffffffu, l_w, o);
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-  }
-  if (lane < LPT) {
-    const float inv = l_w > 0.f ? 1.f / l_w : 0.f;
-    if (o_bf16) {
-      uint16_t* o16 = static_cast<uint16_t*>(O) + qg * D + c * VEC;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) o16[e] = f32_to_bf16_bits(acc[e] * inv);
-    } else {
-      float* o32 = static_cast<float*>(O) + qg * D + c * VEC;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) o32[e] = acc[e] * inv;
-    }
-  }
+  for (int e = 0; e < A::VEC; ++e) acc[e] = 0.f;
+  reg_attn_tokens<TKV, D, PP>(leaves, total, lb, Ku, Vu, qc, qk_scale, 0, 1, lane, m_w, l_w, acc);
+  reg_attn_fold<TKV, D>(l_w, acc);
+  if (lane < A::LPT) store_out(O, o_bf16, qg, D, lane * A::VEC, acc, l_w > 0.f ? 1.f / l_w : 0.f);
 }
 
 // One warp per query, queries qg = blockIdx.x * W + warp, then every gridDim.x * W further.

@@ -95,6 +95,8 @@ cudaError_t launch_route(zha_tree* t, const void* d_Q, zha_dtype q_dtype, int q_
 struct DecodePlan {
   bool fused;
   bool warp;              // many queries: the warp-per-query kernel (route_warp.cu)
+  bool group;             // at most two queries per SM: the CTA-per-query kernel (route_group.cuh)
+  int group_warps;        // its warps per CTA (8 or 16)
   size_t rows_bytes;      // candidate-row / K-V stage region per query
   int stage_tokens;       // tokens per stage buffer
   int nbuf;               // stage buffers (2 or 3)
@@ -104,7 +106,8 @@ struct DecodePlan {
   size_t path_off, path_bytes;  // that append's region inside the row region
 };
 // allow_warp = false: the staged kernel's plan only (the causal and buffered calls run the
-// staged kernel whatever the launch shape).
+// staged kernel whatever the launch shape).  Otherwise many queries take the warp-per-query
+// kernel and few the CTA-per-query kernel, where their shared memory fits.
 DecodePlan plan_decode(const zha_tree* t, int q_heads, int nq, int beam, bool allow_warp = true);
 cudaError_t launch_decode(zha_tree* t, const DecodePlan& p, const void* d_Q, zha_dtype q_dtype,
                           int q_heads, int nq, int beam, const void* d_K, const void* d_V,
